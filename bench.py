@@ -1,0 +1,439 @@
+#!/usr/bin/env python
+"""Benchmark of the CSA2 decode hot path at a 1M-token context on B200.
+
+Workload (default): 1 Full + 1 Reindex layer, batch 4, 1,048,576-token
+context compressed 4:1 to N = 262,144 global entries per sequence, entry dim
+128 (FP4 E2M1 + fp32 per-16 scales), int8 indexer 4 heads x 64, top-k 2048,
+16 query heads, bf16 window 128.  Synthetic seeded inputs, resident in HBM.
+
+A step = one decode token per sequence through both layers: index scan,
+top-k, gather/dequant + attention.  L2 (126 MB) is flushed before every
+layer (a 256 MiB write kept outside the timed events), because the 64 MiB of
+index keys would otherwise stay L2-resident between the two layers that
+share them and between steps.
+
+Prints ONE JSON line (rank 0).  `value` = tokens/s/layer over all ranks
+(each rank is an independent replica: weak scaling).  `--impl reference`
+times the CPU oracle (test infrastructure) on the host cores instead.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from compressed_sparse_attention_topk_b200 import workloads as wl  # noqa: E402
+
+METRIC = "CSA2 decode tokens/s per layer at 1M ctx; achieved HBM GB/s vs B200 peak"
+UNIT = "tokens/s/layer"
+FALLBACK_HBM_GBS = 6650.0
+
+
+def parse_args():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=50)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", default="csa2", choices=["csa2", "reference"])
+    ap.add_argument("--workload", default=wl.LONG.name, choices=sorted(wl.ALL))
+    ap.add_argument("--cpu-seconds", type=float, default=12.0,
+                    help="CPU-baseline budget (oracle on the host cores)")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    return ap.parse_args()
+
+
+def algorithmic_bytes(w0) -> dict:
+    """Per (sequence, layer, token): index keys scanned + selected FP4 entries
+    gathered (codes + scales) + bf16 window K and V."""
+    keys = w0.N * w0.d_I
+    gather = w0.topk * (w0.D // 2 + w0.D // 4)
+    window = 2 * w0.W * w0.D * 2
+    return {"keys": keys, "gather": gather, "window": window, "total": keys + gather + window}
+
+
+def measured_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        d = json.load(open(p))
+        return float(d["hbm_gbs"]), "measured"
+    return FALLBACK_HBM_GBS, "fallback"
+
+
+def scan_source_sha() -> str:
+    h = hashlib.sha256()
+    for f in ("index_scan.cuh", "common.cuh"):
+        h.update(open(os.path.join(ROOT, "compressed_sparse_attention_topk_b200", "csrc", f),
+                      "rb").read())
+    return h.hexdigest()[:16]
+
+
+def ncu_traffic():
+    """DRAM bytes per index-scan launch from a committed ncu summary, only
+    while the kernel source is unchanged since the capture."""
+    p = os.path.join(ROOT, "profiles", "index_scan_traffic.json")
+    if not os.path.exists(p):
+        return None
+    d = json.load(open(p))
+    if d.get("source_sha") != scan_source_sha():
+        return None
+    return d.get("dram_bytes_per_launch_full_size")
+
+
+# --------------------------------------------------------------------------- clocks
+
+class ClockSampler:
+    FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_id: str):
+        self.gpu_id = gpu_id
+        self.proc = None
+        self.lines = []
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", self.gpu_id, f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "200"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.thread = threading.Thread(target=self._read, daemon=True)
+            self.thread.start()
+        except (OSError, FileNotFoundError):
+            self.proc = None
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def stop(self) -> dict:
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        time.sleep(0.3)
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        sm, smax, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in self.lines:
+            parts = [p.strip() for p in ln.split(",")]
+            if len(parts) < 8:
+                continue
+            try:
+                sm.append(float(parts[0]))
+                smax.append(float(parts[1]))
+            except ValueError:
+                continue
+            for nm, v in zip(names, parts[4:8]):
+                if v.lower() == "active":
+                    reasons.add(nm)
+        if not sm:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples"]}
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(smax),
+                "samples": len(sm), "reasons": sorted(reasons)}
+
+
+# --------------------------------------------------------------------------- oracle timing
+
+def oracle_sample(w0, seconds: float, min_runs: int = 1):
+    """Time the CPU oracle on whole sequences (all layers of the workload),
+    one sequence at a time, until `seconds` have passed."""
+    import oracle
+    layers = wl.all_layer_inputs(w0, B=1)
+    for lay in layers:
+        if "entries" in lay:
+            B, N, D = lay["entries"].shape
+            c, s = oracle.pack_fp4(lay["entries"].reshape(B * N, D))
+            lay["codes"], lay["scales"] = c.reshape(B, N, D // 2), s.reshape(B, N, D // 16)
+    runs, t0 = 0, time.perf_counter()
+    while runs < min_runs or time.perf_counter() - t0 < seconds:
+        oracle.layer_group(list(w0.modes), layers, w0.topk, w0.n_prior, w0.ratio)
+        runs += 1
+    dt = time.perf_counter() - t0
+    return runs, dt
+
+
+def run_reference(args, w0):
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return 0
+    import oracle
+    layers = wl.all_layer_inputs(w0, B=1)
+    for lay in layers:
+        if "entries" in lay:
+            B, N, D = lay["entries"].shape
+            c, s = oracle.pack_fp4(lay["entries"].reshape(B * N, D))
+            lay["codes"], lay["scales"] = c.reshape(B, N, D // 2), s.reshape(B, N, D // 16)
+
+    def step():
+        oracle.layer_group(list(w0.modes), layers, w0.topk, w0.n_prior, w0.ratio)
+
+    for _ in range(args.warmup):
+        step()
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        step()
+    dt = time.perf_counter() - t0
+    tokens_layers = args.steps * 1 * w0.T * w0.L
+    value = tokens_layers / dt
+    sample = (f"1 of {w0.B} sequences per step ({w0.L} layers, N={w0.N}), "
+              f"plain C oracle, single thread")
+    line = {
+        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": dt / args.steps * 1e3,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "int8/f64",
+        "data": "synthetic", "impl": "reference",
+        "config": {"workload": w0.name, "B": w0.B, "N": w0.N, "layers": w0.L,
+                   "topk": w0.topk, "parallelism": "host cores, rank 0 only"},
+        "cpu_baseline": {"value": value, "unit": UNIT, "cores": 1, "kind": "oracle",
+                         "sample": sample},
+        "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+# --------------------------------------------------------------------------- GPU arm
+
+def run_gpu(args, w0):
+    import torch
+    import compressed_sparse_attention_topk_b200 as csa2
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    dist = None
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=180),
+                                device_id=torch.device("cuda", local))
+    else:
+        torch.cuda.set_device(0)
+    dev = torch.device("cuda", torch.cuda.current_device())
+    csa2.lib()
+    stream = torch.cuda.current_stream()
+
+    def to_dev(a):
+        a = np.ascontiguousarray(a)
+        if a.dtype == np.uint16:
+            return torch.from_numpy(a.view(np.int16)).to(dev).view(torch.bfloat16)
+        return torch.from_numpy(a).to(dev)
+
+    # ---- inputs resident in HBM (replica per rank, same seeded data) ----
+    host_layers = wl.all_layer_inputs(w0)
+    tens = []
+    for lay in host_layers:
+        d = {}
+        for k in ("q", "q_idx", "w", "win_k", "win_v"):
+            d[k] = to_dev(lay[k])
+        d["q"] = d["q"][:, 0].contiguous()              # decode: [B, H, D]
+        if "entries" in lay:
+            src = to_dev(lay["entries"])
+            d["codes"], d["scales"] = csa2.pack_fp4(src)
+            del src
+            d["k_idx"] = to_dev(lay["k_idx"])
+        d["idx"] = torch.empty((w0.B, 1, w0.topk), dtype=torch.int32, device=dev)
+        d["out"] = torch.empty((w0.B, w0.H, w0.D), dtype=torch.float32, device=dev)
+        d["lse"] = torch.empty((w0.B, w0.H), dtype=torch.float32, device=dev)
+        tens.append(d)
+    torch.cuda.synchronize()
+    ws = csa2.workspace(max(
+        csa2.index_topk_workspace_size(w0.B, 1, w0.H_I, w0.d_I, w0.N, w0.topk),
+        csa2.sparse_attn_workspace_size(w0.B, 1, w0.H, w0.D, w0.topk, w0.W)))
+    flush_buf = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+
+    def flush():
+        flush_buf.fill_(1)
+
+    def layer(l):
+        mode, kv, ix = w0.modes[l]
+        x, st, src = tens[l], tens[kv], tens[ix]
+        if mode != wl.REUSE:
+            csa2.index_topk(x["q_idx"], x["w"], st["k_idx"], w0.topk, idx_out=x["idx"], ws=ws)
+        csa2.sparse_attn_decode(x["q"], st["codes"], st["scales"], src["idx"][:, 0], x["win_k"],
+                                x["win_v"], w0.sm_scale, out=x["out"], lse=x["lse"], ws=ws)
+
+    ev = lambda: torch.cuda.Event(enable_timing=True)  # noqa: E731
+
+    def timed_steps(K, trace=False):
+        """K steps; returns per-step device ms (sum of per-layer events)."""
+        pairs = []
+        for _ in range(K):
+            step_pairs = []
+            for l in range(w0.L):
+                flush()
+                a, b = ev(), ev()
+                a.record(stream)
+                layer(l)
+                b.record(stream)
+                step_pairs.append((a, b))
+            pairs.append(step_pairs)
+        torch.cuda.synchronize()
+        return [sum(a.elapsed_time(b) for a, b in sp) for sp in pairs]
+
+    # ---- warm-up ----
+    timed_steps(max(args.warmup, 3))
+
+    gpu_uuid = str(torch.cuda.get_device_properties(dev).uuid)
+    gpu_id = gpu_uuid if gpu_uuid.startswith("GPU-") else f"GPU-{gpu_uuid}"
+    clocks = ClockSampler(gpu_id)
+    clocks.start()
+    time.sleep(0.4)
+
+    # ---- timed region: K steps ----
+    if dist:
+        dist.barrier()
+    torch.cuda.synchronize()
+    w_t0 = time.perf_counter()
+    step_ms = timed_steps(args.steps)
+    torch.cuda.synchronize()
+    wall_s = time.perf_counter() - w_t0
+    total_ms = float(sum(step_ms))
+    if dist:
+        t = torch.tensor([total_ms], dtype=torch.float64, device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        total_ms = float(t.item())
+        dist.barrier()
+
+    # ---- per-kernel device times (trace on; second timed pass) ----
+    csa2.trace_enable(True)
+    timed_steps(args.steps)
+    recs = csa2.trace_records()
+    csa2.trace_enable(False)
+    per_kernel = {}
+    for name, ms in recs:
+        c, s = per_kernel.get(name, (0, 0.0))
+        per_kernel[name] = (c + 1, s + ms)
+    launches_per_step = len(recs) / args.steps
+
+    # ---- e2e: pinned host inputs -> device, hot path, results -> host ----
+    in_keys = ("q", "q_idx", "w", "win_k", "win_v")
+    out_keys = ("out", "lse", "idx")
+    host_in = [{k: tens[l][k].cpu().pin_memory() for k in in_keys} for l in range(w0.L)]
+    host_out = [{k: torch.empty_like(tens[l][k], device="cpu").pin_memory() for k in out_keys}
+                for l in range(w0.L)]
+    h2d = sum(t.numel() * t.element_size() for d in host_in for t in d.values())
+    d2h = sum(t.numel() * t.element_size() for d in host_out for t in d.values())
+
+    def e2e_steps(K):
+        res = []
+        for _ in range(K):
+            flush()
+            a, b = ev(), ev()
+            a.record(stream)
+            for l in range(w0.L):
+                for k in in_keys:
+                    tens[l][k].copy_(host_in[l][k], non_blocking=True)
+            b.record(stream)
+            segs = [(a, b)]
+            for l in range(w0.L):
+                if l > 0:
+                    flush()
+                a, b = ev(), ev()
+                a.record(stream)
+                layer(l)
+                if l == w0.L - 1:
+                    for ll in range(w0.L):
+                        for k in out_keys:
+                            host_out[ll][k].copy_(tens[ll][k], non_blocking=True)
+                b.record(stream)
+                segs.append((a, b))
+            res.append(segs)
+        torch.cuda.synchronize()
+        return [sum(a.elapsed_time(b) for a, b in s) for s in res]
+
+    e2e_steps(3)
+    e2e_ms = float(sum(e2e_steps(args.steps)))
+    if dist:
+        t = torch.tensor([e2e_ms], dtype=torch.float64, device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        e2e_ms = float(t.item())
+    clk = clocks.stop()
+
+    status = csa2.get_device_status()
+    if status:
+        raise RuntimeError(f"device status word set: {status}")
+
+    tokens_layers = world * args.steps * w0.B * w0.T * w0.L
+    value = tokens_layers / (total_ms * 1e-3)
+    e2e_value = tokens_layers / (e2e_ms * 1e-3)
+
+    ab = algorithmic_bytes(w0)
+    peak, peak_kind = measured_peaks()
+    scan_n, scan_ms = per_kernel.get("index_scan", (0, 0.0))
+    scan_launch_bytes = w0.B * ab["keys"]
+    scan_avg_ms = scan_ms / max(scan_n, 1)
+    achieved = scan_launch_bytes / (scan_avg_ms * 1e-3) / 1e9 if scan_n else None
+    step_bytes = w0.B * w0.L * ab["total"]
+    step_gbs = step_bytes / (total_ms / args.steps * 1e-3) / 1e9
+
+    line = None
+    if rank == 0:
+        cpu = None
+        if world == 1 and not args.no_cpu_baseline:
+            runs, dt = oracle_sample(w0, args.cpu_seconds)
+            cpu = {"value": runs * w0.T * w0.L / dt, "unit": UNIT, "cores": 1, "kind": "oracle",
+                   "sample": f"{runs} sequence(s) x {w0.L} layers of the same workload "
+                             f"(N={w0.N}), plain C oracle, single thread, {dt:.1f} s"}
+        line = {
+            "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": total_ms / args.steps, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "int8", "data": "synthetic",
+            "config": {"workload": w0.name, "B": w0.B, "N": w0.N, "context_tokens": w0.N * 4,
+                       "layers": "Full+Reindex" if w0.L == 2 else w0.L, "topk": w0.topk,
+                       "H": w0.H, "D": w0.D, "H_I": w0.H_I, "d_I": w0.d_I, "W": w0.W,
+                       "parallelism": f"replicas x{world}",
+                       "l2": "flushed (256 MiB write) before every layer, flush not timed",
+                       "step_algorithmic_bytes": step_bytes,
+                       "step_hbm_gbs": step_gbs, "step_hbm_frac": step_gbs / peak,
+                       "wall_s_timed_region": wall_s},
+            "roofline": {"bound": "hbm", "kernel": "index_scan", "achieved": achieved,
+                         "peak": peak, "peak_kind": f"{peak_kind} (copy bandwidth)",
+                         "unit": "GB/s", "frac": (achieved / peak) if achieved else None,
+                         "traffic": ncu_traffic(),
+                         "bytes_per_launch": scan_launch_bytes,
+                         "avg_launch_ms": scan_avg_ms},
+            "kernels": {k: {"launches": c, "avg_us": s / c * 1e3, "share": s / sum(
+                v[1] for v in per_kernel.values())} for k, (c, s) in sorted(per_kernel.items())},
+            "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": h2d,
+                    "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms / args.steps},
+            "gpu_launches": int(round(launches_per_step * args.steps)),
+            "clocks": clk,
+            "cpu_baseline": cpu,
+        }
+    if dist:
+        dist.barrier()
+        dist.destroy_process_group()
+    if line is not None:
+        print(json.dumps(line), flush=True)
+    return 0
+
+
+def main():
+    args = parse_args()
+    w0 = wl.ALL[args.workload]
+    if w0.T != 1 or w0.n_prior >= 0:
+        raise SystemExit("bench.py times decode workloads (T == 1)")
+    if args.impl == "reference":
+        return run_reference(args, w0)
+    return run_gpu(args, w0)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -1,0 +1,349 @@
+"""CSA2 hot path on B200: a thin ctypes binding over libcsa2.so.
+
+Every function here only marshals arguments (torch tensors -> device
+pointers, sizes, the current CUDA stream) and calls the C ABI declared in
+``include/csa2.h``; all computation runs in the library's sm_100a kernels.
+There is no CPU fallback: if the library is missing or a tensor is not on
+a CUDA device, the call raises.
+
+Functions mirror the C entry points: ``pack_fp4``, ``unpack_fp4``,
+``index_topk``, ``sparse_attn_decode``, ``sparse_attn_prefill``,
+``layer_group_run``, plus ``validate_modes``, ``group_cache_bytes`` and
+``get_device_status``.
+"""
+from __future__ import annotations
+
+import ctypes
+import math
+import os
+from typing import Dict, List, Optional, Sequence, Tuple
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_PKG, "libcsa2.so")
+
+CSA2_OK, CSA2_ERR_INVALID_ARG, CSA2_ERR_UNSUPPORTED, CSA2_ERR_CUDA = 0, 1, 2, 3
+CSA2_ERR_WORKSPACE, CSA2_ERR_DEVICE_STATUS = 4, 5
+FULL, REINDEX, REUSE = 0, 1, 2
+
+EXPORTED = (
+    "csa2_status_string", "csa2_version", "csa2_pack_fp4", "csa2_unpack_fp4",
+    "csa2_index_topk_workspace_size", "csa2_index_topk", "csa2_sparse_attn_workspace_size",
+    "csa2_sparse_attn_decode", "csa2_sparse_attn_prefill", "csa2_validate_modes",
+    "csa2_group_cache_bytes", "csa2_layer_group_workspace_size", "csa2_layer_group_run",
+    "csa2_get_device_status", "csa2_trace_enable", "csa2_trace_count", "csa2_trace_get",
+)
+
+
+class CSA2Error(RuntimeError):
+    def __init__(self, status: int, what: str):
+        self.status = status
+        super().__init__(f"{what}: {lib().csa2_status_string(status).decode()}")
+
+
+class LayerMode(ctypes.Structure):
+    _fields_ = [("mode", ctypes.c_int32), ("kv_src", ctypes.c_int32), ("idx_src", ctypes.c_int32)]
+
+
+class Dims(ctypes.Structure):
+    _fields_ = [("B", ctypes.c_int32), ("T", ctypes.c_int32), ("H", ctypes.c_int32),
+                ("D", ctypes.c_int32), ("N", ctypes.c_int64), ("H_I", ctypes.c_int32),
+                ("d_I", ctypes.c_int32), ("topk", ctypes.c_int32), ("W", ctypes.c_int32),
+                ("n_prior", ctypes.c_int64), ("ratio", ctypes.c_int32),
+                ("sm_scale", ctypes.c_float)]
+
+
+class LayerIO(ctypes.Structure):
+    _fields_ = [(n, ctypes.c_void_p) for n in (
+        "q", "q_idx", "w", "win_k", "win_v", "codes", "scales", "k_idx", "idx", "out", "lse")]
+
+
+_lib = None
+
+
+def lib() -> ctypes.CDLL:
+    """Load libcsa2.so (raises if it has not been built)."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    if not os.path.exists(LIB_PATH):
+        raise ImportError(f"{LIB_PATH} is missing: build it with "
+                          "`python -m compressed_sparse_attention_topk_b200.build`")
+    L = ctypes.CDLL(LIB_PATH)
+    P, i32, i64, f32, sz = (ctypes.c_void_p, ctypes.c_int32, ctypes.c_int64, ctypes.c_float,
+                            ctypes.c_size_t)
+    sig = {
+        "csa2_status_string": ([i32], ctypes.c_char_p),
+        "csa2_version": ([], i32),
+        "csa2_pack_fp4": ([P, i64, i32, P, P, P], i32),
+        "csa2_unpack_fp4": ([P, P, i64, i32, P, P], i32),
+        "csa2_index_topk_workspace_size": ([i32, i32, i32, i32, i64, i32], sz),
+        "csa2_index_topk": ([P, P, P, i32, i32, i32, i32, i64, i64, i32, i32, P, P, P, sz, P], i32),
+        "csa2_sparse_attn_workspace_size": ([i32, i32, i32, i32, i32, i32], sz),
+        "csa2_sparse_attn_decode": ([P, P, P, P, P, P, i32, i32, i32, i64, i32, i32, f32, P, P, P,
+                                     sz, P], i32),
+        "csa2_sparse_attn_prefill": ([P, P, P, P, P, P, i32, i32, i32, i32, i64, i32, i32, f32, P,
+                                      P, P, sz, P], i32),
+        "csa2_validate_modes": ([P, i32], i32),
+        "csa2_group_cache_bytes": ([P, i32, i64, i64, i64, P], i32),
+        "csa2_layer_group_workspace_size": ([P], sz),
+        "csa2_layer_group_run": ([P, P, i32, P, P, sz, P], i32),
+        "csa2_get_device_status": ([P, P], i32),
+        "csa2_trace_enable": ([i32], i32),
+        "csa2_trace_count": ([], i32),
+        "csa2_trace_get": ([i32, ctypes.POINTER(ctypes.c_char_p), ctypes.POINTER(f32)], i32),
+    }
+    for name, (args, res) in sig.items():
+        fn = getattr(L, name)
+        fn.argtypes = args
+        fn.restype = res
+    _lib = L
+    return L
+
+
+def _check(rc: int, what: str):
+    if rc != CSA2_OK:
+        raise CSA2Error(rc, what)
+
+
+# --- torch marshalling --------------------------------------------------------
+
+def _torch():
+    import torch
+    return torch
+
+
+def _dev(t, name, dtype=None):
+    torch = _torch()
+    if t is None:
+        return None
+    if not isinstance(t, torch.Tensor) or not t.is_cuda:
+        raise TypeError(f"{name} must be a CUDA tensor")
+    if dtype is not None and t.dtype != dtype:
+        raise TypeError(f"{name} must be {dtype}, got {t.dtype}")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    return t
+
+
+def _ptr(t) -> Optional[int]:
+    return None if t is None else t.data_ptr()
+
+
+def _stream(device=None) -> int:
+    return _torch().cuda.current_stream(device).cuda_stream
+
+
+_ws_cache: Dict[int, object] = {}
+
+
+def workspace(nbytes: int, device=None):
+    """A cached uint8 device buffer of at least nbytes (grown on demand)."""
+    torch = _torch()
+    dev = torch.device("cuda", torch.cuda.current_device()) if device is None else device
+    key = dev.index if dev.index is not None else torch.cuda.current_device()
+    buf = _ws_cache.get(key)
+    if buf is None or buf.numel() < max(nbytes, 1):
+        buf = torch.empty(max(nbytes, 256), dtype=torch.uint8, device=dev)
+        _ws_cache[key] = buf
+    return buf
+
+
+# --- FP4 ----------------------------------------------------------------------
+
+def pack_fp4(src, codes=None, scales=None) -> Tuple[object, object]:
+    """fp32 [..., D] -> (uint8 [..., D/2] codes, fp32 [..., D/16] scales)."""
+    torch = _torch()
+    src = _dev(src, "src", torch.float32)
+    D = src.shape[-1]
+    rows = src.numel() // D if D else 0
+    if codes is None:
+        codes = torch.empty(src.shape[:-1] + (D // 2,), dtype=torch.uint8, device=src.device)
+    if scales is None:
+        scales = torch.empty(src.shape[:-1] + (D // 16,), dtype=torch.float32, device=src.device)
+    _check(lib().csa2_pack_fp4(_ptr(src), rows, D, _ptr(codes), _ptr(scales), _stream()),
+           "csa2_pack_fp4")
+    return codes, scales
+
+
+def unpack_fp4(codes, scales, D: int, out=None):
+    torch = _torch()
+    codes = _dev(codes, "codes", torch.uint8)
+    scales = _dev(scales, "scales", torch.float32)
+    rows = codes.numel() // (D // 2)
+    if out is None:
+        out = torch.empty(codes.shape[:-1] + (D,), dtype=torch.float32, device=codes.device)
+    _check(lib().csa2_unpack_fp4(_ptr(codes), _ptr(scales), rows, D, _ptr(out), _stream()),
+           "csa2_unpack_fp4")
+    return out
+
+
+# --- indexer + top-k ----------------------------------------------------------
+
+def index_topk_workspace_size(B, T, H_I, d_I, N, topk) -> int:
+    return int(lib().csa2_index_topk_workspace_size(B, T, H_I, d_I, N, topk))
+
+
+def index_topk(q_idx, w, k_idx, topk: int, n_prior: int = -1, ratio: int = 4, idx_out=None,
+               want_scores: bool = False, ws=None):
+    """q_idx int8 [B,T,H_I,d_I], w fp32 [B,T,H_I], k_idx int8 [B,N,d_I] ->
+    idx int32 [B,T,topk] (and fp32 scores [B,T,N] when want_scores)."""
+    torch = _torch()
+    q_idx = _dev(q_idx, "q_idx", torch.int8)
+    w = _dev(w, "w", torch.float32)
+    k_idx = _dev(k_idx, "k_idx", torch.int8)
+    B, T, H_I, d_I = q_idx.shape
+    N = k_idx.shape[1]
+    if idx_out is None:
+        idx_out = torch.empty((B, T, topk), dtype=torch.int32, device=q_idx.device)
+    scores = (torch.empty((B, T, N), dtype=torch.float32, device=q_idx.device)
+              if want_scores else None)
+    need = index_topk_workspace_size(B, T, H_I, d_I, N, topk)
+    if ws is None:
+        ws = workspace(need)
+    _check(lib().csa2_index_topk(_ptr(q_idx), _ptr(w), _ptr(k_idx), B, T, H_I, d_I, N, n_prior,
+                                 ratio, topk, _ptr(idx_out), _ptr(scores), _ptr(ws), ws.numel(),
+                                 _stream()), "csa2_index_topk")
+    return (idx_out, scores) if want_scores else idx_out
+
+
+# --- attention ----------------------------------------------------------------
+
+def sparse_attn_workspace_size(B, T, H, D, topk, W) -> int:
+    return int(lib().csa2_sparse_attn_workspace_size(B, T, H, D, topk, W))
+
+
+def _attn_common(q, codes, scales, idx, win_k, win_v):
+    torch = _torch()
+    q = _dev(q, "q", torch.bfloat16)
+    codes = _dev(codes, "codes", torch.uint8)
+    scales = _dev(scales, "scales", torch.float32)
+    idx = _dev(idx, "idx", torch.int32)
+    win_k = _dev(win_k, "win_k", torch.bfloat16)
+    win_v = _dev(win_v, "win_v", torch.bfloat16)
+    return q, codes, scales, idx, win_k, win_v
+
+
+def sparse_attn_decode(q, codes, scales, idx, win_k, win_v, sm_scale: Optional[float] = None,
+                       out=None, lse=None, ws=None):
+    """q bf16 [B,H,D]; codes u8 [B,N,D/2]; scales fp32 [B,N,D/16]; idx int32
+    [B,topk]; win_k/win_v bf16 [B,W,D] (or None) -> (out fp32 [B,H,D], lse fp32 [B,H])."""
+    torch = _torch()
+    q, codes, scales, idx, win_k, win_v = _attn_common(q, codes, scales, idx, win_k, win_v)
+    B, H, D = q.shape
+    N = codes.shape[1]
+    topk = idx.shape[-1]
+    W = 0 if win_k is None else win_k.shape[1]
+    sm_scale = 1.0 / math.sqrt(D) if sm_scale is None else sm_scale
+    if out is None:
+        out = torch.empty((B, H, D), dtype=torch.float32, device=q.device)
+    if lse is None:
+        lse = torch.empty((B, H), dtype=torch.float32, device=q.device)
+    need = sparse_attn_workspace_size(B, 1, H, D, topk, W)
+    if ws is None:
+        ws = workspace(need)
+    _check(lib().csa2_sparse_attn_decode(_ptr(q), _ptr(codes), _ptr(scales), _ptr(idx),
+                                         _ptr(win_k), _ptr(win_v), B, H, D, N, topk, W,
+                                         sm_scale, _ptr(out), _ptr(lse), _ptr(ws), ws.numel(),
+                                         _stream()), "csa2_sparse_attn_decode")
+    return out, lse
+
+
+def sparse_attn_prefill(q, codes, scales, idx, win_k, win_v, sm_scale: Optional[float] = None,
+                        out=None, lse=None, ws=None):
+    """q bf16 [B,T,H,D]; idx int32 [B,T,topk]; win_k/win_v bf16 [B,W-1+T,D]
+    -> (out fp32 [B,T,H,D], lse fp32 [B,T,H])."""
+    torch = _torch()
+    q, codes, scales, idx, win_k, win_v = _attn_common(q, codes, scales, idx, win_k, win_v)
+    B, T, H, D = q.shape
+    N = codes.shape[1]
+    topk = idx.shape[-1]
+    W = 0 if win_k is None else win_k.shape[1] - T + 1
+    sm_scale = 1.0 / math.sqrt(D) if sm_scale is None else sm_scale
+    if out is None:
+        out = torch.empty((B, T, H, D), dtype=torch.float32, device=q.device)
+    if lse is None:
+        lse = torch.empty((B, T, H), dtype=torch.float32, device=q.device)
+    need = sparse_attn_workspace_size(B, T, H, D, topk, W)
+    if ws is None:
+        ws = workspace(need)
+    _check(lib().csa2_sparse_attn_prefill(_ptr(q), _ptr(codes), _ptr(scales), _ptr(idx),
+                                          _ptr(win_k), _ptr(win_v), B, T, H, D, N, topk, W,
+                                          sm_scale, _ptr(out), _ptr(lse), _ptr(ws), ws.numel(),
+                                          _stream()), "csa2_sparse_attn_prefill")
+    return out, lse
+
+
+# --- cross-layer groups ---------------------------------------------------------
+
+def _modes_array(modes: Sequence[Tuple[int, int, int]]):
+    arr = (LayerMode * len(modes))()
+    for i, (m, kv, ix) in enumerate(modes):
+        arr[i].mode, arr[i].kv_src, arr[i].idx_src = m, kv, ix
+    return arr
+
+
+def validate_modes(modes) -> bool:
+    arr = _modes_array(modes)
+    return lib().csa2_validate_modes(arr, len(modes)) == CSA2_OK
+
+
+def group_cache_bytes(modes, entries: int, numbers_per_entry: int, bits_per_number: int) -> int:
+    arr = _modes_array(modes)
+    out = ctypes.c_uint64(0)
+    _check(lib().csa2_group_cache_bytes(arr, len(modes), entries, numbers_per_entry,
+                                        bits_per_number, ctypes.byref(out)),
+           "csa2_group_cache_bytes")
+    return int(out.value)
+
+
+def make_dims(B, T, H, D, N, H_I, d_I, topk, W, n_prior=-1, ratio=4, sm_scale=None) -> Dims:
+    return Dims(B, T, H, D, N, H_I, d_I, topk, W, n_prior, ratio,
+                1.0 / math.sqrt(D) if sm_scale is None else sm_scale)
+
+
+def layer_group_workspace_size(dims: Dims) -> int:
+    return int(lib().csa2_layer_group_workspace_size(ctypes.byref(dims)))
+
+
+def layer_group_run(modes, layers: List[dict], dims: Dims, ws=None):
+    """Run a mode table.  ``layers[l]`` holds the layer's device tensors
+    (q, q_idx, w, win_k, win_v, idx, out, lse and, for Full layers, codes,
+    scales, k_idx)."""
+    arr = _modes_array(modes)
+    io = (LayerIO * len(layers))()
+    for i, lay in enumerate(layers):
+        for name, _ in LayerIO._fields_:
+            t = lay.get(name)
+            if t is not None:
+                _dev(t, f"layers[{i}].{name}")
+            setattr(io[i], name, _ptr(t))
+    need = layer_group_workspace_size(dims)
+    if ws is None:
+        ws = workspace(need)
+    _check(lib().csa2_layer_group_run(arr, io, len(layers), ctypes.byref(dims), _ptr(ws),
+                                      ws.numel(), _stream()), "csa2_layer_group_run")
+
+
+def get_device_status() -> int:
+    code = ctypes.c_int32(0)
+    rc = lib().csa2_get_device_status(_stream(), ctypes.byref(code))
+    if rc not in (CSA2_OK, CSA2_ERR_DEVICE_STATUS):
+        raise CSA2Error(rc, "csa2_get_device_status")
+    return int(code.value)
+
+
+# --- kernel timing trace -----------------------------------------------------------
+
+def trace_enable(on: bool = True):
+    _check(lib().csa2_trace_enable(1 if on else 0), "csa2_trace_enable")
+
+
+def trace_records() -> List[Tuple[str, float]]:
+    """(kernel name, device ms) of every launch recorded since trace_enable."""
+    out = []
+    name = ctypes.c_char_p()
+    ms = ctypes.c_float()
+    for i in range(lib().csa2_trace_count()):
+        _check(lib().csa2_trace_get(i, ctypes.byref(name), ctypes.byref(ms)), "csa2_trace_get")
+        out.append((name.value.decode(), float(ms.value)))
+    return out

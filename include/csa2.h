@@ -1,0 +1,284 @@
+/*
+ * csa2.h -- C ABI of the CSA2 (Compressed Sparse Attention 2) hot path for
+ * NVIDIA B200 (sm_100a).  Library: libcsa2.so.
+ *
+ * What the path computes, per layer and query token (sources are web pages
+ * on DeepSeek-V4.1-Flash, cited by title and section):
+ *   1. an indexer scores every visible compressed global cache entry
+ *      ("Why Is DeepSeek V4.1 Flash So Fast?", section 4, "The indexer");
+ *   2. the Top-K best entries are kept (same page, sections 3-4);
+ *   3. the kept entries, stored as FP4 with per-group scaling ("DeepSeek-
+ *      V4.1-Flash" visual explainer, section "Fast memory, persistent
+ *      storage and recomputation"; "Inference-Efficient LLMs", section 6),
+ *      are gathered and dequantised;
+ *   4. softmax attention runs over them together with the layer's own
+ *      128-token sliding window kept at higher precision (bf16)
+ *      ("Why Is DeepSeek V4.1 Flash So Fast?", section 3; "Inference-
+ *      Efficient LLMs", sections 3 and 6);
+ *   5. layers run in Full, Reindex or Reuse mode ("DeepSeek-V4.1-Flash",
+ *      section "Sharing the cache across layers"; "Why Is DeepSeek V4.1
+ *      Flash So Fast?", section 5).
+ *
+ * The pages fix no formula, size or format detail for any step; the
+ * readings this library takes are stated at each call below.
+ *
+ * Conventions for every call:
+ *  - Pointers named as device pointers must point to device (or managed)
+ *    memory of the current CUDA device; host pointers are named as such.
+ *    All arrays are dense, row-major, and device arrays are 16-byte
+ *    aligned.  The caller owns every buffer; the library allocates no
+ *    device memory.  Scratch ("workspace") is passed in by the caller; its
+ *    size comes from the matching *_workspace_size query.
+ *  - `stream` is a cudaStream_t (NULL = the legacy default stream).  Every
+ *    call only enqueues work on `stream` and returns; nothing synchronises
+ *    except csa2_get_device_status.
+ *  - bf16 arrays are passed as uint16_t bit patterns.
+ *  - Errors are returned, never raised: arguments are validated on the
+ *    host before anything is enqueued, and an invalid call enqueues
+ *    nothing.  CSA2_ERR_CUDA means a launch failed; the CUDA error is then
+ *    also left for cudaGetLastError.  Indices that point outside the entry
+ *    store are skipped on the device and recorded in a device status word
+ *    that csa2_get_device_status reports.
+ */
+#ifndef CSA2_H
+#define CSA2_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum csa2_status {
+    CSA2_OK = 0,
+    CSA2_ERR_INVALID_ARG = 1,   /* null pointer, bad size, misaligned pointer, bad mode table */
+    CSA2_ERR_UNSUPPORTED = 2,   /* valid request outside the compiled shape set */
+    CSA2_ERR_CUDA = 3,          /* a CUDA launch or query failed */
+    CSA2_ERR_WORKSPACE = 4,     /* workspace missing or smaller than the query says */
+    CSA2_ERR_DEVICE_STATUS = 5  /* a kernel recorded a bad index (see csa2_get_device_status) */
+} csa2_status;
+
+/* Layer modes ("DeepSeek-V4.1-Flash", section "Sharing the cache across
+ * layers"): Full computes its own entries and its own selection; Reindex
+ * shares another layer's entries and makes a fresh selection; Reuse shares
+ * both.  Every layer keeps its own queries and its own local window. */
+typedef enum csa2_mode { CSA2_FULL = 0, CSA2_REINDEX = 1, CSA2_REUSE = 2 } csa2_mode;
+
+/* One row of the per-layer mode table.  kv_src: the layer whose entry store
+ * (FP4 codes, scales, int8 index keys) this layer reads; idx_src: the layer
+ * whose selection it uses.  Valid tables: Full names itself twice; Reindex
+ * names an earlier Full layer as kv_src and itself as idx_src; Reuse names
+ * an earlier Full or Reindex layer as idx_src and that layer's kv_src as
+ * its own kv_src. */
+typedef struct csa2_layer_mode {
+    int32_t mode;
+    int32_t kv_src;
+    int32_t idx_src;
+} csa2_layer_mode;
+
+/* Human-readable name of a status code (static string, never NULL). */
+const char *csa2_status_string(int32_t status);
+
+/* Library ABI version (major * 10000 + minor * 100 + patch). */
+int32_t csa2_version(void);
+
+/* ---------------------------------------------------------------------- */
+/* FP4 entry store                                                         */
+/* ---------------------------------------------------------------------- */
+
+/* Pack fp32 entries into FP4 E2M1 codes with one fp32 scale per 16
+ * consecutive elements ("FP4 representation with per-group scaling":
+ * "Inference-Efficient LLMs", section 6; the E2M1 element format and the
+ * group of 16 are this library's reading).  Per group: s = amax / 6 (IEEE
+ * fp32 divide, amax = largest |x|); each element's code is the E2M1 value
+ * nearest to x / s (fp32 divide), ties to the even code, saturating at 6;
+ * a zero magnitude is stored as code 0 (never negative zero); a group with
+ * s == 0 stores all-zero codes.  Element 2i goes in the low nibble of byte i.
+ *   src    device, fp32 [rows, D], finite values
+ *   codes  device, uint8 [rows, D/2]   (output)
+ *   scales device, fp32 [rows, D/16]   (output)
+ *   D % 16 == 0, D > 0; rows >= 0 (rows == 0 enqueues nothing). */
+csa2_status csa2_pack_fp4(const float *src, int64_t rows, int32_t D, uint8_t *codes,
+                          float *scales, void *stream);
+
+/* Dequantise: out[r, i] = E2M1(code[r, i]) * scale[r, i / 16] (one fp32
+ * multiply).  codes device uint8 [rows, D/2]; scales device fp32 [rows,
+ * D/16]; out device fp32 [rows, D]. */
+csa2_status csa2_unpack_fp4(const uint8_t *codes, const float *scales, int64_t rows, int32_t D,
+                            float *out, void *stream);
+
+/* ---------------------------------------------------------------------- */
+/* Indexer score + Top-K                                                   */
+/* ---------------------------------------------------------------------- */
+
+/* Workspace bytes csa2_index_topk needs for these sizes (0 on invalid
+ * sizes). */
+size_t csa2_index_topk_workspace_size(int32_t B, int32_t T, int32_t H_I, int32_t d_I, int64_t N,
+                                      int32_t topk);
+
+/* Indexer scores and Top-K selection ("Why Is DeepSeek V4.1 Flash So
+ * Fast?", section 4: a cheap relevance search over all compressed
+ * positions, then the Top-K go on to attention).
+ * Score of entry n for query (b, t), this library's reading:
+ *   dot_h    = sum_i q_idx[b,t,h,i] * k_idx[b,n,i]   (exact int32)
+ *   score    = (((0 + w[b,t,0]*dot_0) + w[b,t,1]*dot_1) + ...) + 0
+ * each fp32 product and sum rounded on its own (no fused multiply-add).
+ * Visibility: decode (n_prior < 0) sees all N entries; a prefill chunk
+ * (n_prior >= 0) query t sees n < min(N, n_prior + (t + 1) / ratio), i.e.
+ * chunk entry j once all `ratio` tokens it compresses are at or before t.
+ * Selection: the min(topk, visible) visible entries with the largest score,
+ * ties to the lower index, written in ascending index order; the rest of
+ * the row is -1.
+ *   q_idx     device, int8 [B, T, H_I, d_I]
+ *   w         device, fp32 [B, T, H_I]
+ *   k_idx     device, int8 [B, N, d_I]  (the entry store's index keys)
+ *   idx_out   device, int32 [B, T, topk]           (output)
+ *   score_out device, fp32 [B, T, N] or NULL       (optional output: the
+ *             score of every entry, -inf where the query may not see it)
+ *   ws        device workspace of ws_bytes >= csa2_index_topk_workspace_size
+ * Supported: d_I in {16, 32, 64, 128}, H_I in {1, 2, 4, 8}, H_I * d_I <= 256,
+ * 1 <= topk <= 65536, N < 2^31, ratio >= 1 when n_prior >= 0. */
+csa2_status csa2_index_topk(const int8_t *q_idx, const float *w, const int8_t *k_idx, int32_t B,
+                            int32_t T, int32_t H_I, int32_t d_I, int64_t N, int64_t n_prior,
+                            int32_t ratio, int32_t topk, int32_t *idx_out, float *score_out,
+                            void *ws, size_t ws_bytes, void *stream);
+
+/* ---------------------------------------------------------------------- */
+/* Sparse attention over the selected entries + the local window           */
+/* ---------------------------------------------------------------------- */
+
+/* Workspace bytes for csa2_sparse_attn_decode / _prefill (0 on invalid
+ * sizes). */
+size_t csa2_sparse_attn_workspace_size(int32_t B, int32_t T, int32_t H, int32_t D, int32_t topk,
+                                       int32_t W);
+
+/* Decode attention ("Why Is DeepSeek V4.1 Flash So Fast?", section 3: the
+ * selected compressed positions plus a 128-token sliding window).  Per
+ * head h of sequence b, this library's reading: one softmax over the
+ * logits sm_scale * <q[b,h], key> of every selected entry (key = the
+ * dequantised entry, which is also its value: one entry serves all heads)
+ * and every window row (key win_k, value win_v); out = sum p * value,
+ * lse = natural log of sum exp(logit).  Index -1 is padding and skipped;
+ * an index >= N is skipped and recorded in the device status word.  With
+ * nothing to attend to, out = 0 and lse = -inf.  fp32 accumulation.
+ *   q       device, bf16 [B, H, D]
+ *   codes   device, uint8 [B, N, D/2]; scales device, fp32 [B, N, D/16]
+ *   idx     device, int32 [B, topk]
+ *   win_k, win_v  device, bf16 [B, W, D]; row W-1 is the current token
+ *           (may be NULL when W == 0)
+ *   out     device, fp32 [B, H, D] (output); lse device, fp32 [B, H] or NULL
+ * Supported: D in {64, 128}, 1 <= H <= 128, 0 <= topk <= 65536,
+ * 0 <= W <= 4096. */
+csa2_status csa2_sparse_attn_decode(const uint16_t *q, const uint8_t *codes, const float *scales,
+                                    const int32_t *idx, const uint16_t *win_k,
+                                    const uint16_t *win_v, int32_t B, int32_t H, int32_t D,
+                                    int64_t N, int32_t topk, int32_t W, float sm_scale, float *out,
+                                    float *lse, void *ws, size_t ws_bytes, void *stream);
+
+/* Prefill (chunk) attention: as decode, for T query tokens per sequence.
+ *   q       device, bf16 [B, T, H, D]
+ *   idx     device, int32 [B, T, topk]  (e.g. from csa2_index_topk with
+ *           n_prior >= 0)
+ *   win_k, win_v device, bf16 [B, W-1+T, D]; query t reads rows t .. t+W-1
+ *           (row t+W-1 is token t itself)
+ *   out     device, fp32 [B, T, H, D]; lse device, fp32 [B, T, H] or NULL */
+csa2_status csa2_sparse_attn_prefill(const uint16_t *q, const uint8_t *codes, const float *scales,
+                                     const int32_t *idx, const uint16_t *win_k,
+                                     const uint16_t *win_v, int32_t B, int32_t T, int32_t H,
+                                     int32_t D, int64_t N, int32_t topk, int32_t W,
+                                     float sm_scale, float *out, float *lse, void *ws,
+                                     size_t ws_bytes, void *stream);
+
+/* ---------------------------------------------------------------------- */
+/* Cross-layer groups                                                      */
+/* ---------------------------------------------------------------------- */
+
+/* Shapes shared by every layer of a group. */
+typedef struct csa2_dims {
+    int32_t B, T, H, D;      /* batch, query tokens per sequence, heads, entry dim */
+    int64_t N;               /* stored entries per sequence */
+    int32_t H_I, d_I;        /* indexer heads and dim */
+    int32_t topk, W;         /* selected entries, window length */
+    int64_t n_prior;         /* -1: decode; >= 0: prefill chunk after n_prior entries */
+    int32_t ratio;           /* tokens per entry (prefill visibility) */
+    float sm_scale;          /* softmax scale (1/sqrt(D) by convention) */
+} csa2_dims;
+
+/* Per-layer device pointers (shapes as in the calls above).  q, q_idx, w,
+ * win_k, win_v, out, lse are the layer's own.  codes, scales, k_idx are
+ * read only for a layer that is some layer's kv_src (a Full layer).  idx
+ * [B, T, topk] is written for Full and Reindex layers; a Reuse layer's idx
+ * is ignored (it reads its idx_src layer's buffer). */
+typedef struct csa2_layer_io {
+    const uint16_t *q;
+    const int8_t *q_idx;
+    const float *w;
+    const uint16_t *win_k;
+    const uint16_t *win_v;
+    const uint8_t *codes;
+    const float *scales;
+    const int8_t *k_idx;
+    int32_t *idx;
+    float *out;
+    float *lse;
+} csa2_layer_io;
+
+/* CSA2_OK when the table follows the rules of csa2_layer_mode. */
+csa2_status csa2_validate_modes(const csa2_layer_mode *modes, int32_t L);
+
+/* The visual explainer's cache checklist ("DeepSeek-V4.1-Flash", section
+ * "Several mechanisms in one release"): entries x numbers per entry x
+ * stored layer copies x bits per number, in bytes, where stored layer
+ * copies = the table's Full layers.  modes is a host array of L rows. */
+csa2_status csa2_group_cache_bytes(const csa2_layer_mode *modes, int32_t L, int64_t entries,
+                                   int64_t numbers_per_entry, int64_t bits_per_number,
+                                   uint64_t *bytes_out);
+
+/* Workspace bytes for csa2_layer_group_run. */
+size_t csa2_layer_group_workspace_size(const csa2_dims *dims);
+
+/* Run L layers in table order on one stream: Full and Reindex layers run
+ * the index + Top-K step over their kv_src store's index keys with their
+ * own index query; Reuse layers take idx_src's selection; then every layer
+ * runs attention (decode when dims->T == 1 and n_prior < 0, else prefill)
+ * over its kv_src store with its own queries and window.
+ *   modes host array [L]; io host array [L] of device pointers; dims host.
+ * The table is validated before anything is enqueued. */
+csa2_status csa2_layer_group_run(const csa2_layer_mode *modes, const csa2_layer_io *io, int32_t L,
+                                 const csa2_dims *dims, void *ws, size_t ws_bytes, void *stream);
+
+/* ---------------------------------------------------------------------- */
+/* Kernel timing trace                                                     */
+/* ---------------------------------------------------------------------- */
+
+/* Turn the kernel timing trace on (enable != 0; clears earlier records) or
+ * off.  While on, every kernel the library launches is bracketed by a pair
+ * of CUDA events recorded on the launch stream, so per-kernel device time
+ * can be read back.  Host-side state, not thread-safe: enable, run and
+ * read from one host thread.  At most 1<<16 records are kept. */
+csa2_status csa2_trace_enable(int32_t enable);
+
+/* Number of kernel launches recorded since the trace was enabled. */
+int32_t csa2_trace_count(void);
+
+/* Record i: *name receives the kernel's static name, *ms its device time
+ * in milliseconds.  Waits for the record's stop event. */
+csa2_status csa2_trace_get(int32_t i, const char **name, float *ms);
+
+/* ---------------------------------------------------------------------- */
+/* Device status                                                           */
+/* ---------------------------------------------------------------------- */
+
+/* Synchronise `stream`, then read and clear the current device's status
+ * word.  *code_out (may be NULL) receives the raw word: 0 = clean, bit 0 =
+ * an attention index >= N was skipped, bit 1 = a pipeline wait gave up
+ * after its iteration limit.  Returns CSA2_ERR_DEVICE_STATUS when the word
+ * was non-zero, CSA2_ERR_CUDA when the synchronisation failed. */
+csa2_status csa2_get_device_status(void *stream, int32_t *code_out);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* CSA2_H */

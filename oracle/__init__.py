@@ -231,8 +231,14 @@ def layer_group(modes, layers, topk, n_prior=-1, ratio=4, sm_scale=None, rows=No
         store = layers[kv_src]
         B, T = lay["q"].shape[:2]
         if mode in (FULL, REINDEX):
-            idx = index_topk(lay["q_idx"], lay["w"], store["k_idx"], topk, n_prior, ratio)
-            idx = idx.reshape(B, T, topk)
+            sel = index_topk(lay["q_idx"], lay["w"], store["k_idx"], topk, n_prior, ratio,
+                             rows=rows)
+            if rows is None:
+                idx = sel.reshape(B, T, topk)
+            else:  # only the sampled rows are computed; the rest stay -1
+                idx = np.full((B * T, topk), -1, np.int32)
+                idx[np.asarray(rows)] = sel
+                idx = idx.reshape(B, T, topk)
         else:
             idx = results[idx_src]["idx"]
         out, lse = sparse_attn(lay["q"], store["codes"], store["scales"], idx, lay["win_k"],

@@ -1,0 +1,306 @@
+"""GPU parity: the CUDA path (through the C ABI) against the CPU oracle on the
+same seeded inputs.  FP4 codes/scales, unpacked values, indexer scores and
+top-k indices must be bit-exact; attention outputs within 2e-3 absolute +
+1e-2 relative of the fp64 oracle."""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import compressed_sparse_attention_topk_b200 as csa2
+from compressed_sparse_attention_topk_b200 import build as csa2_build
+from compressed_sparse_attention_topk_b200 import workloads as wl
+from tests._parity import (assert_bits_equal, assert_close, dev, gpu_store, host,
+                           oracle_store)
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _built():
+    csa2_build.build()
+    csa2.lib()
+    assert csa2.get_device_status() == 0
+
+
+# ---------------------------------------------------------------------------
+# FP4 pack / unpack
+# ---------------------------------------------------------------------------
+
+def _fp4_sources(D, rows=2000, seed=1):
+    rng = np.random.default_rng(seed)
+    x = (rng.standard_normal((rows, D)) * np.exp(rng.uniform(-30, 30, (rows, 1)))).astype(
+        np.float32)
+    x[:rows // 100] *= np.float32(8.0)            # outliers
+    x[5] = 0.0                                     # zero row
+    x[6, :16] = np.float32(1e-41)                  # subnormal group
+    x[7, :16] = -np.float32(3e-39)
+    mids = np.array([6, 0.25, 0.75, 1.25, 1.75, 2.5, 3.5, 5.0, -0.25, -0.75, -1.25, -1.75, -2.5,
+                     -3.5, -5.0, -6.0], np.float32)
+    for i, e in enumerate(range(-10, 10)):         # exact midpoints: ties
+        x[10 + i, :16] = mids * np.float32(2.0 ** e)
+        if D >= 32:
+            x[10 + i, 16:32] = -mids * np.float32(2.0 ** e)
+    x[40, :16] = np.float32([6, 5.9999995, 6.0000005, 0.2499999, 0.2500001] + [0] * 11)
+    return x
+
+
+@pytest.mark.parametrize("D", [16, 64, 128])
+def test_pack_unpack_bit_exact(D):
+    x = _fp4_sources(D, seed=D)
+    oc, os_ = oracle.pack_fp4(x)
+    gc, gs = csa2.pack_fp4(dev(x))
+    assert_bits_equal(host(gc), oc, "codes")
+    assert_bits_equal(host(gs), os_, "scales")
+    ou = oracle.unpack_fp4(oc, os_, D)
+    gu = csa2.unpack_fp4(gc, gs, D)
+    assert_bits_equal(host(gu), ou, "unpacked")
+
+
+# ---------------------------------------------------------------------------
+# Indexer scores + top-k
+# ---------------------------------------------------------------------------
+
+def _index_case(B, T, H_I, d_I, N, seed, key_levels=None, q_zero=False):
+    rng = np.random.default_rng(seed)
+    q = wl.int8_uniform(rng, (B, T, H_I, d_I))
+    if q_zero:
+        q[:] = 0
+    w = rng.random((B, T, H_I), dtype=np.float32)
+    if key_levels is None:
+        k = wl.int8_uniform(rng, (B, N, d_I))
+    else:
+        k = rng.integers(-key_levels, key_levels + 1, (B, N, d_I)).astype(np.int8)
+    return q, w, k
+
+
+def _check_index(q, w, k, topk, n_prior=-1, ratio=4, rows=None, check_scores=True):
+    B, T = q.shape[:2]
+    N = k.shape[1]
+    g_idx, g_sc = csa2.index_topk(dev(q), dev(w), dev(k), topk, n_prior, ratio,
+                                  want_scores=check_scores)
+    g_idx = host(g_idx).reshape(B * T, topk)
+    if rows is not None:
+        g_idx = g_idx[rows]
+    o_idx, o_sc = oracle.index_topk(q, w, k, topk, n_prior, ratio, rows=rows, want_scores=True)
+    if check_scores:
+        g_sc = host(g_sc).reshape(B * T, N)
+        if rows is not None:
+            g_sc = g_sc[rows]
+        assert_bits_equal(g_sc, o_sc, "scores")
+    assert_bits_equal(g_idx, o_idx, "indices")
+    return g_idx
+
+
+@pytest.mark.parametrize("d_I,H_I", [(16, 1), (16, 8), (32, 2), (32, 4), (32, 8), (64, 1),
+                                     (64, 4), (64, 8), (128, 2), (128, 4)])
+@pytest.mark.parametrize("N", [1, 777, 5000])
+def test_index_topk_shapes(d_I, H_I, N):
+    q, w, k = _index_case(3, 1, H_I, d_I, N, seed=d_I * 100 + H_I + N)
+    _check_index(q, w, k, topk=64)
+
+
+@pytest.mark.parametrize("topk", [1, 7, 64, 2048, 5000])
+def test_index_topk_k_sweep_and_padding(topk):
+    q, w, k = _index_case(2, 1, 4, 64, 3001, seed=topk)
+    _check_index(q, w, k, topk)
+
+
+def test_topk_all_equal_scores_take_lowest_indices():
+    q, w, k = _index_case(2, 1, 4, 32, 9000, seed=3, q_zero=True)
+    idx = _check_index(q, w, k, 300)
+    assert np.array_equal(idx, np.tile(np.arange(300, dtype=np.int32), (2, 1)))
+
+
+@pytest.mark.parametrize("levels", [1, 2])
+def test_topk_heavy_ties_at_boundary(levels):
+    q, w, k = _index_case(4, 1, 2, 16, 20000, seed=levels, key_levels=levels)
+    w[:] = 1.0
+    _check_index(q, w, k, 1000)
+
+
+def test_topk_empty_store():
+    q, w, k = _index_case(2, 1, 4, 64, 0, seed=1)
+    idx = csa2.index_topk(dev(q), dev(w), torch.empty((2, 0, 64), dtype=torch.int8,
+                                                       device="cuda"), 5)
+    assert np.all(host(idx) == -1)
+
+
+def test_prefill_visibility():
+    B, T, H_I, d_I, n_prior, ratio = 2, 67, 4, 64, 301, 4
+    N = n_prior + T // ratio
+    q, w, k = _index_case(B, T, H_I, d_I, N, seed=9)
+    _check_index(q, w, k, 320, n_prior=n_prior, ratio=ratio)
+
+
+@pytest.mark.parametrize("wl_name", ["tiny_decode_n1024", "decode_b32_n131072"])
+def test_index_topk_workload(wl_name):
+    w0 = wl.ALL[wl_name]
+    lay = wl.layer_inputs(w0, 0)
+    _check_index(lay["q_idx"], lay["w"], lay["k_idx"], w0.topk)
+
+
+# ---------------------------------------------------------------------------
+# Attention
+# ---------------------------------------------------------------------------
+
+def _attn_inputs(B, T, H, D, N, topk, W, seed, idx_mode="random"):
+    rng = np.random.default_rng(seed)
+    entries = rng.standard_normal((B, N, D)).astype(np.float32)
+    q = wl.bf16_bits(rng.standard_normal((B, T, H, D)).astype(np.float32))
+    wk = wl.bf16_bits(rng.standard_normal((B, W - 1 + T, D)).astype(np.float32)) if W else None
+    wv = wl.bf16_bits(rng.standard_normal((B, W - 1 + T, D)).astype(np.float32)) if W else None
+    if idx_mode == "random":
+        idx = np.stack([np.sort(rng.choice(N, min(topk, N), replace=False))
+                        for _ in range(B * T)]).astype(np.int32)
+        if topk > N:
+            idx = np.concatenate([idx, np.full((B * T, topk - N), -1, np.int32)], axis=1)
+    else:
+        idx = np.full((B * T, topk), -1, np.int32)
+    return entries, q, wk, wv, idx.reshape(B, T, topk)
+
+
+def _check_attn(entries, q, wk, wv, idx, decode):
+    B, T, H, D = q.shape
+    oc, os_ = oracle_store(entries)
+    gc, gs = gpu_store(entries)
+    ref_out, ref_lse = oracle.sparse_attn(q, oc, os_, idx, wk, wv)
+    if decode:
+        out, lse = csa2.sparse_attn_decode(dev(q[:, 0]), gc, gs, dev(idx[:, 0]),
+                                           None if wk is None else dev(wk),
+                                           None if wv is None else dev(wv))
+    else:
+        out, lse = csa2.sparse_attn_prefill(dev(q), gc, gs, dev(idx),
+                                            None if wk is None else dev(wk),
+                                            None if wv is None else dev(wv))
+    assert_close(host(out).reshape(B * T, H, D), ref_out, "out")
+    assert_close(host(lse).reshape(B * T, H), ref_lse, "lse")
+
+
+@pytest.mark.parametrize("D,H,topk,W", [(64, 8, 64, 128), (128, 16, 2048, 128), (128, 16, 100, 0),
+                                        (128, 20, 130, 70), (64, 3, 0, 5), (128, 16, 37, 1)])
+def test_attention_decode(D, H, topk, W):
+    entries, q, wk, wv, idx = _attn_inputs(3, 1, H, D, 4000, topk, W, seed=D + H + topk + W)
+    _check_attn(entries, q, wk, wv, idx, decode=True)
+
+
+def test_attention_padding_and_nothing_to_attend():
+    entries, q, wk, wv, idx = _attn_inputs(2, 1, 16, 128, 500, 64, 0, seed=5)
+    idx[0, 0, ::3] = -1
+    idx[1, 0, :] = -1          # sequence 1: nothing to attend to
+    _check_attn(entries, q, wk, wv, idx, decode=True)
+
+
+def test_attention_bad_index_recorded_and_skipped():
+    entries, q, wk, wv, idx = _attn_inputs(2, 1, 16, 128, 300, 32, 16, seed=7)
+    bad = idx.copy()
+    bad[0, 0, 4] = 300 + 5
+    skipped = bad.copy()
+    skipped[0, 0, 4] = -1
+    oc, os_ = oracle_store(entries)
+    gc, gs = gpu_store(entries)
+    ref_out, _ = oracle.sparse_attn(q, oc, os_, skipped, wk, wv)
+    out, _ = csa2.sparse_attn_decode(dev(q[:, 0]), gc, gs, dev(bad[:, 0]), dev(wk), dev(wv))
+    assert_close(host(out), ref_out, "out")
+    assert csa2.get_device_status() & 1
+    assert csa2.get_device_status() == 0   # reading clears it
+
+
+@pytest.mark.parametrize("T,W", [(37, 16), (5, 128), (64, 1)])
+def test_attention_prefill(T, W):
+    entries, q, wk, wv, idx = _attn_inputs(2, T, 16, 128, 700, 96, W, seed=T + W)
+    _check_attn(entries, q, wk, wv, idx, decode=False)
+
+
+# ---------------------------------------------------------------------------
+# Whole workloads through the C ABI
+# ---------------------------------------------------------------------------
+
+def _store_for(lay):
+    return oracle_store(lay["entries"]), gpu_store(lay["entries"])
+
+
+def test_tiny_workload_end_to_end():
+    w0 = wl.TINY
+    lay = wl.layer_inputs(w0, 0)
+    (oc, os_), (gc, gs) = _store_for(lay)
+    assert_bits_equal(host(gc), oc, "codes")
+    g_idx = csa2.index_topk(dev(lay["q_idx"]), dev(lay["w"]), dev(lay["k_idx"]), w0.topk)
+    o_idx = oracle.index_topk(lay["q_idx"], lay["w"], lay["k_idx"], w0.topk)
+    assert_bits_equal(host(g_idx).reshape(1, -1), o_idx, "idx")
+    out, lse = csa2.sparse_attn_decode(dev(lay["q"][:, 0]), gc, gs, g_idx[:, 0],
+                                       dev(lay["win_k"]), dev(lay["win_v"]))
+    ref_out, ref_lse = oracle.sparse_attn(lay["q"], oc, os_, o_idx.reshape(1, 1, -1),
+                                          lay["win_k"], lay["win_v"])
+    assert_close(host(out), ref_out, "out")
+    assert_close(host(lse), ref_lse, "lse")
+
+
+def _group_tensors(w0, layers):
+    tens = []
+    for l, lay in enumerate(layers):
+        d = {k: dev(v) for k, v in lay.items() if k != "entries"}
+        d["q"] = d["q"] if w0.T > 1 else d["q"][:, 0].contiguous()
+        if "entries" in lay:
+            d["codes"], d["scales"] = gpu_store(lay["entries"])
+        d["idx"] = torch.empty((w0.B, w0.T, w0.topk), dtype=torch.int32, device="cuda")
+        shape = (w0.B, w0.T, w0.H) if w0.T > 1 else (w0.B, w0.H)
+        d["out"] = torch.empty(shape + (w0.D,), dtype=torch.float32, device="cuda")
+        d["lse"] = torch.empty(shape, dtype=torch.float32, device="cuda")
+        tens.append(d)
+    return tens
+
+
+def _run_group_and_compare(w0, rows=None):
+    layers = wl.all_layer_inputs(w0)
+    tens = _group_tensors(w0, layers)
+    dims = csa2.make_dims(w0.B, w0.T, w0.H, w0.D, w0.N, w0.H_I, w0.d_I, w0.topk, w0.W,
+                          w0.n_prior, w0.ratio)
+    csa2.layer_group_run(list(w0.modes), tens, dims)
+    for lay in layers:
+        if "entries" in lay:
+            lay["codes"], lay["scales"] = oracle_store(lay["entries"])
+    ref = oracle.layer_group(list(w0.modes), layers, w0.topk, w0.n_prior, w0.ratio, rows=rows)
+    for l, (mode, kv, ix) in enumerate(w0.modes):
+        g_idx = host(tens[ix]["idx"]).reshape(w0.B * w0.T, w0.topk)
+        o_idx = ref[l]["idx"].reshape(w0.B * w0.T, w0.topk)
+        if rows is not None:
+            g_idx, o_idx = g_idx[rows], o_idx[rows]
+        assert_bits_equal(g_idx, o_idx, f"layer {l} idx")
+        out = host(tens[l]["out"]).reshape(w0.B * w0.T, w0.H, w0.D)
+        lse = host(tens[l]["lse"]).reshape(w0.B * w0.T, w0.H)
+        if rows is not None:
+            out, lse = out[rows], lse[rows]
+        assert_close(out, ref[l]["out"], f"layer {l} out")
+        assert_close(lse, ref[l]["lse"], f"layer {l} lse")
+    assert csa2.get_device_status() == 0
+    return tens
+
+
+def test_group_workload_16_layers():
+    """4 groups of (Full, Reindex, Reuse, Reuse), B=8, N=4096, k=512."""
+    w0 = wl.GROUP
+    tens = _run_group_and_compare(w0)
+    assert csa2.group_cache_bytes(list(w0.modes), w0.N, 128, 8) == 2 * 1024 * 1024
+
+
+def test_long_decode_workload_full_size():
+    """The 1M-token decode workload at full size (B=4, N=262144, Full +
+    Reindex), in the launch configuration the benchmark times."""
+    _run_group_and_compare(wl.LONG)
+
+
+def test_decode_workload_full_size():
+    """B=32, N=131072, d_I=32, k=2048, with salient outlier entries."""
+    _run_group_and_compare(wl.DECODE)
+
+
+def test_prefill_workload_sampled_rows():
+    """Chunked prefill at full size (T=4096 after 262,144 prior entries):
+    every row computed on the GPU, a spread sample checked against the
+    oracle (first 16, last 16, 32 seeded)."""
+    w0 = wl.PREFILL
+    rng = np.random.default_rng(1234)
+    rows = np.unique(np.concatenate([np.arange(16), np.arange(w0.T - 16, w0.T),
+                                     rng.choice(w0.T, 32, replace=False)])).astype(np.int64)
+    _run_group_and_compare(w0, rows=rows)
