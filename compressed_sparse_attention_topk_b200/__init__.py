@@ -31,6 +31,7 @@ EXPORTED = (
     "csa2_sparse_attn_decode", "csa2_sparse_attn_prefill", "csa2_validate_modes",
     "csa2_group_cache_bytes", "csa2_layer_group_workspace_size", "csa2_layer_group_run",
     "csa2_get_device_status", "csa2_trace_enable", "csa2_trace_count", "csa2_trace_get",
+    "csa2_layer_run",
 )
 
 
@@ -87,6 +88,7 @@ def lib() -> ctypes.CDLL:
         "csa2_group_cache_bytes": ([P, i32, i64, i64, i64, P], i32),
         "csa2_layer_group_workspace_size": ([P], sz),
         "csa2_layer_group_run": ([P, P, i32, P, P, sz, P], i32),
+        "csa2_layer_run": ([P, P, i32, i32, P, P, sz, P], i32),
         "csa2_get_device_status": ([P, P], i32),
         "csa2_trace_enable": ([i32], i32),
         "csa2_trace_count": ([], i32),
@@ -322,6 +324,36 @@ def layer_group_run(modes, layers: List[dict], dims: Dims, ws=None):
         ws = workspace(need)
     _check(lib().csa2_layer_group_run(arr, io, len(layers), ctypes.byref(dims), _ptr(ws),
                                       ws.numel(), _stream()), "csa2_layer_group_run")
+
+
+class LayerGroup:
+    """A mode table with its layers' device tensors, marshalled once, so a
+    layer (or the whole group) can be launched repeatedly with one C call
+    (e.g. inside CUDA graph capture)."""
+
+    def __init__(self, modes, layers: List[dict], dims: Dims, ws=None):
+        self.modes = _modes_array(modes)
+        self.L = len(layers)
+        self.layers = layers
+        self.io = (LayerIO * self.L)()
+        for i, lay in enumerate(layers):
+            for name, _ in LayerIO._fields_:
+                t = lay.get(name)
+                if t is not None:
+                    _dev(t, f"layers[{i}].{name}")
+                setattr(self.io[i], name, _ptr(t))
+        self.dims = dims
+        need = layer_group_workspace_size(dims)
+        self.ws = workspace(need) if ws is None else ws
+
+    def run_layer(self, layer: int):
+        _check(lib().csa2_layer_run(self.modes, self.io, self.L, layer, ctypes.byref(self.dims),
+                                    _ptr(self.ws), self.ws.numel(), _stream()), "csa2_layer_run")
+
+    def run(self):
+        _check(lib().csa2_layer_group_run(self.modes, self.io, self.L, ctypes.byref(self.dims),
+                                          _ptr(self.ws), self.ws.numel(), _stream()),
+               "csa2_layer_group_run")
 
 
 def get_device_status() -> int:

@@ -28,6 +28,12 @@ __device__ __forceinline__ uint32_t score_key(float f) {
   return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
 }
 
+__host__ __device__ __forceinline__ int64_t min64(int64_t a, int64_t b) { return a < b ? a : b; }
+
+__device__ __forceinline__ float bf16_to_f32_bits(uint16_t b) {
+  return __uint_as_float(((uint32_t)b) << 16);
+}
+
 // Radix digits of a key used by the top-k selection: 11 + 11 + 10 bits.
 constexpr int kBins1 = 2048, kBins2 = 2048, kBins3 = 1024;
 __device__ __forceinline__ uint32_t key_d1(uint32_t k) { return k >> 21; }
@@ -116,6 +122,11 @@ __device__ __forceinline__ float warp_sum(float v) {
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
   return v;
+}
+__device__ __forceinline__ uint32_t lanemask_lt_u32() {
+  uint32_t m;
+  asm("mov.u32 %0, %%lanemask_lt;" : "=r"(m));
+  return m;
 }
 __device__ __forceinline__ uint32_t warp_incl_scan(uint32_t v) {
   const int lane = threadIdx.x & 31;

@@ -7,11 +7,10 @@
 #include <cstdint>
 #include <cstring>
 
-#include "attention.cuh"
 #include "common.cuh"
 #include "index_scan.cuh"
 #include "pack.cuh"
-#include "topk.cuh"
+#include "row_cluster.cuh"
 
 using namespace csa2;
 
@@ -98,18 +97,18 @@ int64_t topk_rows_per_pass(int64_t rows, int64_t N) {
   return std::min<int64_t>(R, std::max<int64_t>(rows, 1));
 }
 
-int topk_regions(int64_t N) {
-  return (int)std::min<int64_t>(kMaxRegions, std::max<int64_t>(1, ceil_div(N, kSelSpan)));
-}
+// Row stride of the workspace score rows: a multiple of 4 floats, so every
+// row starts 16-byte aligned for bulk copies.
+inline int64_t score_stride(int64_t N) { return (N + 3) & ~int64_t(3); }
 
 struct TopkWs {
   float *scores;
   uint2 *cand;
-  uint32_t *hist1, *hist2, *cnt;
+  uint32_t *hist1;
   size_t bytes;
 };
 
-TopkWs topk_ws_layout(void *base, int64_t R, int64_t N, int G2) {
+TopkWs topk_ws_layout(void *base, int64_t R, int64_t N) {
   TopkWs w{};
   size_t off = 0;
   auto take = [&](size_t bytes) {
@@ -117,30 +116,52 @@ TopkWs topk_ws_layout(void *base, int64_t R, int64_t N, int G2) {
     off += align_up(bytes, 256);
     return o;
   };
-  const size_t o_scores = take(size_t(R) * N * 4);
+  const size_t o_scores = take(size_t(R) * score_stride(N) * 4);
   const size_t o_cand = take(size_t(R) * N * 8);
-  const size_t o_hist = take(size_t(R) * (kBins1 + kBins2) * 4);
-  const size_t o_cnt = take(size_t(R) * G2 * 4);
+  const size_t o_hist = take(size_t(R) * kBins1 * 4);
   char *p = static_cast<char *>(base);
   w.scores = reinterpret_cast<float *>(p + o_scores);
   w.cand = reinterpret_cast<uint2 *>(p + o_cand);
   w.hist1 = reinterpret_cast<uint32_t *>(p + o_hist);
-  w.hist2 = w.hist1 + size_t(R) * kBins1;
-  w.cnt = reinterpret_cast<uint32_t *>(p + o_cnt);
   w.bytes = off;
   return w;
+}
+
+// Per-device one-time kernel attribute setup (dynamic shared memory above
+// 48 KiB, non-portable cluster size).  Must run before any stream capture;
+// the entry points call it on their first use on a device.
+template <typename K>
+csa2_status set_smem_attr(K kernel, size_t bytes, bool big_cluster) {
+  if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes) !=
+      cudaSuccess)
+    return CSA2_ERR_CUDA;
+  if (big_cluster &&
+      cudaFuncSetAttribute(kernel, cudaFuncAttributeNonPortableClusterSizeAllowed, 1) !=
+          cudaSuccess)
+    return CSA2_ERR_CUDA;
+  return CSA2_OK;
 }
 
 template <int DI, int HI>
 void launch_scan(dim3 grid, cudaStream_t st, const int8_t *q_idx, const float *w,
                  const int8_t *k_idx, int32_t T, int64_t N, int64_t n_prior, int32_t ratio,
-                 int64_t row0, float *scores, uint32_t *hist1, int write_masked) {
-  index_scan_kernel<DI, HI><<<grid, kScanThreads, 0, st>>>(q_idx, w, k_idx, T, N, n_prior, ratio,
-                                                            row0, scores, hist1, write_masked);
+                 int64_t row0, float *scores, int64_t stride, uint32_t *hist1,
+                 int write_masked) {
+  using S = ScanShape<DI, HI>;
+  static bool done[256] = {false};
+  int dev = 0;
+  cudaGetDevice(&dev);
+  if (dev < 0 || dev >= 256 || !done[dev]) {
+    set_smem_attr(index_scan_kernel<DI, HI>, S::SMEM, false);
+    if (dev >= 0 && dev < 256) done[dev] = true;
+  }
+  index_scan_kernel<DI, HI><<<grid, kScanThreads, S::SMEM, st>>>(
+      q_idx, w, k_idx, T, N, n_prior, ratio, row0, scores, stride, hist1, write_masked);
 }
 
 using ScanLaunch = void (*)(dim3, cudaStream_t, const int8_t *, const float *, const int8_t *,
-                            int32_t, int64_t, int64_t, int32_t, int64_t, float *, uint32_t *, int);
+                            int32_t, int64_t, int64_t, int32_t, int64_t, float *, int64_t,
+                            uint32_t *, int);
 
 ScanLaunch pick_scan(int32_t d_I, int32_t H_I) {
 #define CSA2_SCAN_CASE(DI, HI) \
@@ -151,6 +172,85 @@ ScanLaunch pick_scan(int32_t d_I, int32_t H_I) {
   CSA2_SCAN_CASE(128, 1) CSA2_SCAN_CASE(128, 2) CSA2_SCAN_CASE(128, 4)
 #undef CSA2_SCAN_CASE
   return nullptr;
+}
+
+// ---- the per-row cluster kernel -------------------------------------------
+template <int D, int CL>
+csa2_status launch_row_cl(const RowParams &p, int64_t nr, cudaStream_t st) {
+  const size_t smem = sizeof(RowSmem<D>);
+  static bool done[256] = {false};
+  int dev = 0;
+  cudaGetDevice(&dev);
+  if (dev < 0 || dev >= 256 || !done[dev]) {
+    if (set_smem_attr(row_cluster_kernel<D, CL>, smem, CL > 8) != CSA2_OK) return CSA2_ERR_CUDA;
+    if (dev >= 0 && dev < 256) done[dev] = true;
+  }
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3((unsigned)(nr * CL), 1, 1);
+  cfg.blockDim = dim3(kRowThreads, 1, 1);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = CL;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, row_cluster_kernel<D, CL>, p) == cudaSuccess ? CSA2_OK
+                                                                                : CSA2_ERR_CUDA;
+}
+
+// Can clusters of 16 CTAs of the row kernel be scheduled on this device?
+template <int D>
+bool cluster16_ok() {
+  static int cache[256] = {0};  // 0 unknown, 1 yes, 2 no
+  int dev = 0;
+  cudaGetDevice(&dev);
+  if (dev >= 0 && dev < 256 && cache[dev]) return cache[dev] == 1;
+  const size_t smem = sizeof(RowSmem<D>);
+  bool ok = set_smem_attr(row_cluster_kernel<D, 16>, smem, true) == CSA2_OK;
+  if (ok) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(16, 1, 1);
+    cfg.blockDim = dim3(kRowThreads, 1, 1);
+    cfg.dynamicSmemBytes = smem;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = 16;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    int n = 0;
+    ok = cudaOccupancyMaxActiveClusters(&n, row_cluster_kernel<D, 16>, &cfg) == cudaSuccess &&
+         n > 0;
+  }
+  cudaGetLastError();
+  if (dev >= 0 && dev < 256) cache[dev] = ok ? 1 : 2;
+  return ok;
+}
+
+// Rows of one launch -> CTAs per row: as many as keep about two CTAs per SM.
+int row_cluster_size(int64_t nr, int D) {
+  const int64_t target = 2 * int64_t(device_sms());
+  int cl = 4;
+  if (nr * 8 <= target) cl = 8;
+  if (nr * 16 <= target && (D == 128 ? cluster16_ok<128>() : cluster16_ok<64>())) cl = 16;
+  return cl;
+}
+
+csa2_status launch_row(const RowParams &p, int D, int64_t nr, cudaStream_t st) {
+  TraceScope ts(p.do_topk ? (p.do_attn ? "topk_attend" : "topk_select") : "attend", st);
+  const int cl = row_cluster_size(nr, D);
+  if (D == 128) {
+    if (cl == 16) return launch_row_cl<128, 16>(p, nr, st);
+    if (cl == 8) return launch_row_cl<128, 8>(p, nr, st);
+    return launch_row_cl<128, 4>(p, nr, st);
+  }
+  if (cl == 16) return launch_row_cl<64, 16>(p, nr, st);
+  if (cl == 8) return launch_row_cl<64, 8>(p, nr, st);
+  return launch_row_cl<64, 4>(p, nr, st);
 }
 
 csa2_status check_topk_args(const int8_t *q_idx, const float *w, const int8_t *k_idx, int32_t B,
@@ -173,82 +273,87 @@ csa2_status check_topk_args(const int8_t *q_idx, const float *w, const int8_t *k
 size_t topk_ws_bytes(int32_t B, int32_t T, int64_t N) {
   const int64_t rows = int64_t(B) * T;
   const int64_t R = topk_rows_per_pass(rows, N);
-  return topk_ws_layout(nullptr, R, N, topk_regions(N)).bytes;
+  return topk_ws_layout(nullptr, R, N).bytes;
 }
 
+struct AttnArgs {  // attention inputs of one layer (all device pointers)
+  const uint16_t *q;
+  const uint8_t *codes;
+  const float *scales;
+  const uint16_t *win_k, *win_v;
+  int32_t H, D, W;
+  float sm_scale;
+  float *out, *lse;
+};
+
+// Index + top-k (and, when `att` is given, the layer's attention fused into
+// the same per-row cluster kernel), in passes of R rows.
 csa2_status run_index_topk(const int8_t *q_idx, const float *w, const int8_t *k_idx, int32_t B,
                            int32_t T, int32_t H_I, int32_t d_I, int64_t N, int64_t n_prior,
                            int32_t ratio, int32_t topk, int32_t *idx_out, float *score_out,
-                           void *ws, size_t ws_bytes, cudaStream_t st) {
+                           const AttnArgs *att, void *ws, size_t ws_bytes, cudaStream_t st) {
   const int64_t rows = int64_t(B) * T;
   const int64_t R = topk_rows_per_pass(rows, N);
-  const int G2 = topk_regions(N);
-  const TopkWs L0 = topk_ws_layout(nullptr, R, N, G2);
+  const TopkWs L0 = topk_ws_layout(nullptr, R, N);
   if (!ws || ws_bytes < L0.bytes || !aligned(ws, 16)) return CSA2_ERR_WORKSPACE;
-  const TopkWs L = topk_ws_layout(ws, R, N, G2);
+  const TopkWs L = topk_ws_layout(ws, R, N);
   const ScanLaunch scan = pick_scan(d_I, H_I);
   if (!scan) return CSA2_ERR_UNSUPPORTED;
   const int sms = device_sms();
 
   for (int64_t row0 = 0; row0 < rows; row0 += R) {
     const int64_t nr = std::min<int64_t>(R, rows - row0);
-    // hist1 and hist2 of all R rows are one contiguous block
-    if (cudaMemsetAsync(L.hist1, 0, size_t(R) * (kBins1 + kBins2) * 4, st) != cudaSuccess)
+    if (cudaMemsetAsync(L.hist1, 0, size_t(nr) * kBins1 * 4, st) != cudaSuccess)
       return CSA2_ERR_CUDA;
+    const int64_t stride = score_out ? N : score_stride(N);
     float *scores = score_out ? score_out + row0 * N : L.scores;
-    // scan: ~3 CTAs per SM in total, at least 256 keys per CTA
-    const int64_t g_want = ceil_div(3 * sms, nr);
-    const int64_t g_max = std::max<int64_t>(1, ceil_div(N, 256));
-    const int G = (int)std::max<int64_t>(1, std::min(g_want, g_max));
+    // scan: about two CTAs per SM in total (the slices of a row are balanced
+    // to 16 keys), at least 256 keys per CTA
+    const int64_t g_want = std::max<int64_t>(1, (2 * sms + nr / 2) / nr);
+    const int64_t g_max = std::max<int64_t>(1, N / 256);
+    const int G = (int)std::min(g_want, g_max);
     {
       TraceScope ts("index_scan", st);
       scan(dim3(G, (unsigned)nr), st, q_idx, w, k_idx, T, N, n_prior, ratio, row0, scores,
-           L.hist1, score_out != nullptr);
+           stride, L.hist1, score_out != nullptr);
     }
     if (after_launch() != CSA2_OK) return CSA2_ERR_CUDA;
-    {
-      TraceScope ts("topk_select", st);
-      topk_select_kernel<<<dim3(G2, (unsigned)nr), kSelThreads, 0, st>>>(
-          scores, N, T, n_prior, ratio, row0, topk, L.hist1, L.hist2, L.cand, L.cnt);
+    RowParams p{};
+    p.scores = scores;
+    p.score_stride = stride;
+    p.hist1 = L.hist1;
+    p.cand = L.cand;
+    p.N = N;
+    p.T = T;
+    p.n_prior = n_prior;
+    p.ratio = ratio;
+    p.row0 = row0;
+    p.topk = topk;
+    p.idx = idx_out;
+    p.do_topk = 1;
+    int D = 64;
+    if (att) {
+      p.q = att->q;
+      p.codes = att->codes;
+      p.scales = att->scales;
+      p.win_k = att->win_k;
+      p.win_v = att->win_v;
+      p.H = att->H;
+      p.W = att->W;
+      p.q_scale = att->sm_scale * 1.4426950408889634f;
+      p.out = att->out;
+      p.lse = att->lse;
+      p.do_attn = 1;
+      D = att->D;
     }
-    if (after_launch() != CSA2_OK) return CSA2_ERR_CUDA;
-    {
-      TraceScope ts("topk_finalize", st);
-      topk_finalize_kernel<<<(unsigned)nr, kFinThreads, 0, st>>>(N, T, n_prior, ratio, row0,
-                                                                 topk, L.hist1, L.hist2, L.cand,
-                                                                 L.cnt, G2, idx_out);
-    }
-    if (after_launch() != CSA2_OK) return CSA2_ERR_CUDA;
+    if (launch_row(p, D, nr, st) != CSA2_OK) return CSA2_ERR_CUDA;
   }
   return CSA2_OK;
 }
 
 // ---------------------------------------------------------------------------
-// Attention: shapes, workspace, launches.
+// Attention with given indices.
 // ---------------------------------------------------------------------------
-constexpr int64_t kAttnMaxRowsPerLaunch = 65535;
-
-struct AttnPlan {
-  int64_t rows_per_launch;
-  int n_chunks, splits, chunks_per_split, hgroups;
-  size_t part_bytes;
-};
-
-AttnPlan attn_plan(int32_t B, int32_t T, int32_t H, int32_t D, int32_t topk, int32_t W) {
-  AttnPlan p{};
-  const int64_t rows = int64_t(B) * T;
-  p.rows_per_launch = std::max<int64_t>(1, std::min<int64_t>(rows, kAttnMaxRowsPerLaunch));
-  p.n_chunks = (int)(ceil_div(topk, kAttnKeys) + ceil_div(W, kAttnKeys));
-  p.hgroups = (int)ceil_div(H, kAttnHeads);
-  const int64_t want = ceil_div(2 * int64_t(device_sms()), p.rows_per_launch * p.hgroups);
-  p.splits = (int)std::max<int64_t>(1, std::min<int64_t>(want, std::max(1, p.n_chunks)));
-  p.chunks_per_split = (int)ceil_div(p.n_chunks, p.splits);
-  if (p.chunks_per_split > 0) p.splits = (int)ceil_div(p.n_chunks, p.chunks_per_split);
-  if (p.splits < 1) p.splits = 1;
-  p.part_bytes = align_up(size_t(p.rows_per_launch) * H * p.splits * (D + 2) * 4, 256);
-  return p;
-}
-
 csa2_status check_attn_args(const uint16_t *q, const uint8_t *codes, const float *scales,
                             const int32_t *idx, const uint16_t *win_k, const uint16_t *win_v,
                             int32_t B, int32_t T, int32_t H, int32_t D, int64_t N, int32_t topk,
@@ -269,74 +374,37 @@ csa2_status check_attn_args(const uint16_t *q, const uint8_t *codes, const float
   return CSA2_OK;
 }
 
-template <int D>
-csa2_status launch_attn(const AttnPlan &p, int64_t row0, int64_t nr, const uint16_t *q,
-                        const uint8_t *codes, const float *scales, const int32_t *idx,
-                        const uint16_t *win_k, const uint16_t *win_v, int32_t T, int32_t H,
-                        int64_t N, int32_t topk, int32_t W, float q_scale, float *part,
-                        float *out, float *lse, cudaStream_t st) {
-  const size_t smem = sizeof(AttnSmem<D>);
-  static bool attr_set[256] = {false};
-  int dev = 0;
-  cudaGetDevice(&dev);
-  if (dev < 0 || dev >= 256 || !attr_set[dev]) {
-    if (cudaFuncSetAttribute(sparse_attn_partial_kernel<D>,
-                             cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess)
-      return CSA2_ERR_CUDA;
-    if (dev >= 0 && dev < 256) attr_set[dev] = true;
-  }
-  // Offset the row-indexed inputs so the kernel's row 0 is global row row0.
-  // The kernel derives (b, t) from its row, so launches start on a
-  // sequence boundary.
-  const int64_t b0 = row0 / T;
-  const uint16_t *q0 = q + row0 * H * (int64_t)D;
-  const int32_t *idx0 = idx ? idx + row0 * (int64_t)topk : nullptr;
-  const uint8_t *codes0 = codes ? codes + b0 * N * (D / 2) : nullptr;
-  const float *scales0 = scales ? scales + b0 * N * (D / 16) : nullptr;
-  const int64_t win_rows = int64_t(W) - 1 + T;
-  const uint16_t *wk0 = win_k ? win_k + b0 * win_rows * D : nullptr;
-  const uint16_t *wv0 = win_v ? win_v + b0 * win_rows * D : nullptr;
-  {
-    TraceScope ts("attn_partial", st);
-    sparse_attn_partial_kernel<D>
-        <<<dim3(p.splits, (unsigned)nr, p.hgroups), kAttnThreads, smem, st>>>(
-            q0, codes0, scales0, idx0, wk0, wv0, T, H, N, topk, W, q_scale, p.chunks_per_split,
-            part);
-  }
-  if (after_launch() != CSA2_OK) return CSA2_ERR_CUDA;
-  const int64_t warps = nr * H;
-  {
-    TraceScope ts("attn_combine", st);
-    sparse_attn_combine_kernel<D><<<(unsigned)ceil_div(warps, 8), 256, 0, st>>>(
-        part, p.splits, warps, out + row0 * H * (int64_t)D, lse ? lse + row0 * H : nullptr);
-  }
-  return after_launch();
-}
+constexpr int64_t kAttnRowsPerLaunch = 16384;
 
 csa2_status run_attn(const uint16_t *q, const uint8_t *codes, const float *scales,
                      const int32_t *idx, const uint16_t *win_k, const uint16_t *win_v, int32_t B,
                      int32_t T, int32_t H, int32_t D, int64_t N, int32_t topk, int32_t W,
-                     float sm_scale, float *out, float *lse, void *ws, size_t ws_bytes,
-                     cudaStream_t st) {
+                     float sm_scale, float *out, float *lse, cudaStream_t st) {
   const int64_t rows = int64_t(B) * T;
-  // Launch chunks start on sequence boundaries.
-  AttnPlan p = attn_plan(B, T, H, D, topk, W);
-  int64_t seq_per_launch = std::max<int64_t>(1, p.rows_per_launch / std::max(T, 1));
-  if (T > kAttnMaxRowsPerLaunch) return CSA2_ERR_UNSUPPORTED;
-  if (!ws || ws_bytes < p.part_bytes || !aligned(ws, 16)) return CSA2_ERR_WORKSPACE;
-  float *part = static_cast<float *>(ws);
-  const float q_scale = sm_scale * 1.4426950408889634f;
-  for (int64_t s0 = 0; s0 < B; s0 += seq_per_launch) {
-    const int64_t ns = std::min<int64_t>(seq_per_launch, B - s0);
-    const int64_t row0 = s0 * T, nr = ns * T;
-    csa2_status rc =
-        (D == 128) ? launch_attn<128>(p, row0, nr, q, codes, scales, idx, win_k, win_v, T, H, N,
-                                      topk, W, q_scale, part, out, lse, st)
-                   : launch_attn<64>(p, row0, nr, q, codes, scales, idx, win_k, win_v, T, H, N,
-                                     topk, W, q_scale, part, out, lse, st);
-    if (rc != CSA2_OK) return rc;
+  RowParams p{};
+  p.N = N;
+  p.T = T;
+  p.n_prior = -1;
+  p.ratio = 1;
+  p.topk = topk;
+  p.idx = const_cast<int32_t *>(idx);
+  p.q = q;
+  p.codes = codes;
+  p.scales = scales;
+  p.win_k = win_k;
+  p.win_v = win_v;
+  p.H = H;
+  p.W = W;
+  p.q_scale = sm_scale * 1.4426950408889634f;
+  p.out = out;
+  p.lse = lse;
+  p.do_topk = 0;
+  p.do_attn = 1;
+  for (int64_t row0 = 0; row0 < rows; row0 += kAttnRowsPerLaunch) {
+    const int64_t nr = std::min<int64_t>(kAttnRowsPerLaunch, rows - row0);
+    p.row0 = row0;
+    if (launch_row(p, D, nr, st) != CSA2_OK) return CSA2_ERR_CUDA;
   }
-  (void)rows;
   return CSA2_OK;
 }
 
@@ -426,13 +494,18 @@ csa2_status csa2_index_topk(const int8_t *q_idx, const float *w, const int8_t *k
                                    idx_out, score_out);
   if (rc != CSA2_OK || int64_t(B) * T == 0) return rc;
   return run_index_topk(q_idx, w, k_idx, B, T, H_I, d_I, N, n_prior, ratio, topk, idx_out,
-                        score_out, ws, ws_bytes, as_stream(stream));
+                        score_out, nullptr, ws, ws_bytes, as_stream(stream));
 }
 
 size_t csa2_sparse_attn_workspace_size(int32_t B, int32_t T, int32_t H, int32_t D, int32_t topk,
                                        int32_t W) {
-  if (B < 0 || T < 0 || H < 1 || (D != 64 && D != 128) || topk < 0 || W < 0) return 0;
-  return attn_plan(B, T, H, D, topk, W).part_bytes;
+  (void)B;
+  (void)T;
+  (void)H;
+  (void)D;
+  (void)topk;
+  (void)W;
+  return 0;  // partial softmax states are merged on chip
 }
 
 csa2_status csa2_sparse_attn_decode(const uint16_t *q, const uint8_t *codes, const float *scales,
@@ -440,11 +513,13 @@ csa2_status csa2_sparse_attn_decode(const uint16_t *q, const uint8_t *codes, con
                                     const uint16_t *win_v, int32_t B, int32_t H, int32_t D,
                                     int64_t N, int32_t topk, int32_t W, float sm_scale, float *out,
                                     float *lse, void *ws, size_t ws_bytes, void *stream) {
+  (void)ws;
+  (void)ws_bytes;
   csa2_status rc = check_attn_args(q, codes, scales, idx, win_k, win_v, B, 1, H, D, N, topk, W,
                                    out, lse);
   if (rc != CSA2_OK || B == 0) return rc;
   return run_attn(q, codes, scales, idx, win_k, win_v, B, 1, H, D, N, topk, W, sm_scale, out, lse,
-                  ws, ws_bytes, as_stream(stream));
+                  as_stream(stream));
 }
 
 csa2_status csa2_sparse_attn_prefill(const uint16_t *q, const uint8_t *codes, const float *scales,
@@ -453,11 +528,13 @@ csa2_status csa2_sparse_attn_prefill(const uint16_t *q, const uint8_t *codes, co
                                      int32_t D, int64_t N, int32_t topk, int32_t W,
                                      float sm_scale, float *out, float *lse, void *ws,
                                      size_t ws_bytes, void *stream) {
+  (void)ws;
+  (void)ws_bytes;
   csa2_status rc = check_attn_args(q, codes, scales, idx, win_k, win_v, B, T, H, D, N, topk, W,
                                    out, lse);
   if (rc != CSA2_OK || int64_t(B) * T == 0) return rc;
   return run_attn(q, codes, scales, idx, win_k, win_v, B, T, H, D, N, topk, W, sm_scale, out, lse,
-                  ws, ws_bytes, as_stream(stream));
+                  as_stream(stream));
 }
 
 csa2_status csa2_validate_modes(const csa2_layer_mode *modes, int32_t L) {
@@ -481,19 +558,21 @@ csa2_status csa2_group_cache_bytes(const csa2_layer_mode *modes, int32_t L, int6
 
 size_t csa2_layer_group_workspace_size(const csa2_dims *d) {
   if (!d) return 0;
-  const size_t a = csa2_index_topk_workspace_size(d->B, d->T, d->H_I, d->d_I, d->N, d->topk);
-  const size_t b = csa2_sparse_attn_workspace_size(d->B, d->T, d->H, d->D, d->topk, d->W);
-  if (a == 0 || b == 0) return 0;
-  return std::max(a, b);
+  if (d->B < 0 || d->T < 0 || d->H < 1 || (d->D != 64 && d->D != 128) || d->W < 0) return 0;
+  return csa2_index_topk_workspace_size(d->B, d->T, d->H_I, d->d_I, d->N, d->topk);
 }
 
-csa2_status csa2_layer_group_run(const csa2_layer_mode *modes, const csa2_layer_io *io, int32_t L,
-                                 const csa2_dims *d, void *ws, size_t ws_bytes, void *stream) {
+}  // extern "C"
+
+namespace {
+
+// Validate the table and the pointers of the layers in [l0, l1).
+csa2_status check_layers(const csa2_layer_mode *modes, const csa2_layer_io *io, int32_t L,
+                         int32_t l0, int32_t l1, const csa2_dims *d) {
   if (!io || !d) return CSA2_ERR_INVALID_ARG;
   csa2_status rc = check_modes(modes, L);
   if (rc != CSA2_OK) return rc;
-  // Validate every layer's pointers before enqueueing anything.
-  for (int32_t l = 0; l < L; ++l) {
+  for (int32_t l = l0; l < l1; ++l) {
     const csa2_layer_io &x = io[l];
     const csa2_layer_io &kv = io[modes[l].kv_src];
     const csa2_layer_io &ix = io[modes[l].idx_src];
@@ -506,22 +585,54 @@ csa2_status csa2_layer_group_run(const csa2_layer_mode *modes, const csa2_layer_
                          d->D, d->N, d->topk, d->W, x.out, x.lse);
     if (rc != CSA2_OK) return rc;
   }
+  return CSA2_OK;
+}
+
+csa2_status run_layer(const csa2_layer_mode *modes, const csa2_layer_io *io, int32_t l,
+                      const csa2_dims *d, void *ws, size_t ws_bytes, cudaStream_t st) {
+  const csa2_layer_io &x = io[l];
+  const csa2_layer_io &kv = io[modes[l].kv_src];
+  const csa2_layer_io &ix = io[modes[l].idx_src];
+  if (modes[l].mode != CSA2_REUSE) {
+    // Full / Reindex: scan this layer's index query over the kv store's keys,
+    // then select and attend in one per-row cluster kernel.
+    AttnArgs att{x.q, kv.codes, kv.scales, x.win_k, x.win_v, d->H, d->D, d->W, d->sm_scale,
+                 x.out, x.lse};
+    return run_index_topk(x.q_idx, x.w, kv.k_idx, d->B, d->T, d->H_I, d->d_I, d->N, d->n_prior,
+                          d->ratio, d->topk, x.idx, nullptr, &att, ws, ws_bytes, st);
+  }
+  // Reuse: attend with the source layer's selection.
+  return run_attn(x.q, kv.codes, kv.scales, ix.idx, x.win_k, x.win_v, d->B, d->T, d->H, d->D,
+                  d->N, d->topk, d->W, d->sm_scale, x.out, x.lse, st);
+}
+
+}  // namespace
+
+extern "C" {
+
+csa2_status csa2_layer_run(const csa2_layer_mode *modes, const csa2_layer_io *io, int32_t L,
+                           int32_t layer, const csa2_dims *d, void *ws, size_t ws_bytes,
+                           void *stream) {
+  if (layer < 0 || layer >= L) return CSA2_ERR_INVALID_ARG;
+  csa2_status rc = check_layers(modes, io, L, layer, layer + 1, d);
+  if (rc != CSA2_OK) return rc;
   if (int64_t(d->B) * d->T == 0) return CSA2_OK;
   const size_t need = csa2_layer_group_workspace_size(d);
   if (need == 0) return CSA2_ERR_UNSUPPORTED;
   if (!ws || ws_bytes < need || !aligned(ws, 16)) return CSA2_ERR_WORKSPACE;
-  cudaStream_t st = as_stream(stream);
+  return run_layer(modes, io, layer, d, ws, ws_bytes, as_stream(stream));
+}
+
+csa2_status csa2_layer_group_run(const csa2_layer_mode *modes, const csa2_layer_io *io, int32_t L,
+                                 const csa2_dims *d, void *ws, size_t ws_bytes, void *stream) {
+  csa2_status rc = check_layers(modes, io, L, 0, L, d);
+  if (rc != CSA2_OK) return rc;
+  if (int64_t(d->B) * d->T == 0) return CSA2_OK;
+  const size_t need = csa2_layer_group_workspace_size(d);
+  if (need == 0) return CSA2_ERR_UNSUPPORTED;
+  if (!ws || ws_bytes < need || !aligned(ws, 16)) return CSA2_ERR_WORKSPACE;
   for (int32_t l = 0; l < L; ++l) {
-    const csa2_layer_io &x = io[l];
-    const csa2_layer_io &kv = io[modes[l].kv_src];
-    const csa2_layer_io &ix = io[modes[l].idx_src];
-    if (modes[l].mode != CSA2_REUSE) {
-      rc = run_index_topk(x.q_idx, x.w, kv.k_idx, d->B, d->T, d->H_I, d->d_I, d->N, d->n_prior,
-                          d->ratio, d->topk, x.idx, nullptr, ws, ws_bytes, st);
-      if (rc != CSA2_OK) return rc;
-    }
-    rc = run_attn(x.q, kv.codes, kv.scales, ix.idx, x.win_k, x.win_v, d->B, d->T, d->H, d->D,
-                  d->N, d->topk, d->W, d->sm_scale, x.out, x.lse, ws, ws_bytes, st);
+    rc = run_layer(modes, io, l, d, ws, ws_bytes, as_stream(stream));
     if (rc != CSA2_OK) return rc;
   }
   return CSA2_OK;

@@ -1,4 +1,4 @@
-// Indexer scan (decode and small-T queries): score every visible entry.
+// Indexer scan: score every visible entry of a query row.
 //
 // "Why Is DeepSeek V4.1 Flash So Fast?", section 4 ("The indexer"): index
 // heads run a cheap relevance search over all compressed positions.  Score
@@ -6,16 +6,19 @@
 //   dot_h = sum_i q_idx[r, h, i] * k_idx[b, n, i]        exact int32 (dp4a)
 //   score = ((0 + w_0 * dot_0) + w_1 * dot_1) + ... + 0   fp32, each op rounded
 //
-// Layout and data movement.  Keys are int8 [B, N, d_I]; a key is d_I/16
-// 16-byte chunks.  Each warp load instruction reads 512 contiguous bytes
-// (lane l: bytes 16l .. 16l+15), so the lanes of one key hold its chunks.
-// A warp issues NCH loads (NCH = d_I/16) per 32-key group, each lane forms
-// per-head partial dot products of its chunk, and a butterfly
-// reduce-scatter across the NCH lanes of a key leaves lane l holding the
-// complete per-head dots of exactly one key.  That lane then forms the fp32
-// score, writes it, and adds the key's top radix digit to a shared-memory
-// histogram (merged into the row's global histogram at the end), which the
-// top-k selection uses to find its threshold without another pass.
+// Data movement.  The scan is HBM-bound (d_I bytes per entry, a few hundred
+// integer ops), so it streams keys, it does not reshape them into a GEMM.
+// Each CTA owns a contiguous slice of one row's entries and pulls it through
+// a STAGES-deep ring of shared-memory tiles with 1-D bulk copies
+// (cp.async.bulk, completion counted on an mbarrier); one elected thread
+// issues the copies, so loads cost no per-thread address arithmetic.  Each
+// thread scores whole keys from shared memory.  A key is d_I/16 chunks of 16
+// bytes; thread t reads chunk c ^ x(t) at step c, with x(t) chosen so the 8
+// threads of a 128-byte shared-memory phase hit 8 different 16-byte bank
+// groups, and holds its index-query chunks pre-permuted the same way, so the
+// dot product needs no data-dependent register indexing.  The score's top
+// radix digit goes to a shared-memory histogram (warp-aggregated), merged
+// into the row's global histogram at the end for the top-k selection.
 #pragma once
 #include "common.cuh"
 
@@ -25,32 +28,38 @@ constexpr int kScanThreads = 256;
 
 template <int DI, int HI>
 struct ScanShape {
-  static constexpr int NCH = DI / 16;     // 16-byte chunks (= lanes) per key
-  static constexpr int KPL = 32 / NCH;    // keys covered by one warp load
-  // 32-key groups a warp processes per iteration: at least 8 loads of
-  // 16 bytes per lane in flight (4 KB per warp).
-  static constexpr int GROUPS = (NCH >= 8) ? 1 : 8 / NCH;
-  static constexpr int KEYS_PER_ITER = 32 * GROUPS;
+  static constexpr int NCH = DI / 16;                     // 16-byte chunks per key
+  static constexpr int KPT = (DI >= 64) ? 1 : 64 / DI;    // keys per thread per tile
+  static constexpr int TILE_KEYS = kScanThreads * KPT;
+  static constexpr int TILE_BYTES = TILE_KEYS * DI;       // 16 KiB (32 KiB for d_I = 128)
+  static constexpr int STAGES = (TILE_BYTES > 16384) ? 3 : 4;
+  static constexpr bool QREG = HI * NCH <= 16;            // index query fits in registers
+  static constexpr size_t SMEM = size_t(STAGES) * TILE_BYTES;
   static_assert(DI % 16 == 0 && NCH >= 1 && NCH <= 8, "d_I in {16,32,64,128}");
-  static_assert(HI * NCH <= 32, "register budget of the per-lane partials");
 };
 
-__device__ __forceinline__ int dp4a(int a, int b, int c) { return __dp4a(a, b, c); }
+// Rotation of the chunk order of thread t (see the header comment).
+template <int NCH>
+__device__ __forceinline__ int chunk_xor(int t) {
+  return (NCH == 1) ? 0 : (t / (8 / NCH)) % NCH;
+}
 
-// grid = (G slices, rows); rows = B * T query rows.
+// grid = (G slices, rows).
 template <int DI, int HI>
-__global__ void __launch_bounds__(kScanThreads, 3)
+__global__ void __launch_bounds__(kScanThreads, 2)
     index_scan_kernel(const int8_t *__restrict__ q_idx, const float *__restrict__ w,
                       const int8_t *__restrict__ k_idx, int32_t T, int64_t N, int64_t n_prior,
                       int32_t ratio, int64_t row0, float *__restrict__ scores,
-                      uint32_t *__restrict__ hist1, int write_masked) {
+                      int64_t score_stride, uint32_t *__restrict__ hist1, int write_masked) {
   using S = ScanShape<DI, HI>;
-  constexpr int NCH = S::NCH, KPL = S::KPL, GROUPS = S::GROUPS;
+  constexpr int NCH = S::NCH, STAGES = S::STAGES, TK = S::TILE_KEYS;
+  extern __shared__ __align__(128) unsigned char smem_tiles[];
+  __shared__ uint64_t full_bar[STAGES];
   __shared__ uint32_t sh_hist[kBins1];
+  __shared__ __align__(16) int4 sh_q[S::QREG ? 1 : HI * NCH];
 
-  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  const int64_t r_local = blockIdx.y;       // row within this launch
-  const int64_t r = row0 + r_local;         // global query row b*T + t
+  const int tid = threadIdx.x, lane = tid & 31;
+  const int64_t r_local = blockIdx.y, r = row0 + r_local;
   const int64_t b = r / T, t = r % T;
   const int G = gridDim.x, g = blockIdx.x;
 
@@ -59,83 +68,118 @@ __global__ void __launch_bounds__(kScanThreads, 3)
     V = n_prior + (t + 1) / ratio;
     if (V > N) V = N;
   }
+  // Slice [n0, n1) of [0, V); inner boundaries on multiples of 16 keys.
+  const int64_t n0 = ((V * g) / G) & ~int64_t(15);
+  const int64_t n1 = (g == G - 1) ? V : (((V * (g + 1)) / G) & ~int64_t(15));
+  const int ntiles = (int)((n1 - n0 + TK - 1) / TK);
+  const int8_t *src = k_idx + (b * N + n0) * DI;
 
   for (int i = tid; i < kBins1; i += kScanThreads) sh_hist[i] = 0u;
-
-  // Slice [n0, n1) of [0, V), boundaries on 32-key multiples.
-  int64_t n0 = ((V * g) / G) & ~int64_t(31);
-  int64_t n1 = (g == G - 1) ? V : (((V * (g + 1)) / G) & ~int64_t(31));
-
-  // This lane's chunk of every head's index query, and the head weights.
-  const int c = lane % NCH;
-  int4 qv[HI];
-  float wh[HI];
-#pragma unroll
-  for (int h = 0; h < HI; ++h) {
-    qv[h] = *reinterpret_cast<const int4 *>(q_idx + (r * HI + h) * DI + c * 16);
-    wh[h] = w[r * HI + h];
+  if (tid == 0) {
+    for (int s = 0; s < STAGES; ++s) mbar_init(&full_bar[s], 1);
+    fence_barrier_init();
   }
   __syncthreads();
+  if (tid == 0) {
+    for (int s = 0; s < STAGES && s < ntiles; ++s) {
+      const int64_t keys = min64(TK, n1 - n0 - (int64_t)s * TK);
+      const uint32_t bytes = (uint32_t)(keys * DI);
+      mbar_arrive_expect_tx(&full_bar[s], bytes);
+      bulk_g2s(smem_tiles + s * S::TILE_BYTES, src + (int64_t)s * TK * DI, bytes, &full_bar[s]);
+    }
+  }
 
-  const int8_t *keys = k_idx + b * N * DI;
-  float *srow = scores + r_local * N;
-  const int NW = kScanThreads / 32;
+  // This thread's index-query chunks, pre-permuted by its chunk rotation.
+  const int x = chunk_xor<NCH>(tid);
+  int4 qreg[S::QREG ? HI * NCH : 1];
+  const int4 *qrow = reinterpret_cast<const int4 *>(q_idx + r * HI * DI);
+  if constexpr (S::QREG) {
+#pragma unroll
+    for (int h = 0; h < HI; ++h)
+#pragma unroll
+      for (int c = 0; c < NCH; ++c) qreg[h * NCH + c] = qrow[h * NCH + (c ^ x)];
+  } else {
+    for (int i = tid; i < HI * NCH; i += kScanThreads) sh_q[i] = qrow[i];
+  }
+  float wh[HI];
+#pragma unroll
+  for (int h = 0; h < HI; ++h) wh[h] = w[r * HI + h];
+  if constexpr (!S::QREG) __syncthreads();
 
-  for (int64_t base = n0 + (int64_t)warp * S::KEYS_PER_ITER; base < n1;
-       base += (int64_t)NW * S::KEYS_PER_ITER) {
-    // ---- loads: GROUPS x NCH loads of 16 bytes per lane ----
-    int4 kv[GROUPS][NCH];
+  float *srow = scores + r_local * score_stride;
+  int abort_it = -1;
+  for (int it = 0; it < ntiles; ++it) {
+    const int s = it % STAGES;
+    const bool ok = mbar_wait_bounded(&full_bar[s], (uint32_t)(it / STAGES) & 1u);
+    // One barrier per tile: uniform abort decision, and every thread is done
+    // with tile it-1, so its stage can be refilled with tile it-1+STAGES.
+    if (__syncthreads_or(!ok)) {
+      abort_it = it;
+      break;
+    }
+    if (tid == 0 && it >= 1 && it - 1 + STAGES < ntiles) {
+      const int nt = it - 1 + STAGES, ps = (it - 1) % STAGES;
+      const int64_t keys = min64(TK, n1 - n0 - (int64_t)nt * TK);
+      const uint32_t bytes = (uint32_t)(keys * DI);
+      asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+      mbar_arrive_expect_tx(&full_bar[ps], bytes);
+      bulk_g2s(smem_tiles + ps * S::TILE_BYTES, src + (int64_t)nt * TK * DI, bytes,
+               &full_bar[ps]);
+    }
+    const unsigned char *tile = smem_tiles + s * S::TILE_BYTES;
+    const int64_t tbase = n0 + (int64_t)it * TK;
+    const int tkeys = (int)min64(TK, n1 - tbase);
 #pragma unroll
-    for (int gr = 0; gr < GROUPS; ++gr)
+    for (int j = 0; j < S::KPT; ++j) {
+      const int kl = tid + j * kScanThreads;
+      const bool valid = kl < tkeys;
+      float score = 0.0f;
+      if (valid) {
+        const unsigned char *krow = tile + kl * DI;
+        int dot[HI];
 #pragma unroll
-      for (int u = 0; u < NCH; ++u) {
-        const int64_t key = base + gr * 32 + u * KPL + lane / NCH;
-        if (key < n1)
-          kv[gr][u] = ld_stream_v4(keys + key * DI + c * 16);
-        else
-          kv[gr][u] = make_int4(0, 0, 0, 0);
-      }
+        for (int h = 0; h < HI; ++h) dot[h] = 0;
 #pragma unroll
-    for (int gr = 0; gr < GROUPS; ++gr) {
-      // ---- per-lane partial dots of its chunk ----
-      int p[NCH][HI];
-#pragma unroll
-      for (int u = 0; u < NCH; ++u)
-#pragma unroll
-        for (int h = 0; h < HI; ++h) {
-          int a = dp4a(kv[gr][u].x, qv[h].x, 0);
-          a = dp4a(kv[gr][u].y, qv[h].y, a);
-          a = dp4a(kv[gr][u].z, qv[h].z, a);
-          p[u][h] = dp4a(kv[gr][u].w, qv[h].w, a);
-        }
-      // ---- reduce-scatter over the NCH lanes of each key ----
-#pragma unroll
-      for (int m = NCH / 2; m >= 1; m >>= 1) {
-        const bool upper = (c & m) != 0;
-#pragma unroll
-        for (int i = 0; i < m; ++i)
+        for (int c = 0; c < NCH; ++c) {
+          const int4 kv = *reinterpret_cast<const int4 *>(krow + ((c ^ x) << 4));
 #pragma unroll
           for (int h = 0; h < HI; ++h) {
-            const int send = upper ? p[i][h] : p[i + m][h];
-            const int keep = upper ? p[i + m][h] : p[i][h];
-            p[i][h] = keep + __shfl_xor_sync(0xffffffffu, send, m);
+            int4 qv;
+            if constexpr (S::QREG)
+              qv = qreg[h * NCH + c];
+            else
+              qv = sh_q[h * NCH + (c ^ x)];
+            dot[h] = __dp4a(kv.x, qv.x, dot[h]);
+            dot[h] = __dp4a(kv.y, qv.y, dot[h]);
+            dot[h] = __dp4a(kv.z, qv.z, dot[h]);
+            dot[h] = __dp4a(kv.w, qv.w, dot[h]);
           }
-      }
-      // lane now holds the dots of key (c * KPL + lane / NCH) of this group
-      const int64_t key = base + gr * 32 + c * KPL + lane / NCH;
-      const bool valid = key < n1;
-      float acc = 0.0f;
+        }
+        float acc = 0.0f;
 #pragma unroll
-      for (int h = 0; h < HI; ++h) acc = __fadd_rn(acc, __fmul_rn(wh[h], __int2float_rn(p[0][h])));
-      const float score = __fadd_rn(acc, 0.0f);
+        for (int h = 0; h < HI; ++h) acc = __fadd_rn(acc, __fmul_rn(wh[h], __int2float_rn(dot[h])));
+        score = __fadd_rn(acc, 0.0f);
+        srow[tbase + kl] = score;
+      }
       const uint32_t bin = key_d1(score_key(score));
-      if (valid) srow[key] = score;
       const uint32_t active = __ballot_sync(0xffffffffu, valid);
       if (valid) {
         const uint32_t peers = __match_any_sync(active, bin);
         if (lane == __ffs(peers) - 1) atomicAdd(&sh_hist[bin], __popc(peers));
       }
     }
+  }
+  if (abort_it >= 0) {
+    // Drain the copies this CTA issued (tiles [0, upto)) before exiting.
+    if (tid == 0) {
+      const int upto = min(ntiles, max(abort_it - 1, 0) + STAGES);
+      for (int k = 0; k < STAGES && k < upto; ++k) {
+        const int last = k + ((upto - 1 - k) / STAGES) * STAGES;  // last tile issued into stage k
+        mbar_wait_bounded(&full_bar[k], (uint32_t)(last / STAGES) & 1u);
+      }
+    }
+    __syncthreads();
+    return;
   }
 
   // Entries the row may not see (prefill): -inf when scores are requested.

@@ -137,7 +137,7 @@ size_t csa2_index_topk_workspace_size(int32_t B, int32_t T, int32_t H_I, int32_t
  *   score_out device, fp32 [B, T, N] or NULL       (optional output: the
  *             score of every entry, -inf where the query may not see it)
  *   ws        device workspace of ws_bytes >= csa2_index_topk_workspace_size
- * Supported: d_I in {16, 32, 64, 128}, H_I in {1, 2, 4, 8}, H_I * d_I <= 256,
+ * Supported: d_I in {16, 32, 64, 128}, H_I in {1, 2, 4, 8}, H_I * d_I <= 512,
  * 1 <= topk <= 65536, N < 2^31, ratio >= 1 when n_prior >= 0. */
 csa2_status csa2_index_topk(const int8_t *q_idx, const float *w, const int8_t *k_idx, int32_t B,
                             int32_t T, int32_t H_I, int32_t d_I, int64_t N, int64_t n_prior,
@@ -148,8 +148,9 @@ csa2_status csa2_index_topk(const int8_t *q_idx, const float *w, const int8_t *k
 /* Sparse attention over the selected entries + the local window           */
 /* ---------------------------------------------------------------------- */
 
-/* Workspace bytes for csa2_sparse_attn_decode / _prefill (0 on invalid
- * sizes). */
+/* Workspace bytes for csa2_sparse_attn_decode / _prefill.  The current
+ * kernels merge their partial softmax states on chip and need none (0);
+ * ws may then be NULL. */
 size_t csa2_sparse_attn_workspace_size(int32_t B, int32_t T, int32_t H, int32_t D, int32_t topk,
                                        int32_t W);
 
@@ -235,8 +236,15 @@ csa2_status csa2_group_cache_bytes(const csa2_layer_mode *modes, int32_t L, int6
                                    int64_t numbers_per_entry, int64_t bits_per_number,
                                    uint64_t *bytes_out);
 
-/* Workspace bytes for csa2_layer_group_run. */
+/* Workspace bytes for csa2_layer_group_run and csa2_layer_run. */
 size_t csa2_layer_group_workspace_size(const csa2_dims *dims);
+
+/* Run only layer `layer` (0 <= layer < L) of the table, exactly as
+ * csa2_layer_group_run runs it (the table is validated whole; `layer`'s
+ * sources must already hold their outputs when it reads them). */
+csa2_status csa2_layer_run(const csa2_layer_mode *modes, const csa2_layer_io *io, int32_t L,
+                           int32_t layer, const csa2_dims *dims, void *ws, size_t ws_bytes,
+                           void *stream);
 
 /* Run L layers in table order on one stream: Full and Reindex layers run
  * the index + Top-K step over their kv_src store's index keys with their
