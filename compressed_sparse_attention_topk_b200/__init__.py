@@ -31,7 +31,7 @@ EXPORTED = (
     "csa2_sparse_attn_decode", "csa2_sparse_attn_prefill", "csa2_validate_modes",
     "csa2_group_cache_bytes", "csa2_layer_group_workspace_size", "csa2_layer_group_run",
     "csa2_get_device_status", "csa2_trace_enable", "csa2_trace_count", "csa2_trace_get",
-    "csa2_layer_run",
+    "csa2_layer_run", "csa2_index_topk_noalloc",
 )
 
 
@@ -89,6 +89,8 @@ def lib() -> ctypes.CDLL:
         "csa2_layer_group_workspace_size": ([P], sz),
         "csa2_layer_group_run": ([P, P, i32, P, P, sz, P], i32),
         "csa2_layer_run": ([P, P, i32, i32, P, P, sz, P], i32),
+        "csa2_index_topk_noalloc": ([P, P, P, i32, i32, i32, i32, i64, i64, i32, i32, P, P, P],
+                                    i32),
         "csa2_get_device_status": ([P, P], i32),
         "csa2_trace_enable": ([i32], i32),
         "csa2_trace_count": ([], i32),

@@ -655,6 +655,56 @@ csa2_status csa2_trace_get(int32_t i, const char **name, float *ms) {
   return CSA2_OK;
 }
 
+}  // extern "C"
+
+// ---------------------------------------------------------------------------
+// Index + top-k for callers that cannot allocate device memory.
+// ---------------------------------------------------------------------------
+// Fixed scratch in the library's own device memory: every GPU that loads the
+// library keeps these 16 MiB until the process exits.  All calls share it.
+constexpr size_t kNoAllocScratchBytes = size_t(16) << 20;
+static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocScratchBytes];
+
+namespace {
+
+// Device address of the scratch on the current device, looked up once per
+// device (the name itself is only a host-side stand-in).
+void *noalloc_scratch(csa2_status *rc) {
+  static void *addr[256] = {nullptr};
+  int dev = -1;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 256) {
+    *rc = CSA2_ERR_CUDA;
+    return nullptr;
+  }
+  if (!addr[dev]) {
+    void *ptr = nullptr;
+    if (cudaGetSymbolAddress(&ptr, g_noalloc_scratch) != cudaSuccess || !ptr) {
+      *rc = CSA2_ERR_CUDA;
+      return nullptr;
+    }
+    addr[dev] = ptr;
+  }
+  return addr[dev];
+}
+
+}  // namespace
+
+extern "C" {
+
+csa2_status csa2_index_topk_noalloc(const int8_t *q_idx, const float *w, const int8_t *k_idx,
+                                    int32_t B, int32_t T, int32_t H_I, int32_t d_I, int64_t N,
+                                    int64_t n_prior, int32_t ratio, int32_t topk,
+                                    int32_t *idx_out, float *score_out, void *stream) {
+  csa2_status rc = check_topk_args(q_idx, w, k_idx, B, T, H_I, d_I, N, n_prior, ratio, topk,
+                                   idx_out, score_out);
+  if (rc != CSA2_OK || int64_t(B) * T == 0) return rc;
+  if (topk_ws_bytes(B, T, N) > kNoAllocScratchBytes) return CSA2_ERR_UNSUPPORTED;
+  void *ws = noalloc_scratch(&rc);
+  if (!ws) return rc;
+  return run_index_topk(q_idx, w, k_idx, B, T, H_I, d_I, N, n_prior, ratio, topk, idx_out,
+                        score_out, nullptr, ws, kNoAllocScratchBytes, as_stream(stream));
+}
+
 csa2_status csa2_get_device_status(void *stream, int32_t *code_out) {
   if (cudaStreamSynchronize(as_stream(stream)) != cudaSuccess) return CSA2_ERR_CUDA;
   uint32_t v = 0, zero = 0;

@@ -144,6 +144,29 @@ csa2_status csa2_index_topk(const int8_t *q_idx, const float *w, const int8_t *k
                             int32_t ratio, int32_t topk, int32_t *idx_out, float *score_out,
                             void *ws, size_t ws_bytes, void *stream);
 
+/* Same computation and results as csa2_index_topk, for callers that cannot
+ * allocate device memory: e.g. a host runtime that owns all device memory
+ * through its own allocator and hands extensions no workspace, or a serving
+ * loop that must not allocate after start-up because an allocation there
+ * could fail or stall at the wrong moment.  The pages describe no such call;
+ * it has no counterpart there.
+ * Scratch comes from a fixed 16 MiB array inside the library (held on every
+ * GPU that loads the library until the process exits); this call allocates
+ * nothing itself.  Sizes whose scratch would exceed it
+ * (csa2_index_topk_workspace_size(...) > 16 MiB) return CSA2_ERR_UNSUPPORTED
+ * before anything is enqueued.  The first call on a device looks up the
+ * array's device address and sets kernel attributes; make that first call
+ * before any stream capture.  All calls share the one array and leave their
+ * contents in it (the parts that must start at zero are cleared by each
+ * call), so calls that overlap on the GPU -- on different streams, or from
+ * several host threads -- race and corrupt each other's results: serialise
+ * them.  Keep the kernel timing trace off (its default).  Arguments as for
+ * csa2_index_topk, without ws / ws_bytes. */
+csa2_status csa2_index_topk_noalloc(const int8_t *q_idx, const float *w, const int8_t *k_idx,
+                                    int32_t B, int32_t T, int32_t H_I, int32_t d_I, int64_t N,
+                                    int64_t n_prior, int32_t ratio, int32_t topk,
+                                    int32_t *idx_out, float *score_out, void *stream);
+
 /* ---------------------------------------------------------------------- */
 /* Sparse attention over the selected entries + the local window           */
 /* ---------------------------------------------------------------------- */
