@@ -111,6 +111,18 @@ __device__ __forceinline__ void bulk_g2s(void *smem_dst, const void *gmem_src, u
 }
 
 // ---------------------------------------------------------------------------
+// Programmatic dependent launch: a kernel launched with programmatic stream
+// serialisation may start before the previous kernel on its stream ends;
+// it must wait before reading that kernel's results.
+// ---------------------------------------------------------------------------
+__device__ __forceinline__ void pdl_wait_primary() {
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+}
+__device__ __forceinline__ void pdl_allow_dependents() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
+// ---------------------------------------------------------------------------
 // Warp / block reductions and scans.
 // ---------------------------------------------------------------------------
 __device__ __forceinline__ float warp_max(float v) {

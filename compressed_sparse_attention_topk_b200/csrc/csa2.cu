@@ -190,13 +190,16 @@ csa2_status launch_row_cl(const RowParams &p, int64_t nr, cudaStream_t st) {
   cfg.blockDim = dim3(kRowThreads, 1, 1);
   cfg.dynamicSmemBytes = smem;
   cfg.stream = st;
-  cudaLaunchAttribute attr[1];
+  cudaLaunchAttribute attr[2];
   attr[0].id = cudaLaunchAttributeClusterDimension;
   attr[0].val.clusterDim.x = CL;
   attr[0].val.clusterDim.y = 1;
   attr[0].val.clusterDim.z = 1;
+  // After a scan, start early: the kernel waits for the scan's results itself.
+  attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[1].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
-  cfg.numAttrs = 1;
+  cfg.numAttrs = p.do_topk ? 2 : 1;
   return cudaLaunchKernelEx(&cfg, row_cluster_kernel<D, CL>, p) == cudaSuccess ? CSA2_OK
                                                                                 : CSA2_ERR_CUDA;
 }

@@ -74,6 +74,9 @@ __global__ void __launch_bounds__(kScanThreads, 2)
   const int ntiles = (int)((n1 - n0 + TK - 1) / TK);
   const int8_t *src = k_idx + (b * N + n0) * DI;
 
+  // The per-row selection kernel that follows may be scheduled now; it waits
+  // for this grid's results before reading them.
+  pdl_allow_dependents();
   for (int i = tid; i < kBins1; i += kScanThreads) sh_hist[i] = 0u;
   if (tid == 0) {
     for (int s = 0; s < STAGES; ++s) mbar_init(&full_bar[s], 1);

@@ -114,6 +114,7 @@ struct RowSmem {
   int32_t sel[kSelCap];         // this CTA's selected indices, ascending
   int32_t raw_idx[kRawCap];     // entries of the gathered batch
   uint32_t wa[kRowWarps], wb[kRowWarps], wc[kRowWarps], wd[kRowWarps];
+  uint32_t masks[kRowWarps][kStageScores / kRowWarps / 32];  // per-warp ballots of a round
   // attention
   uint16_t kb[kChunkKeys][D + 8];   // keys, row-major bf16 (+8: conflict-free B loads)
   uint16_t vt[D][kChunkKeys + 8];   // values, transposed bf16
@@ -233,22 +234,30 @@ __device__ void row_topk(RowSmem<D> &sm, const RowParams &p, cg::cluster_group &
       }
       __syncthreads();
     }
+    // one ballot per 32 elements of the warp's segment, kept in shared memory
     const int seg0 = (n * warp) / kRowWarps, seg1 = (n * (warp + 1)) / kRowWarps;
+    constexpr int STEPS = kStageScores / kRowWarps / 32;
     uint32_t mine = 0;
 #pragma unroll 8
-    for (int i = seg0 + lane; i < seg1; i += 32) mine += key_d1(score_key(sm.st.sc[i])) >= t1;
-    mine = __reduce_add_sync(0xffffffffu, mine);
+    for (int j = 0; j < STEPS; ++j) {
+      const int i = seg0 + 32 * j + lane;
+      const bool in = (i < seg1) && key_d1(score_key(sm.st.sc[i])) >= t1;
+      const uint32_t bal = __ballot_sync(0xffffffffu, in);
+      if (lane == (j & 31)) sm.masks[warp][j] = bal;
+      mine += __popc(bal);
+    }
     if (lane == 0) sm.wa[warp] = mine;
     __syncthreads();
     if (warp == 0) warp0_prefix16(sm.wa, sm.wb, &sm.scratch[0]);
     __syncthreads();
+    // write pass: only the steps that hold candidates
     uint32_t pos = count + sm.wb[warp];
-    for (int i0 = seg0; i0 < seg1; i0 += 32) {
-      const int i = i0 + lane;
-      const uint32_t key = (i < seg1) ? score_key(sm.st.sc[i]) : 0u;
-      const bool in = (i < seg1) && key_d1(key) >= t1;
-      const uint32_t bal = __ballot_sync(0xffffffffu, in);
-      if (in) {
+    for (int j = 0; j < STEPS; ++j) {
+      const uint32_t bal = sm.masks[warp][j];
+      if (bal == 0u) continue;  // warp-uniform
+      if ((bal >> lane) & 1u) {
+        const int i = seg0 + 32 * j + lane;
+        const uint32_t key = score_key(sm.st.sc[i]);
         const uint32_t at = pos + __popc(bal & lt);
         const uint2 e = make_uint2(key, (uint32_t)(rb - s0 + i));
         if (at < (uint32_t)kCandCap)
@@ -604,9 +613,13 @@ __device__ void attend_chunk(RowSmem<D> &sm, const RowParams &p, AttnState &st, 
 
 template <int D>
 __device__ void load_q(RowSmem<D> &sm, const RowParams &p, int64_t r, int h0, int nh) {
-  for (int i = threadIdx.x; i < kHeads * D; i += kRowThreads) {
-    const int h = i / D, d = i % D;
-    sm.qb[h][d] = (h < nh) ? p.q[(r * p.H + h0 + h) * (int64_t)D + d] : (uint16_t)0;
+  // 16-byte pieces: 16 heads x D/8 pieces
+  constexpr int PPH = D / 8;
+  for (int i = threadIdx.x; i < kHeads * PPH; i += kRowThreads) {
+    const int h = i / PPH, u = i % PPH;
+    uint4 v = make_uint4(0u, 0u, 0u, 0u);
+    if (h < nh) v = *reinterpret_cast<const uint4 *>(p.q + (r * p.H + h0 + h) * (int64_t)D + 8 * u);
+    *reinterpret_cast<uint4 *>(&sm.qb[h][8 * u]) = v;
   }
 }
 
@@ -757,8 +770,16 @@ __global__ void __launch_bounds__(kRowThreads, 1) row_cluster_kernel(const RowPa
     fence_barrier_init();
   }
   __syncthreads();
-  // Prologue: issue the top-k inputs, then do the window part of attention
-  // while they arrive.
+  // Prologue, independent of the scan that produced the scores: the query and
+  // the window part of attention.  With programmatic dependent launch this
+  // overlaps the scan's tail.
+  for (int i = tid; i < kBins2; i += kRowThreads) sm.h2[i] = 0u;
+  AttnState st{{0.0f, 0.0f, 0.0f, 0.0f}, -INFINITY, 0.0f};
+  if (p.do_attn) {
+    load_q<D>(sm, p, r, 0, min(kHeads, p.H));
+    attend_window<D, CL>(sm, p, st, r, c, min(kHeads, p.H));
+  }
+  pdl_wait_primary();  // the scores and histograms are complete from here on
   if (topk_here && tid == 0) {
     const int n0 = (int)min64(kStageScores, s1 - s0);
     uint32_t bytes = kBins1 * 4;
@@ -768,12 +789,6 @@ __global__ void __launch_bounds__(kRowThreads, 1) row_cluster_kernel(const RowPa
     if (bulk && n0 > 0)
       bulk_g2s(sm.st.sc, p.scores + r_local * p.score_stride + s0,
                (uint32_t)(((n0 + 3) & ~3) * 4), &sm.bar);
-  }
-  for (int i = tid; i < kBins2; i += kRowThreads) sm.h2[i] = 0u;
-  AttnState st{{0.0f, 0.0f, 0.0f, 0.0f}, -INFINITY, 0.0f};
-  if (p.do_attn) {
-    load_q<D>(sm, p, r, 0, min(kHeads, p.H));
-    attend_window<D, CL>(sm, p, st, r, c, min(kHeads, p.H));
   }
 
   bool abort = false;
