@@ -462,13 +462,69 @@ def run_gpu(args, w0):
     return 0
 
 
+def run_prefill(args, w0):
+    """Supplementary measurement of a chunked-prefill layer (index + top-k
+    over the visible prefix of every query, then attention), one GPU."""
+    import torch
+    import compressed_sparse_attention_topk_b200 as csa2
+    torch.cuda.set_device(0)
+    dev = torch.device("cuda", 0)
+    csa2.lib()
+    lay = wl.layer_inputs(w0, 0)
+
+    def to_dev(a):
+        a = np.ascontiguousarray(a)
+        if a.dtype == np.uint16:
+            return torch.from_numpy(a.view(np.int16)).to(dev).view(torch.bfloat16)
+        return torch.from_numpy(a).to(dev)
+
+    t = {k: to_dev(lay[k]) for k in ("q", "q_idx", "w", "win_k", "win_v", "k_idx")}
+    src = to_dev(lay["entries"])
+    t["codes"], t["scales"] = csa2.pack_fp4(src)
+    del src
+    t["idx"] = torch.empty((w0.B, w0.T, w0.topk), dtype=torch.int32, device=dev)
+    t["out"] = torch.empty((w0.B, w0.T, w0.H, w0.D), dtype=torch.float32, device=dev)
+    t["lse"] = torch.empty((w0.B, w0.T, w0.H), dtype=torch.float32, device=dev)
+    dims = csa2.make_dims(w0.B, w0.T, w0.H, w0.D, w0.N, w0.H_I, w0.d_I, w0.topk, w0.W,
+                          w0.n_prior, w0.ratio, w0.sm_scale)
+    group = csa2.LayerGroup([(0, 0, 0)], [t], dims)
+    for _ in range(max(args.warmup, 1)):
+        group.run_layer(0)
+    torch.cuda.synchronize()
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a.record()
+    for _ in range(args.steps):
+        group.run_layer(0)
+    b.record()
+    torch.cuda.synchronize()
+    ms = a.elapsed_time(b) / args.steps
+    csa2.trace_enable(True)
+    group.run_layer(0)
+    recs = csa2.trace_records()
+    csa2.trace_enable(False)
+    per = {}
+    for name, m in recs:
+        c, s_ = per.get(name, (0, 0.0))
+        per[name] = (c + 1, s_ + m)
+    print(json.dumps({
+        "metric": "CSA2 chunked-prefill tokens/s per layer (supplementary)",
+        "value": w0.B * w0.T / (ms * 1e-3), "unit": "tokens/s/layer", "ms_per_layer": ms,
+        "steps": args.steps, "config": {"workload": w0.name, "T": w0.T, "N": w0.N,
+                                          "n_prior": w0.n_prior, "topk": w0.topk},
+        "kernels": {k: {"launches": c, "total_ms": s_} for k, (c, s_) in per.items()},
+    }), flush=True)
+    return 0
+
+
 def main():
     args = parse_args()
     w0 = wl.ALL[args.workload]
-    if w0.T != 1 or w0.n_prior >= 0:
-        raise SystemExit("bench.py times decode workloads (T == 1)")
     if args.impl == "reference":
+        if w0.T != 1:
+            raise SystemExit("the reference leg times decode workloads")
         return run_reference(args, w0)
+    if w0.T != 1 or w0.n_prior >= 0:
+        return run_prefill(args, w0)
     return run_gpu(args, w0)
 
 
