@@ -10,6 +10,7 @@
 #include "common.cuh"
 #include "index_scan.cuh"
 #include "pack.cuh"
+#include "prefill_gemm.cuh"
 #include "row_cluster.cuh"
 
 using namespace csa2;
@@ -279,6 +280,302 @@ size_t topk_ws_bytes(int32_t B, int32_t T, int64_t N) {
   return topk_ws_layout(nullptr, R, N).bytes;
 }
 
+// ---------------------------------------------------------------------------
+// Chunked prefill on the tensor cores (see prefill_gemm.cuh): shapes,
+// workspace, tensor maps and the per-pass launch sequence.
+// ---------------------------------------------------------------------------
+constexpr int64_t kPfMinT = 64;  // below this many queries per sequence the per-row scan is used
+
+int pf_cap(int32_t topk) { return std::max(8192, 4 * topk); }
+
+bool pf_eligible(int32_t T, int32_t H_I, int32_t d_I, int64_t N, int32_t topk,
+                 const float *score_out);
+
+struct PfWs {
+  int8_t *qa;
+  double *sigma, *err;
+  int32_t *tau, *fail_rows, *fail_count;
+  int32_t *smp;
+  uint32_t *bits;
+  int64_t smp_pitch, bits_pitch;
+  size_t bytes;
+};
+
+PfWs pf_ws_layout(void *base, int64_t R, int64_t N, int32_t d_I) {
+  PfWs w{};
+  w.smp_pitch = pf::kSampleMax;
+  w.bits_pitch = align_up(size_t(ceil_div(N, 32)), 32);
+  size_t off = 0;
+  auto take = [&](size_t bytes) {
+    size_t o = off;
+    off += align_up(bytes, 256);
+    return o;
+  };
+  const size_t o_qa = take(size_t(R) * 2 * d_I);
+  const size_t o_sigma = take(size_t(R) * 8);
+  const size_t o_err = take(size_t(R) * 8);
+  const size_t o_tau = take(size_t(R) * 4);
+  const size_t o_fail = take(size_t(R) * 4);
+  const size_t o_failn = take(4);
+  const size_t o_smp = take(size_t(R) * w.smp_pitch * 4);
+  const size_t o_bits = take(size_t(R) * w.bits_pitch * 4);
+  char *p = static_cast<char *>(base);
+  w.qa = reinterpret_cast<int8_t *>(p + o_qa);
+  w.sigma = reinterpret_cast<double *>(p + o_sigma);
+  w.err = reinterpret_cast<double *>(p + o_err);
+  w.tau = reinterpret_cast<int32_t *>(p + o_tau);
+  w.fail_rows = reinterpret_cast<int32_t *>(p + o_fail);
+  w.fail_count = reinterpret_cast<int32_t *>(p + o_failn);
+  w.smp = reinterpret_cast<int32_t *>(p + o_smp);
+  w.bits = reinterpret_cast<uint32_t *>(p + o_bits);
+  w.bytes = off;
+  return w;
+}
+
+// Query rows per pass: a multiple of 128 within the per-pass budget.
+int64_t pf_rows_per_pass(int32_t T, int64_t N, int32_t d_I) {
+  const int64_t per_row =
+      2 * d_I + 32 + int64_t(pf::kSampleMax) * 4 + int64_t(align_up(size_t(ceil_div(N, 32)), 32)) * 4;
+  int64_t R = std::max<int64_t>(pf::kQ, kTopkWsRowBudget / per_row / pf::kQ * pf::kQ);
+  return std::min<int64_t>(R, ceil_div(T, pf::kQ) * pf::kQ);
+}
+
+size_t pf_ws_bytes(int32_t T, int64_t N, int32_t d_I) {
+  return pf_ws_layout(nullptr, pf_rows_per_pass(T, N, d_I), N, d_I).bytes;
+}
+
+// cuTensorMapEncodeTiled through the runtime's driver entry point (no link
+// dependency on the driver library).
+using EncodeTiledFn = CUresult (*)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *,
+                                   const cuuint64_t *, const cuuint64_t *, const cuuint32_t *,
+                                   const cuuint32_t *, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                   CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_tiled() {
+  static EncodeTiledFn fn = nullptr;
+  static bool tried = false;
+  if (!tried) {
+    tried = true;
+    void *ptr = nullptr;
+    cudaDriverEntryPointQueryResult q = cudaDriverEntryPointSymbolNotFound;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(ptr);
+    cudaGetLastError();
+  }
+  return fn;
+}
+
+// 3-D byte tensor map: dims {d0, d1, d2}, byte strides of dims 1 and 2, box
+// {d0, b1, b2}, swizzled over d0 bytes (d0 in {32, 64, 128}).
+bool make_map_u8(CUtensorMap *m, const void *base, uint64_t d0, uint64_t d1, uint64_t d2,
+                 uint64_t s1, uint64_t s2, uint32_t b1, uint32_t b2) {
+  EncodeTiledFn f = encode_tiled();
+  if (!f || d1 == 0 || d2 == 0) return false;
+  const cuuint64_t dims[3] = {d0, d1, d2};
+  const cuuint64_t strides[2] = {s1, s2};
+  const cuuint32_t box[3] = {(cuuint32_t)d0, b1, b2};
+  const cuuint32_t es[3] = {1, 1, 1};
+  const CUtensorMapSwizzle sw = d0 == 128  ? CU_TENSOR_MAP_SWIZZLE_128B
+                                : d0 == 64 ? CU_TENSOR_MAP_SWIZZLE_64B
+                                           : CU_TENSOR_MAP_SWIZZLE_32B;
+  return f(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, const_cast<void *>(base), dims, strides, box, es,
+           CU_TENSOR_MAP_INTERLEAVE_NONE, sw, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+           CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+bool pf_eligible(int32_t T, int32_t H_I, int32_t d_I, int64_t N, int32_t topk,
+                 const float *score_out) {
+  return T >= kPfMinT && (d_I == 32 || d_I == 64 || d_I == 128) &&
+         scan_shape_supported(H_I, d_I) && N >= 1 && N < (int64_t(1) << 31) - 1 &&
+         4 * int64_t(topk) <= 16384 && score_out == nullptr && encode_tiled() != nullptr;
+}
+
+// Key-axis positions per CTA: minimises (waves of CTAs) x (tiles per CTA +
+// a fixed per-CTA cost), over multiples of the staging unit.
+int64_t pf_split_len(int64_t axis, int64_t nblk, int sms) {
+  const int64_t units = std::max<int64_t>(1, ceil_div(axis, pf::kAxisUnit));
+  int64_t best_len = units * pf::kAxisUnit, best_cost = INT64_MAX;
+  for (int64_t ns = 1; ns <= units; ++ns) {
+    const int64_t len = ceil_div(units, ns) * pf::kAxisUnit;
+    const int64_t nsplit = ceil_div(axis, len);
+    const int64_t waves = ceil_div(nblk * nsplit, sms);
+    const int64_t cost = waves * (len / pf::kN + 6);
+    if (cost < best_cost) {
+      best_cost = cost;
+      best_len = len;
+    }
+  }
+  return best_len;
+}
+
+template <int DI, bool SAMPLE>
+csa2_status launch_pf_gemm(const CUtensorMap &amap, const CUtensorMap &bmap,
+                           const pf::GemmParams &p, int64_t nsplit, int64_t nblk,
+                           cudaStream_t st) {
+  const size_t smem = pf::gemm_smem_bytes<DI>();
+  static bool done[256] = {false};
+  int dev = 0;
+  cudaGetDevice(&dev);
+  if (dev < 0 || dev >= 256 || !done[dev]) {
+    if (set_smem_attr(pf::pf_gemm_kernel<DI, SAMPLE>, smem, false) != CSA2_OK)
+      return CSA2_ERR_CUDA;
+    if (dev >= 0 && dev < 256) done[dev] = true;
+  }
+  TraceScope ts(SAMPLE ? "pf_sample_mma" : "pf_filter_mma", st);
+  pf::pf_gemm_kernel<DI, SAMPLE>
+      <<<dim3((unsigned)nsplit, (unsigned)nblk), pf::kGemmThreads, smem, st>>>(amap, bmap, p);
+  return after_launch();
+}
+
+template <int DI, int HI>
+csa2_status pf_run_rows(const int8_t *q_idx, const float *w, const int8_t *k_idx, int32_t B,
+                        int32_t T, int64_t N, int64_t n_prior, int32_t ratio, int32_t topk,
+                        int32_t *idx_out, const PfWs &L, int64_t R, cudaStream_t st) {
+  const int sms = device_sms();
+  const int cap = pf_cap(topk);
+  const size_t sel_smem = pf::sel_head_bytes<DI, HI>() + size_t(cap) * 8;
+  {
+    static bool done[256] = {false};
+    int dev = 0;
+    cudaGetDevice(&dev);
+    if (dev < 0 || dev >= 256 || !done[dev]) {
+      if (set_smem_attr(pf::pf_select_kernel<DI, HI>, pf::sel_head_bytes<DI, HI>() + 16384 * 8,
+                        false) != CSA2_OK)
+        return CSA2_ERR_CUDA;
+      if (dev >= 0 && dev < 256) done[dev] = true;
+    }
+  }
+  CUtensorMap kmap;
+  if (!make_map_u8(&kmap, k_idx, DI, uint64_t(N), uint64_t(B), DI, uint64_t(N) * DI, pf::kN, 1))
+    return CSA2_ERR_CUDA;
+  for (int32_t b = 0; b < B; ++b) {
+    for (int32_t t0 = 0; t0 < T; t0 += (int32_t)R) {
+      const int32_t tc = (int32_t)std::min<int64_t>(R, T - t0);
+      const int64_t nblk = ceil_div(tc, pf::kQ);
+      const int64_t vmax = pf::visible_count(N, n_prior, ratio, (int64_t)t0 + tc - 1);
+      if (cudaMemsetAsync(L.fail_count, 0, 4, st) != cudaSuccess) return CSA2_ERR_CUDA;
+      {
+        TraceScope ts("pf_prep", st);
+        pf::pf_prep_kernel<DI, HI><<<(unsigned)ceil_div(tc, 8), 256, 0, st>>>(
+            q_idx, w, T, b, t0, tc, L.qa, L.sigma, L.err);
+        if (after_launch() != CSA2_OK) return CSA2_ERR_CUDA;
+      }
+      CUtensorMap amap;
+      if (!make_map_u8(&amap, L.qa, DI, 2, uint64_t(tc), DI, 2 * DI, 1, pf::kQ))
+        return CSA2_ERR_CUDA;
+      pf::GemmParams gp{};
+      gp.N = N;
+      gp.T = T;
+      gp.n_prior = n_prior;
+      gp.ratio = ratio;
+      gp.b = b;
+      gp.t_begin = t0;
+      gp.t_count = tc;
+      // sample pass (only needed when some row has more visible entries
+      // than the selection capacity)
+      const int32_t sstride =
+          (int32_t)std::max<int64_t>(1, ceil_div(std::max<int64_t>(vmax, 1), pf::kSampleMax));
+      const int64_t nsamp = ceil_div(std::max<int64_t>(vmax, 1), sstride);
+      if (vmax > cap) {
+        CUtensorMap smap;
+        const uint64_t seq_samples = uint64_t(ceil_div(N, sstride));
+        if (!make_map_u8(&smap, k_idx, DI, seq_samples, uint64_t(B), uint64_t(sstride) * DI,
+                         uint64_t(N) * DI, pf::kN, 1))
+          return CSA2_ERR_CUDA;
+        gp.sstride = sstride;
+        gp.smp = L.smp;
+        gp.smp_pitch = L.smp_pitch;
+        gp.axis_len = nsamp;
+        gp.split_len = pf_split_len(nsamp, nblk, sms);
+        const int64_t nsplit = ceil_div(nsamp, gp.split_len);
+        if (launch_pf_gemm<DI, true>(amap, smap, gp, nsplit, nblk, st) != CSA2_OK)
+          return CSA2_ERR_CUDA;
+      }
+      {
+        pf::ThetaParams tp{};
+        tp.N = N;
+        tp.n_prior = n_prior;
+        tp.ratio = ratio;
+        tp.t_begin = t0;
+        tp.t_count = tc;
+        tp.sstride = sstride;
+        tp.nsamp = nsamp;
+        tp.smp = L.smp;
+        tp.smp_pitch = L.smp_pitch;
+        tp.target = 2 * topk;
+        tp.cap = cap;
+        tp.sigma = L.sigma;
+        tp.err = L.err;
+        tp.tau = L.tau;
+        TraceScope ts("pf_theta", st);
+        pf::pf_theta_kernel<<<(unsigned)tc, pf::kThetaThreads, 0, st>>>(tp);
+        if (after_launch() != CSA2_OK) return CSA2_ERR_CUDA;
+      }
+      gp.axis_len = vmax;
+      gp.split_len = pf_split_len(vmax, nblk, sms);
+      gp.tau = L.tau;
+      gp.bits = L.bits;
+      gp.bits_pitch = L.bits_pitch;
+      gp.sstride = 1;
+      gp.smp = nullptr;
+      {
+        const int64_t nsplit = ceil_div(std::max<int64_t>(vmax, 1), gp.split_len);
+        if (launch_pf_gemm<DI, false>(amap, kmap, gp, nsplit, nblk, st) != CSA2_OK)
+          return CSA2_ERR_CUDA;
+      }
+      pf::SelParams sp{};
+      sp.q_idx = q_idx;
+      sp.w = w;
+      sp.k_idx = k_idx;
+      sp.N = N;
+      sp.T = T;
+      sp.n_prior = n_prior;
+      sp.ratio = ratio;
+      sp.b = b;
+      sp.t_begin = t0;
+      sp.t_count = tc;
+      sp.topk = topk;
+      sp.cap = cap;
+      sp.bits = L.bits;
+      sp.bits_pitch = L.bits_pitch;
+      sp.tau = L.tau;
+      sp.sigma = L.sigma;
+      sp.err = L.err;
+      sp.idx = idx_out;
+      sp.fail_rows = L.fail_rows;
+      sp.fail_count = L.fail_count;
+      {
+        TraceScope ts("pf_select", st);
+        pf::pf_select_kernel<DI, HI><<<(unsigned)tc, pf::kSelThreads, sel_smem, st>>>(sp);
+        if (after_launch() != CSA2_OK) return CSA2_ERR_CUDA;
+      }
+      {
+        TraceScope ts("pf_fallback", st);
+        pf::pf_fallback_kernel<DI, HI>
+            <<<(unsigned)std::min<int64_t>(tc, sms), pf::kSelThreads, 0, st>>>(sp);
+        if (after_launch() != CSA2_OK) return CSA2_ERR_CUDA;
+      }
+    }
+  }
+  return CSA2_OK;
+}
+
+using PfRun = csa2_status (*)(const int8_t *, const float *, const int8_t *, int32_t, int32_t,
+                              int64_t, int64_t, int32_t, int32_t, int32_t *, const PfWs &,
+                              int64_t, cudaStream_t);
+
+PfRun pick_pf(int32_t d_I, int32_t H_I) {
+#define CSA2_PF_CASE(DI, HI) \
+  if (d_I == DI && H_I == HI) return &pf_run_rows<DI, HI>;
+  CSA2_PF_CASE(32, 1) CSA2_PF_CASE(32, 2) CSA2_PF_CASE(32, 4) CSA2_PF_CASE(32, 8)
+  CSA2_PF_CASE(64, 1) CSA2_PF_CASE(64, 2) CSA2_PF_CASE(64, 4) CSA2_PF_CASE(64, 8)
+  CSA2_PF_CASE(128, 1) CSA2_PF_CASE(128, 2) CSA2_PF_CASE(128, 4)
+#undef CSA2_PF_CASE
+  return nullptr;
+}
+
 struct AttnArgs {  // attention inputs of one layer (all device pointers)
   const uint16_t *q;
   const uint8_t *codes;
@@ -289,6 +586,11 @@ struct AttnArgs {  // attention inputs of one layer (all device pointers)
   float *out, *lse;
 };
 
+csa2_status run_attn(const uint16_t *q, const uint8_t *codes, const float *scales,
+                     const int32_t *idx, const uint16_t *win_k, const uint16_t *win_v, int32_t B,
+                     int32_t T, int32_t H, int32_t D, int64_t N, int32_t topk, int32_t W,
+                     float sm_scale, float *out, float *lse, cudaStream_t st);
+
 // Index + top-k (and, when `att` is given, the layer's attention fused into
 // the same per-row cluster kernel), in passes of R rows.
 csa2_status run_index_topk(const int8_t *q_idx, const float *w, const int8_t *k_idx, int32_t B,
@@ -296,6 +598,19 @@ csa2_status run_index_topk(const int8_t *q_idx, const float *w, const int8_t *k_
                            int32_t ratio, int32_t topk, int32_t *idx_out, float *score_out,
                            const AttnArgs *att, void *ws, size_t ws_bytes, cudaStream_t st) {
   const int64_t rows = int64_t(B) * T;
+  if (pf_eligible(T, H_I, d_I, N, topk, score_out)) {
+    const int64_t Rp = pf_rows_per_pass(T, N, d_I);
+    const PfWs Lp0 = pf_ws_layout(nullptr, Rp, N, d_I);
+    if (!ws || ws_bytes < Lp0.bytes || !aligned(ws, 16)) return CSA2_ERR_WORKSPACE;
+    const PfRun run = pick_pf(d_I, H_I);
+    if (!run) return CSA2_ERR_UNSUPPORTED;
+    const PfWs Lp = pf_ws_layout(ws, Rp, N, d_I);
+    if (run(q_idx, w, k_idx, B, T, N, n_prior, ratio, topk, idx_out, Lp, Rp, st) != CSA2_OK)
+      return CSA2_ERR_CUDA;
+    if (!att) return CSA2_OK;
+    return run_attn(att->q, att->codes, att->scales, idx_out, att->win_k, att->win_v, B, T,
+                    att->H, att->D, N, topk, att->W, att->sm_scale, att->out, att->lse, st);
+  }
   const int64_t R = topk_rows_per_pass(rows, N);
   const TopkWs L0 = topk_ws_layout(nullptr, R, N);
   if (!ws || ws_bytes < L0.bytes || !aligned(ws, 16)) return CSA2_ERR_WORKSPACE;
@@ -486,7 +801,9 @@ csa2_status csa2_unpack_fp4(const uint8_t *codes, const float *scales, int64_t r
 size_t csa2_index_topk_workspace_size(int32_t B, int32_t T, int32_t H_I, int32_t d_I, int64_t N,
                                       int32_t topk) {
   if (B < 0 || T < 0 || N < 0 || topk < 1 || !scan_shape_supported(H_I, d_I)) return 0;
-  return topk_ws_bytes(B, T, N);
+  size_t bytes = topk_ws_bytes(B, T, N);
+  if (pf_eligible(T, H_I, d_I, N, topk, nullptr)) bytes = std::max(bytes, pf_ws_bytes(T, N, d_I));
+  return bytes;
 }
 
 csa2_status csa2_index_topk(const int8_t *q_idx, const float *w, const int8_t *k_idx, int32_t B,

@@ -77,8 +77,9 @@ def _index_case(B, T, H_I, d_I, N, seed, key_levels=None, q_zero=False):
 def _check_index(q, w, k, topk, n_prior=-1, ratio=4, rows=None, check_scores=True):
     B, T = q.shape[:2]
     N = k.shape[1]
-    g_idx, g_sc = csa2.index_topk(dev(q), dev(w), dev(k), topk, n_prior, ratio,
-                                  want_scores=check_scores)
+    res = csa2.index_topk(dev(q), dev(w), dev(k), topk, n_prior, ratio,
+                          want_scores=check_scores)
+    g_idx, g_sc = res if check_scores else (res, None)
     g_idx = host(g_idx).reshape(B * T, topk)
     if rows is not None:
         g_idx = g_idx[rows]
@@ -131,6 +132,75 @@ def test_prefill_visibility():
     N = n_prior + T // ratio
     q, w, k = _index_case(B, T, H_I, d_I, N, seed=9)
     _check_index(q, w, k, 320, n_prior=n_prior, ratio=ratio)
+
+
+# ---------------------------------------------------------------------------
+# Chunked prefill through the tensor-core indexer: T >= 64 queries per
+# sequence and no score output select this path (approximate two-level int8
+# products on tcgen05, exact rescoring of the candidates, exact fallback).
+# ---------------------------------------------------------------------------
+
+@pytest.mark.parametrize("d_I,H_I", [(32, 4), (32, 8), (64, 1), (64, 4), (64, 8), (128, 2),
+                                     (128, 4)])
+def test_prefill_tensor_core_shapes(d_I, H_I):
+    B, T, n_prior, ratio = 2, 130, 12000, 4
+    N = n_prior + T // ratio
+    q, w, k = _index_case(B, T, H_I, d_I, N, seed=7 * d_I + H_I)
+    _check_index(q, w, k, 512, n_prior=n_prior, ratio=ratio, check_scores=False)
+
+
+@pytest.mark.parametrize("topk", [64, 2048, 4096])
+def test_prefill_tensor_core_all_visible(topk):
+    q, w, k = _index_case(1, 128, 4, 64, 30000, seed=topk)
+    _check_index(q, w, k, topk, check_scores=False)
+
+
+@pytest.mark.parametrize("N,topk", [(3000, 64), (3000, 2999), (3000, 4000), (8192, 2048)])
+def test_prefill_tensor_core_every_entry_a_candidate(N, topk):
+    q, w, k = _index_case(1, 129, 4, 64, N, seed=N + topk)
+    _check_index(q, w, k, topk, check_scores=False)
+
+
+def test_prefill_tensor_core_padding_and_empty_rows():
+    B, T, n_prior, ratio = 2, 300, 0, 4        # rows t < 3 see nothing; V_t = (t+1)//4
+    N = T // ratio
+    q, w, k = _index_case(B, T, 4, 64, N, seed=11)
+    idx = _check_index(q, w, k, 100, n_prior=n_prior, ratio=ratio, check_scores=False)
+    assert np.all(idx[:3] == -1)
+
+
+def test_prefill_tensor_core_heavy_ties():
+    q, w, k = _index_case(1, 64, 4, 64, 20000, seed=5, key_levels=1)
+    w[:] = 1.0                                 # integer scores in [-256, 256]: many ties
+    _check_index(q, w, k, 1000, check_scores=False)
+
+
+def test_prefill_tensor_core_all_equal_scores():
+    q, w, k = _index_case(1, 64, 4, 64, 20000, seed=6, q_zero=True)
+    idx = _check_index(q, w, k, 700, check_scores=False)
+    assert np.array_equal(idx, np.tile(np.arange(700, dtype=np.int32), (64, 1)))
+
+
+def _aligned_keys(q, w, n_keys):
+    """Keys that maximise the score of every row (all rows share q and w)."""
+    comb = (w[0, 0][:, None].astype(np.float64) * q[0, 0].astype(np.float64)).sum(axis=0)
+    return np.where(comb >= 0, 127, -127).astype(np.int8)[None, :].repeat(n_keys, axis=0)
+
+
+@pytest.mark.parametrize("where", ["sampled", "between_samples"])
+def test_prefill_tensor_core_misleading_sample(where):
+    """Top entries placed only on, or only between, the strided sample
+    positions (every 3rd entry for N = 20000): the sampled threshold then
+    misjudges the row (too few candidates, or more than the selection
+    capacity), and the exact fallback must still return the exact top-k."""
+    T, N, topk = 64, 20000, 2048
+    q, w, k = _index_case(1, T, 4, 64, N, seed=17)
+    q[:] = q[:, :1]
+    w[:] = w[:, :1]
+    n = np.arange(N)
+    pos = n[(n % 3 == 0)][:1400] if where == "sampled" else n[(n % 3 != 0)][:9000]
+    k[0, pos] = _aligned_keys(q, w, len(pos))
+    _check_index(q, w, k, topk, check_scores=False)
 
 
 @pytest.mark.parametrize("wl_name", ["tiny_decode_n1024", "decode_b32_n131072"])
