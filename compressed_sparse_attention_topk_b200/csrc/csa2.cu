@@ -473,6 +473,7 @@ csa2_status pf_run_rows(const int8_t *q_idx, const float *w, const int8_t *k_idx
       gp.b = b;
       gp.t_begin = t0;
       gp.t_count = tc;
+      gp.level_scale = 256;
       // sample pass (only needed when some row has more visible entries
       // than the selection capacity)
       const int32_t sstride =

@@ -69,7 +69,10 @@ template <int DI>
 struct GemmSmem {
   alignas(1024) uint8_t a[2][kQ * DI];
   alignas(1024) uint8_t b[kBRing];
-  uint32_t stage[kQ][32];  // mask words of up to 8 tiles; word w of row r at (w + r) & 31
+  union {
+    uint32_t stage[kQ][32];           // filter: mask words of up to 8 tiles; word w of row r at (w + r) & 31
+    int32_t sbuf[kEpiWarps][32][33];  // sample: one warp's 32 rows x 32 values, transposed on write
+  };
   uint64_t a_full;
   uint64_t full[GemmShape<DI>::STAGES], empty[GemmShape<DI>::STAGES];
   uint64_t acc_full[2], acc_empty[2];
@@ -100,6 +103,8 @@ struct GemmParams {
   const int32_t *tau;  // filter: [t_count] thresholds
   uint32_t *bits;      // filter: [t_count][bits_pitch] words, bit j of word w = entry 32w + j
   int64_t bits_pitch;
+  int32_t level_scale; // 256: weight of the first query level (a runtime value, so the
+                       // combine compiles to a multiply-add on the FMA pipe)
   int32_t sstride;     // sample: entries between samples
   int32_t *smp;        // sample: [t_count][smp_pitch] approximate scores, INT_MIN if invisible
   int64_t smp_pitch;
@@ -184,10 +189,23 @@ __device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t (&v)[32]) {
 __device__ __forceinline__ void tmem_wait_ld() {
   asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
 }
+// The same 32-bit value into 32 consecutive TMEM columns of this warp's lanes.
+__device__ __forceinline__ void tmem_st32_fill(uint32_t taddr, uint32_t x) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], {%1, %1, %1, %1, %1, %1, %1, %1, %1, %1, %1, "
+      "%1, %1, %1, %1, %1, %1, %1, %1, %1, %1, %1, %1, %1, %1, %1, %1, %1, %1, %1, %1, %1};" ::"r"(
+          taddr),
+      "r"(x)
+      : "memory");
+}
+__device__ __forceinline__ void tmem_wait_st() {
+  asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
+}
 
 // Bounded wait that also gives up once another role has aborted.
 template <int DI>
 __device__ __forceinline__ bool role_wait(GemmSmem<DI> &sm, uint64_t *bar, uint32_t parity) {
+  if (mbar_try_wait(bar, parity)) return true;  // no clock read on the fast path
   const long long start = clock64();
   while (!mbar_try_wait(bar, parity)) {
     if (sm.abort_flag) return false;
@@ -305,7 +323,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     }
     for (int a = 0; a < 2; ++a) {
       mbar_init(&sm.acc_full[a], 1);
-      mbar_init(&sm.acc_empty[a], kEpiWarps);
+      mbar_init(&sm.acc_empty[a], kEpiWarps / 2);
     }
     sm.abort_flag = 0u;
     fence_barrier_init();
@@ -358,7 +376,9 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       int issued = 0;
       for (int t = 0; ok && t < ntiles; ++t) {
         const int s = t % S::STAGES, acc = t & 1;
-        if (t >= 2 && !role_wait(sm, &sm.acc_empty[acc], (uint32_t)((t >> 1) - 1) & 1u)) break;
+        // buffer free: completion (t >> 1) of its barrier (the first one is the
+        // epilogue's bias initialisation)
+        if (!role_wait(sm, &sm.acc_empty[acc], (uint32_t)(t >> 1) & 1u)) break;
         if (!role_wait(sm, &sm.full[s], (uint32_t)(t / S::STAGES) & 1u)) break;
         tc_fence_after();
         const uint64_t bd = smem_desc<DI>(sm.b + s * S::B_BYTES);
@@ -366,7 +386,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
 #pragma unroll
         for (int k = 0; k < S::KSTEPS; ++k) {  // +32 bytes per K step = +2 in the address field
           umma_i8(d1, a0 + 2 * k, bd + 2 * k, k > 0 ? 1u : 0u);
-          umma_i8(d2, a1 + 2 * k, bd + 2 * k, k > 0 ? 1u : 0u);
+          umma_i8(d2, a1 + 2 * k, bd + 2 * k, 1u);  // onto the row's bias
         }
         umma_commit(&sm.empty[s]);
         umma_commit(&sm.acc_full[acc]);
@@ -379,83 +399,115 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     }
   } else if (ntiles > 0) {
     // ---------------- epilogue ----------------
-    // Every epilogue warp runs the same tile loop and the same quarter
-    // barriers, aborted or not, so the barriers always complete.
+    // Two groups of 8 warps (2 per TMEM lane quarter) take alternate tiles,
+    // so one group's TMEM loads overlap the other's arithmetic; group g owns
+    // accumulator buffer g.  A warp covers 64 columns (two 32-column chunks)
+    // of its group's tiles.  Every epilogue warp runs the same loop of
+    // 8-tile groups and the same quarter barriers, aborted or not, so the
+    // barriers always complete.
+    const int ew = warp - 2;
     const int quarter = warp & 3;
-    const int chunk = (warp - 2) >> 2;
+    const int grp = (ew >> 2) & 1;
+    const int half = ew >> 3;
     const int row = quarter * 32 + lane;
-    const int lt = lt0 + row;
-    const bool row_ok = lt < p.t_count;
     const int32_t vis = sm.vis[row];
     const int32_t tau = sm.tau[row];
-    const uint32_t taddr = tmem + ((uint32_t)(quarter * 32) << 16) + (uint32_t)(chunk * 32);
-    for (int t = 0; t < ntiles; ++t) {
-      const int acc = t & 1;
-      // warp-uniform decision: the TMEM loads below are .sync.aligned
-      const bool ok = __all_sync(0xffffffffu, role_wait(sm, &sm.acc_full[acc], (uint32_t)(t >> 1) & 1u));
-      uint32_t v1[32], v2[32];
-      if (ok) {
-        tc_fence_after();
-        tmem_ld32(taddr + (uint32_t)(acc * 2 * kN), v1);
-        tmem_ld32(taddr + (uint32_t)(acc * 2 * kN + kN), v2);
-        tmem_wait_ld();
-        tc_fence_before();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&sm.acc_empty[acc]);
-      } else {
+    const uint32_t tbase = tmem + ((uint32_t)(quarter * 32) << 16) + (uint32_t)(grp * 2 * kN);
+    const int32_t mul = p.level_scale;
+    // The level-2 accumulator of every tile starts at the row's bias, -tau
+    // (0 when sampling), so 256 v1 + v2 already is the difference to tau.
+    const uint32_t bias = SAMPLE ? 0u : (uint32_t)(-tau);
+    auto release = [&]() {  // bias stores done -> buffer free for the next MMA
+      tmem_wait_st();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&sm.acc_empty[grp]);
+    };
+    tmem_st32_fill(tbase + (uint32_t)(kN + half * 64), bias);
+    tmem_st32_fill(tbase + (uint32_t)(kN + half * 64 + 32), bias);
+    release();
+    const int ngroups = (ntiles + kGroupTiles - 1) / kGroupTiles;
+    for (int G = 0; G < ngroups; ++G) {
+      const int t_end = min(ntiles, (G + 1) * kGroupTiles);
+      for (int t = G * kGroupTiles + grp; t < t_end; t += 2) {
+        // warp-uniform decision: the TMEM loads below are .sync.aligned
+        const bool ok =
+            __all_sync(0xffffffffu, role_wait(sm, &sm.acc_full[grp], (uint32_t)(t >> 1) & 1u));
+        if (ok) tc_fence_after();
+#pragma unroll 1
+        for (int cc = 0; cc < 2; ++cc) {
+          const int chunk = half * 2 + cc;  // 32-column chunk of the tile
+          uint32_t v1[32], v2[32];
+          if (ok) {
+            tmem_ld32(tbase + (uint32_t)(chunk * 32), v1);
+            tmem_ld32(tbase + (uint32_t)(kN + chunk * 32), v2);
+            tmem_wait_ld();
+          } else {
 #pragma unroll
-        for (int j = 0; j < 32; ++j) v1[j] = v2[j] = 0u;
-      }
-      const int64_t c0 = k_lo + (int64_t)t * kN + chunk * 32;  // first key-axis position
-      if constexpr (SAMPLE) {
-        if (row_ok) {
-          int32_t *dst = p.smp + (int64_t)lt * p.smp_pitch;
+            for (int j = 0; j < 32; ++j) v1[j] = v2[j] = 0u;
+          }
+          const int64_t c0 = k_lo + (int64_t)t * kN + chunk * 32;  // first key-axis position
+          if constexpr (SAMPLE) {
+            // through shared memory so that each row's 32 values leave as one line
+            int32_t(*buf)[33] = sm.sbuf[ew];
 #pragma unroll
-          for (int j = 0; j < 32; ++j) {
-            const int64_t i = c0 + j;
-            if (i < k_hi)
-              dst[i] = (i * p.sstride < vis) ? (int32_t)(v1[j] << 8) + (int32_t)v2[j] : INT_MIN;
+            for (int j = 0; j < 32; ++j) buf[lane][j] = (int32_t)v1[j] * mul + (int32_t)v2[j];
+            __syncwarp();
+            const int64_t i = c0 + lane;
+            for (int rr = 0; rr < 32; ++rr) {
+              const int ltr = lt0 + quarter * 32 + rr;
+              if (ltr < p.t_count && i < k_hi)
+                p.smp[(int64_t)ltr * p.smp_pitch + i] =
+                    (i * p.sstride < sm.vis[quarter * 32 + rr]) ? buf[rr][lane] : INT_MIN;
+            }
+            __syncwarp();
+          } else {
+            // bit j = (256 v1_j + v2_j - tau >= 0): shift the sign bits in,
+            // highest column first, then invert
+            uint32_t m = 0u;
+#pragma unroll
+            for (int j = 31; j >= 0; --j) {
+              const int32_t d = (int32_t)v1[j] * mul + (int32_t)v2[j];  // 256 v1 + v2 - tau
+              m = __funnelshift_l((uint32_t)d, m, 1);
+            }
+            m = ~m;
+            if (c0 + 32 > vis) m = (c0 >= vis) ? 0u : (m & ((1u << (uint32_t)(vis - c0)) - 1u));
+            const int wl = (t % kGroupTiles) * 4 + chunk;
+            sm.stage[row][(wl + row) & 31] = m;
           }
         }
-      } else {
-        // bit j = (256 v1_j + v2_j >= tau): shift the sign bits of the
-        // differences in, highest column first, then invert
-        uint32_t m = 0u;
-#pragma unroll
-        for (int j = 31; j >= 0; --j) {
-          const int32_t d = (int32_t)(v1[j] << 8) + ((int32_t)v2[j] - tau);
-          m = __funnelshift_l((uint32_t)d, m, 1);
+        if (ok) {  // (a TMEM store between the two chunks' loads would stall the second)
+          tmem_st32_fill(tbase + (uint32_t)(kN + half * 64), bias);
+          tmem_st32_fill(tbase + (uint32_t)(kN + half * 64 + 32), bias);
+          release();
         }
-        m = ~m;
-        if (c0 + 32 > vis) m = (c0 >= vis) ? 0u : (m & ((1u << (uint32_t)(vis - c0)) - 1u));
-        const int g = t % kGroupTiles;
-        const int wl = g * 4 + chunk;
-        sm.stage[row][(wl + row) & 31] = m;
-        if (g == kGroupTiles - 1 || t == ntiles - 1) {
-          named_bar(1 + quarter, 128);
-          const int nw = (g + 1) * 4;                             // words staged per row
-          const int64_t wb = (k_lo + (int64_t)(t - g) * kN) / 32;  // first word
-          const int u = chunk * 32 + lane;
-          const int rr = quarter * 32 + (u >> 2);
-          const int part = (u & 3) * 8;
-          const int ltr = lt0 + rr;
-          if (ltr < p.t_count) {
-            uint32_t *dst = p.bits + (int64_t)ltr * p.bits_pitch + wb;
+      }
+      if constexpr (!SAMPLE) {
+        // the quarter's 32 rows x (tiles of this group x 4) words, 16 bytes
+        // per thread, whole lines per row
+        named_bar(1 + quarter, 128);
+        const int nw = (t_end - G * kGroupTiles) * 4;
+        const int64_t wb = (k_lo + (int64_t)G * kGroupTiles * kN) / 32;
+        const int u = (ew >> 2) * 32 + lane;
+        const int rr = quarter * 32 + (u >> 2);
+        const int part = (u & 3) * 8;
+        const int ltr = lt0 + rr;
+        if (ltr < p.t_count) {
+          uint32_t *dst = p.bits + (int64_t)ltr * p.bits_pitch + wb;
 #pragma unroll
-            for (int h = 0; h < 2; ++h) {
-              const int w0 = part + 4 * h;
-              if (w0 < nw) {
-                uint4 o;
-                o.x = sm.stage[rr][(w0 + rr) & 31];
-                o.y = sm.stage[rr][(w0 + 1 + rr) & 31];
-                o.z = sm.stage[rr][(w0 + 2 + rr) & 31];
-                o.w = sm.stage[rr][(w0 + 3 + rr) & 31];
-                *reinterpret_cast<uint4 *>(dst + w0) = o;
-              }
+          for (int h = 0; h < 2; ++h) {
+            const int w0 = part + 4 * h;
+            if (w0 < nw) {
+              uint4 o;
+              o.x = sm.stage[rr][(w0 + rr) & 31];
+              o.y = sm.stage[rr][(w0 + 1 + rr) & 31];
+              o.z = sm.stage[rr][(w0 + 2 + rr) & 31];
+              o.w = sm.stage[rr][(w0 + 3 + rr) & 31];
+              *reinterpret_cast<uint4 *>(dst + w0) = o;
             }
           }
-          named_bar(1 + quarter, 128);
         }
+        named_bar(1 + quarter, 128);
       }
     }
   }
@@ -471,8 +523,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
 }
 
 // ---------------------------------------------------------------------------
-// 3. theta: filter threshold per row from the sampled approximate scores.
-// One CTA of kThetaThreads per row; the row's samples live in registers.
+// 3. theta: filter threshold per row from the sampled approximate scores
+// (kernel below, after the selection helper it shares with step 5).
 // ---------------------------------------------------------------------------
 struct ThetaParams {
   int64_t N;
@@ -488,65 +540,6 @@ struct ThetaParams {
   const double *sigma, *err;
   int32_t *tau;
 };
-
-__global__ void __launch_bounds__(kThetaThreads) pf_theta_kernel(const ThetaParams p) {
-  constexpr int VPT = kSampleMax / kThetaThreads;
-  __shared__ uint32_t hist[kBins1];
-  __shared__ uint32_t scratch[40];
-  __shared__ uint32_t res[2];
-  const int tid = threadIdx.x;
-  const int lt = blockIdx.x;
-  const int64_t V = visible_count(p.N, p.n_prior, p.ratio, (int64_t)p.t_begin + lt);
-  const int64_t S_t = min64((V + p.sstride - 1) / p.sstride, p.nsamp);
-  const int64_t j = (p.target + p.sstride - 1) / p.sstride;
-  if (V <= p.cap || j > S_t) {  // select over every visible entry
-    if (tid == 0) p.tau[lt] = kTauAll;
-    return;
-  }
-  // keys of the samples: order-preserving unsigned view of the int32 values
-  uint32_t key[VPT];
-  const int32_t *row = p.smp + (int64_t)lt * p.smp_pitch;
-#pragma unroll
-  for (int i = 0; i < VPT; ++i) {
-    const int64_t s = tid + (int64_t)i * kThetaThreads;
-    key[i] = s < S_t ? ((uint32_t)row[s] ^ 0x80000000u) : 0u;
-  }
-  // three radix digits (11, 11, 10 bits) of the j-th largest key
-  uint32_t need = (uint32_t)j, prefix = 0u;
-  for (int level = 0; level < 3; ++level) {
-    for (int i = tid; i < kBins1; i += kThetaThreads) hist[i] = 0u;
-    __syncthreads();
-#pragma unroll
-    for (int i = 0; i < VPT; ++i) {
-      const int64_t s = tid + (int64_t)i * kThetaThreads;
-      if (s >= S_t) continue;
-      const uint32_t k = key[i];
-      if (level == 0)
-        atomicAdd(&hist[key_d1(k)], 1u);
-      else if (level == 1) {
-        if (key_d1(k) == prefix) atomicAdd(&hist[key_d2(k)], 1u);
-      } else if ((k >> 10) == prefix)
-        atomicAdd(&hist[key_d3(k)], 1u);
-    }
-    __syncthreads();
-    if (level < 2)
-      radix_threshold<kThetaThreads, kBins1>(hist, need, scratch, res);
-    else
-      radix_threshold<kThetaThreads, kBins3>(hist, need, scratch, res);
-    const uint32_t bin = res[0];
-    need -= res[1];
-    prefix = level == 0 ? bin : (level == 1 ? (prefix << 11) | bin : (prefix << 10) | bin);
-    __syncthreads();
-  }
-  if (tid == 0) {
-    const int64_t theta = (int64_t)(int32_t)(prefix ^ 0x80000000u);
-    const double es = p.err[lt] * p.sigma[lt];
-    const int64_t margin = 3 * (int64_t)ceil(es) + 4;
-    int64_t t = theta - margin;
-    if (t < kTauAll) t = kTauAll;
-    p.tau[lt] = (int32_t)t;
-  }
-}
 
 // ---------------------------------------------------------------------------
 // Exact score of one entry (the definition used everywhere in the library).
@@ -646,6 +639,40 @@ __device__ void select_threshold(const uint32_t *ckey, int n, uint32_t need, uin
 }
 
 // ---------------------------------------------------------------------------
+// 3. theta kernel: the j-th largest sampled value, less margins of the
+// bound.  One CTA of kThetaThreads per row.
+// ---------------------------------------------------------------------------
+__global__ void __launch_bounds__(kThetaThreads) pf_theta_kernel(const ThetaParams p) {
+  __shared__ uint32_t skey[kSampleMax];
+  __shared__ uint32_t hist[kBins1];
+  __shared__ uint32_t scratch[40];
+  __shared__ uint32_t res[2];
+  const int tid = threadIdx.x;
+  const int lt = blockIdx.x;
+  const int64_t V = visible_count(p.N, p.n_prior, p.ratio, (int64_t)p.t_begin + lt);
+  const int64_t S_t = min64((V + p.sstride - 1) / p.sstride, p.nsamp);
+  const int64_t j = (p.target + p.sstride - 1) / p.sstride;
+  if (V <= p.cap || j > S_t) {  // select over every visible entry
+    if (tid == 0) p.tau[lt] = kTauAll;
+    return;
+  }
+  // order-preserving unsigned keys of the sampled int32 values
+  const int32_t *row = p.smp + (int64_t)lt * p.smp_pitch;
+  for (int i = tid; i < S_t; i += kThetaThreads) skey[i] = (uint32_t)row[i] ^ 0x80000000u;
+  __syncthreads();
+  uint32_t kstar, ties;
+  select_threshold<kThetaThreads>(skey, (int)S_t, (uint32_t)j, hist, scratch, res, kstar, ties);
+  if (tid == 0) {
+    const int64_t theta = (int64_t)(int32_t)(kstar ^ 0x80000000u);
+    const double es = p.err[lt] * p.sigma[lt];
+    const int64_t margin = 3 * (int64_t)ceil(es) + 4;
+    int64_t t = theta - margin;
+    if (t < kTauAll) t = kTauAll;
+    p.tau[lt] = (int32_t)t;
+  }
+}
+
+// ---------------------------------------------------------------------------
 // 5. select: candidates of a row -> exact rescoring -> exact top-k, or hand
 // the row to the fallback.  One CTA of kSelThreads per row.
 // ---------------------------------------------------------------------------
@@ -669,43 +696,85 @@ __global__ void __launch_bounds__(kSelThreads) pf_select_kernel(const SelParams 
   for (int i = tid; i < HI * DI / 16; i += kSelThreads) sm.q[i] = qsrc[i];
   if (tid < HI) sm.w[tid] = p.w[r * HI + tid];
 
-  // candidates in ascending entry order: thread u owns a contiguous range
-  // of mask words
+  // candidates in ascending entry order: thread u owns a contiguous,
+  // 16-byte aligned range of mask words; the first kWordsCached of them stay
+  // in registers between the count and the extraction
+  constexpr int kWordsCached = 32;
   const uint32_t *brow = p.bits + (int64_t)lt * p.bits_pitch;
   const int64_t nw = (V + 31) / 32;
-  const int64_t wpt = (nw + kSelThreads - 1) / kSelThreads;
+  const int64_t wpt = ((nw + kSelThreads - 1) / kSelThreads + 3) & ~int64_t(3);
   const int64_t w0 = min64(nw, (int64_t)tid * wpt), w1 = min64(nw, w0 + wpt);
+  const uint32_t last_mask = (V & 31) ? (1u << (uint32_t)(V & 31)) - 1u : 0xffffffffu;
+  auto word = [&](int64_t wi, uint32_t raw) -> uint32_t {
+    if (wi >= w1) return 0u;
+    return wi == nw - 1 ? (raw & last_mask) : raw;
+  };
+  uint32_t wv[kWordsCached];
+#pragma unroll
+  for (int c = 0; c < kWordsCached / 4; ++c) {
+    const int64_t wi = w0 + 4 * c;
+    uint4 x = make_uint4(0u, 0u, 0u, 0u);
+    if (wi < w1) x = __ldg(reinterpret_cast<const uint4 *>(brow + wi));
+    wv[4 * c] = word(wi, x.x);
+    wv[4 * c + 1] = word(wi + 1, x.y);
+    wv[4 * c + 2] = word(wi + 2, x.z);
+    wv[4 * c + 3] = word(wi + 3, x.w);
+  }
   uint32_t cnt = 0;
-  for (int64_t wi = w0; wi < w1; ++wi) {
-    uint32_t m = __ldg(brow + wi);
-    if (wi == nw - 1 && (V & 31)) m &= (1u << (uint32_t)(V & 31)) - 1u;
-    cnt += __popc(m);
+#pragma unroll
+  for (int c = 0; c < kWordsCached; ++c) cnt += __popc(wv[c]);
+  for (int64_t wi = w0 + kWordsCached; wi < w1; wi += 4) {  // rows longer than 512 x 32 words
+    const uint4 x = __ldg(reinterpret_cast<const uint4 *>(brow + wi));
+    cnt += __popc(word(wi, x.x)) + __popc(word(wi + 1, x.y)) + __popc(word(wi + 2, x.z)) +
+           __popc(word(wi + 3, x.w));
   }
   uint32_t C;
   uint32_t pos = block_excl_scan<kSelThreads>(cnt, sm.scratch, C);
   const bool overflow = C > (uint32_t)p.cap;
   if (!overflow) {
-    for (int64_t wi = w0; wi < w1; ++wi) {
-      uint32_t m = __ldg(brow + wi);
-      if (wi == nw - 1 && (V & 31)) m &= (1u << (uint32_t)(V & 31)) - 1u;  // never past V
+#pragma unroll
+    for (int c = 0; c < kWordsCached; ++c) {
+      uint32_t m = wv[c];
       while (m) {
-        const int bit = __ffs(m) - 1;
-        cidx[pos++] = (uint32_t)(wi * 32 + bit);
+        cidx[pos++] = (uint32_t)((w0 + c) * 32 + (__ffs(m) - 1));
         m &= m - 1u;
+      }
+    }
+    for (int64_t wi = w0 + kWordsCached; wi < w1; wi += 4) {
+      const uint4 x = __ldg(reinterpret_cast<const uint4 *>(brow + wi));
+      const uint32_t xs[4] = {x.x, x.y, x.z, x.w};
+      for (int e = 0; e < 4; ++e) {
+        uint32_t m = word(wi + e, xs[e]);
+        while (m) {
+          cidx[pos++] = (uint32_t)((wi + e) * 32 + (__ffs(m) - 1));
+          m &= m - 1u;
+        }
       }
     }
   }
   __syncthreads();
   bool fail = overflow;
   if (!fail) {
-    // exact scores; count those certified above every entry left out
+    // exact scores, four candidates per thread in flight; count those
+    // certified above every entry left out
     const double U = ((double)p.tau[lt] - 1.0) / p.sigma[lt] + p.err[lt];
     const int8_t *kseq = p.k_idx + (int64_t)p.b * p.N * DI;
     uint32_t above = 0;
-    for (uint32_t i = tid; i < C; i += kSelThreads) {
-      const float s = exact_score<DI, HI>(kseq + (int64_t)cidx[i] * DI, sm.q, sm.w);
-      ckey[i] = score_key(s);
-      above += (double)s > U;
+    for (uint32_t i0 = tid; i0 < C; i0 += 4 * kSelThreads) {
+      float s[4];
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        const uint32_t i = i0 + u * kSelThreads;
+        s[u] = i < C ? exact_score<DI, HI>(kseq + (int64_t)cidx[i] * DI, sm.q, sm.w) : 0.0f;
+      }
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        const uint32_t i = i0 + u * kSelThreads;
+        if (i < C) {
+          ckey[i] = score_key(s[u]);
+          above += (double)s[u] > U;
+        }
+      }
     }
     uint32_t total_above;
     block_excl_scan<kSelThreads>(above, sm.scratch, total_above);
