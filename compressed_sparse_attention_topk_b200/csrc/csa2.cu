@@ -7,6 +7,7 @@
 #include <cstdint>
 #include <cstring>
 
+#include "attn_rows.cuh"
 #include "common.cuh"
 #include "index_scan.cuh"
 #include "pack.cuh"
@@ -695,11 +696,57 @@ csa2_status check_attn_args(const uint16_t *q, const uint8_t *codes, const float
 
 constexpr int64_t kAttnRowsPerLaunch = 16384;
 
+// Many rows: one CTA per (row, 16-head pass), every SM busy with whole rows.
+template <int D>
+csa2_status launch_attn_rows(const ar::Params &p, int64_t nr, cudaStream_t st) {
+  const size_t smem = sizeof(ar::Smem<D>);
+  static bool done[256] = {false};
+  int dev = 0;
+  cudaGetDevice(&dev);
+  if (dev < 0 || dev >= 256 || !done[dev]) {
+    if (set_smem_attr(ar::attn_rows_kernel<D>, smem, false) != CSA2_OK) return CSA2_ERR_CUDA;
+    if (dev >= 0 && dev < 256) done[dev] = true;
+  }
+  TraceScope ts("attend_rows", st);
+  const unsigned passes = (unsigned)ceil_div(p.H, ar::kHeads);
+  ar::attn_rows_kernel<D><<<dim3((unsigned)nr, passes), ar::kThreads, smem, st>>>(p);
+  return after_launch();
+}
+
+// Rows at which the per-row CTA kernel takes over from the cluster kernel
+// (which spreads one row over up to 16 SMs: better while rows are few).
+inline int64_t attn_rows_threshold() { return 2 * int64_t(device_sms()); }
+
 csa2_status run_attn(const uint16_t *q, const uint8_t *codes, const float *scales,
                      const int32_t *idx, const uint16_t *win_k, const uint16_t *win_v, int32_t B,
                      int32_t T, int32_t H, int32_t D, int64_t N, int32_t topk, int32_t W,
                      float sm_scale, float *out, float *lse, cudaStream_t st) {
   const int64_t rows = int64_t(B) * T;
+  if (rows >= attn_rows_threshold()) {
+    ar::Params a{};
+    a.q = q;
+    a.codes = codes;
+    a.scales = scales;
+    a.idx = idx;
+    a.win_k = win_k;
+    a.win_v = win_v;
+    a.N = N;
+    a.T = T;
+    a.H = H;
+    a.W = W;
+    a.topk = topk;
+    a.q_scale = sm_scale * 1.4426950408889634f;
+    a.out = out;
+    a.lse = lse;
+    for (int64_t row0 = 0; row0 < rows; row0 += kAttnRowsPerLaunch) {
+      const int64_t nr = std::min<int64_t>(kAttnRowsPerLaunch, rows - row0);
+      a.row0 = row0;
+      const csa2_status rc =
+          D == 128 ? launch_attn_rows<128>(a, nr, st) : launch_attn_rows<64>(a, nr, st);
+      if (rc != CSA2_OK) return rc;
+    }
+    return CSA2_OK;
+  }
   RowParams p{};
   p.N = N;
   p.T = T;

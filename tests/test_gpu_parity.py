@@ -282,6 +282,34 @@ def test_attention_prefill(T, W):
     _check_attn(entries, q, wk, wv, idx, decode=False)
 
 
+@pytest.mark.parametrize("D,H,topk,W", [(128, 16, 2048, 128), (64, 8, 100, 5), (128, 20, 64, 0),
+                                        (128, 16, 37, 17)])
+def test_attention_many_rows(D, H, topk, W):
+    """320 query rows (more than two per SM) take the one-CTA-per-row kernel:
+    ragged key chunks, a second head pass, padding inside a row and a row
+    with no selected entry."""
+    entries, q, wk, wv, idx = _attn_inputs(2, 160, H, D, 3000, topk, W, seed=D * 7 + H + topk + W)
+    idx[0, 3, ::5] = -1
+    idx[1, 7, :] = -1
+    _check_attn(entries, q, wk, wv, idx, decode=False)
+
+
+def test_attention_many_rows_bad_index_recorded_and_skipped():
+    entries, q, wk, wv, idx = _attn_inputs(2, 160, 16, 128, 900, 64, 16, seed=9)
+    bad = idx.copy()
+    bad[1, 100, 7] = 900 + 3
+    skipped = bad.copy()
+    skipped[1, 100, 7] = -1
+    oc, os_ = oracle_store(entries)
+    gc, gs = gpu_store(entries)
+    ref_out, ref_lse = oracle.sparse_attn(q, oc, os_, skipped, wk, wv)
+    out, lse = csa2.sparse_attn_prefill(dev(q), gc, gs, dev(bad), dev(wk), dev(wv))
+    assert_close(host(out).reshape(ref_out.shape), ref_out, "out")
+    assert_close(host(lse).reshape(ref_lse.shape), ref_lse, "lse")
+    assert csa2.get_device_status() & 1
+    assert csa2.get_device_status() == 0
+
+
 # ---------------------------------------------------------------------------
 # Whole workloads through the C ABI
 # ---------------------------------------------------------------------------
