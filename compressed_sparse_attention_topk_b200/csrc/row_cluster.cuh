@@ -31,12 +31,12 @@
 //      ranks and warps give every warp its offset in the output row, so the
 //      indices come out ascending.
 //
-// Attention: each CTA attends over an even share of the window rows (done
-// first, while the top-k inputs are still arriving) and over the entries it
-// selected itself (their raw FP4 rows gathered in batches of async copies),
-// in chunks of 64 keys with an online softmax in base 2.  A chunk is two
-// small tensor-core products (mma.sync m16n8k16, bf16 in, fp32 out; 16
-// heads is exactly the M = 16 of that shape):
+// Attention: each CTA attends over an even share of the window rows and over
+// the entries it selected itself (with given indices, an even share of the
+// index slots), cut into 16-key chunks that kAttnWarps warps take in turn,
+// each with its own online softmax in base 2 (the per-warp blocks of
+// attn_rows.cuh: gather by cp.async with invalid keys zero-filled, E2M1 ->
+// exact bf16, mma.sync m16n8k16 with 16 heads as M):
 //   logits  S[h, n] = sum_g s[n, g] * sum_{i in g} q[h, i] * e2m1[n, i]
 //           one product per 16-element scale group g; E2M1 values and the
 //           bf16 query are exact in bf16, so every product is exact and the
@@ -44,15 +44,17 @@
 //   values  O[h, d] += sum_n (P[h, n] * s[n, g(d)]) * e2m1[n, d]
 //           with the fp32 weight P*s split into a bf16 pair hi + lo (two
 //           products), so the weight keeps ~16 bits.
-// Window rows use the same path with scale 1 (bf16 keys and values).  Each
-// CTA pushes its partial (max, sum, acc) of head h into the shared memory of
-// the CTA that owns h (h mod CL); after one cluster barrier the owners merge
-// locally by log-sum-exp.  Which CTA handles which key does not change the
-// result, so no entry is moved between CTAs.  With given indices (attention
-// only), CTA c takes an even share of the selected slots.
+// Window rows use the same path with scale 1 (bf16 keys and values).  The
+// warps' states are merged in shared memory (their buffers alias the dead
+// top-k working set), and each CTA pushes its partial (max, sum, acc) of
+// head h into the shared memory of the CTA that owns h (h mod CL); after one
+// cluster barrier the owners merge locally by log-sum-exp.  Which CTA
+// handles which key does not change the result, so no entry is moved
+// between CTAs.
 #pragma once
 #include <cooperative_groups.h>
 
+#include "attn_rows.cuh"
 #include "common.cuh"
 #include "pack.cuh"
 
@@ -65,9 +67,8 @@ constexpr int kRowWarps = kRowThreads / 32;
 constexpr int kStageScores = 16384;  // scores staged in shared memory per round
 constexpr int kCandCap = 4096;       // candidates kept in shared memory
 constexpr int kSelCap = 4096;        // selected indices kept in shared memory
-constexpr int kRawCap = 512;         // entries gathered per batch
-constexpr int kChunkKeys = 64;
 constexpr int kHeads = 16;           // heads per pass (the MMA's M)
+constexpr int kAttnWarps = 8;        // warps that run attention chunks
 
 struct RowParams {
   // top-k
@@ -97,33 +98,24 @@ struct RowParams {
 
 template <int D>
 struct RowSmem {
-  static constexpr int G = D / 16;  // scale groups per entry
   union {
-    float sc[kStageScores];  // staged score slice (top-k)
-    struct {                 // raw gathered entries (attention)
-      uint8_t codes[kRawCap][D / 2];
-      float scales[kRawCap][D / 16];
-    } raw;
-  } st;
+    struct {  // top-k working set
+      float sc[kStageScores];                                    // staged score slice
+      uint2 cand[kCandCap];                                      // candidates (key, index - slice start)
+      uint32_t masks[kRowWarps][kStageScores / kRowWarps / 32];  // per-warp ballots of a round
+    } tk;
+    ar::WarpArea<D> aw[kAttnWarps];  // attention: per-warp chunk buffers, then partial states
+  } u;
   uint32_t h1[kBins1];          // staged digit-1 histogram
   uint32_t h2[kBins2];          // own digit-2 (then digit-3) histogram
   uint32_t hin[kBins2];         // bin slice this CTA owns, one row per source rank (pushed)
   uint32_t full[kBins2];        // cluster-wide histogram (reduced slices pushed by owners)
   uint32_t cnt_all[32][2];      // every rank's (above, tie) counts (pushed)
-  uint2 cand[kCandCap];         // candidates (key, index - slice start), index order
   int32_t sel[kSelCap];         // this CTA's selected indices, ascending
-  int32_t raw_idx[kRawCap];     // entries of the gathered batch
   uint32_t wa[kRowWarps], wb[kRowWarps], wc[kRowWarps], wd[kRowWarps];
-  uint32_t masks[kRowWarps][kStageScores / kRowWarps / 32];  // per-warp ballots of a round
-  // attention
-  uint16_t kb[kChunkKeys][D + 8];   // keys, row-major bf16 (+8: conflict-free B loads)
-  uint16_t vt[D][kChunkKeys + 8];   // values, transposed bf16
-  float ks[kChunkKeys][G];          // per-key group scales (1 for window rows)
-  float s[kHeads][kChunkKeys + 4];  // logits, then probabilities
-  float corr[kHeads];
-  uint16_t qb[kHeads][D + 8];       // query, bf16
-  float inbox[kHeads][D + 2];       // pushed partials (m, l, acc) of the heads this CTA merges
-  int valid[kChunkKeys];
+  uint16_t qb[kHeads][D + 8];   // query of the head pass, bf16
+  float inbox[kHeads][D + 2];   // pushed partials (m, l, acc) of the heads this CTA merges
+  float mf[kHeads][kAttnWarps + 1];  // per head: each attention warp's factor, then the max
   uint32_t scratch[40];
   uint32_t thr[8];
   uint32_t cnt[4];  // [1] above-threshold, [2] equal-to-threshold, [3] reduced-slice total
@@ -213,9 +205,12 @@ __device__ void row_topk(RowSmem<D> &sm, const RowParams &p, cg::cluster_group &
   radix_threshold<kRowThreads, kBins1>(sm.h1, (uint32_t)K, sm.scratch, sm.thr);
   const uint32_t t1 = sm.thr[0], r1 = (uint32_t)K - sm.thr[1];
 
-  // 1. candidate list in index order: warp w owns segment [seg0, seg1) of
-  //    each staged round; a counting pass, one prefix over warps, a ballot
-  //    pass that writes the candidates.
+  // 1. candidate list in index order: thread t owns the contiguous run
+  //    [32t, 32t + 32) of each staged round; a mask of its elements with
+  //    digit 1 >= t1 (16-byte reads, rotated per thread: conflict-free),
+  //    one block prefix over the counts, then each thread writes its
+  //    candidates and histograms digit 2 of those exactly at t1.
+  static_assert(kStageScores == 32 * kRowThreads, "one 32-bit mask per thread and round");
   uint32_t count = 0;
   for (int64_t rb = s0; rb < s1; rb += kStageScores) {
     const int n = (int)min64(kStageScores, s1 - rb);
@@ -225,60 +220,47 @@ __device__ void row_topk(RowSmem<D> &sm, const RowParams &p, cg::cluster_group &
         if (tid == 0) {
           const uint32_t bytes = (uint32_t)(((n + 3) & ~3) * 4);
           mbar_arrive_expect_tx(&sm.bar, bytes);
-          bulk_g2s(sm.st.sc, srow + rb, bytes, &sm.bar);
+          bulk_g2s(sm.u.tk.sc, srow + rb, bytes, &sm.bar);
         }
         if (!mbar_wait_bounded(&sm.bar, phase & 1u)) abort = true;
         ++phase;
       } else {
-        for (int i = tid; i < n; i += kRowThreads) sm.st.sc[i] = srow[rb + i];
+        for (int i = tid; i < n; i += kRowThreads) sm.u.tk.sc[i] = srow[rb + i];
       }
       __syncthreads();
     }
-    // one ballot per 32 elements of the warp's segment, kept in shared memory
-    const int seg0 = (n * warp) / kRowWarps, seg1 = (n * (warp + 1)) / kRowWarps;
-    constexpr int STEPS = kStageScores / kRowWarps / 32;
-    uint32_t mine = 0;
-#pragma unroll 8
-    for (int j = 0; j < STEPS; ++j) {
-      const int i = seg0 + 32 * j + lane;
-      const bool in = (i < seg1) && key_d1(score_key(sm.st.sc[i])) >= t1;
-      const uint32_t bal = __ballot_sync(0xffffffffu, in);
-      if (lane == (j & 31)) sm.masks[warp][j] = bal;
-      mine += __popc(bal);
+    const int base = 32 * tid;
+    uint32_t bits = 0u;
+#pragma unroll
+    for (int q = 0; q < 8; ++q) {
+      const int qq = (q + tid) & 7;
+      const int i = base + 4 * qq;
+      const float4 v = *reinterpret_cast<const float4 *>(&sm.u.tk.sc[i]);
+      bits |= (uint32_t)((i + 0 < n) && key_d1(score_key(v.x)) >= t1) << (4 * qq + 0);
+      bits |= (uint32_t)((i + 1 < n) && key_d1(score_key(v.y)) >= t1) << (4 * qq + 1);
+      bits |= (uint32_t)((i + 2 < n) && key_d1(score_key(v.z)) >= t1) << (4 * qq + 2);
+      bits |= (uint32_t)((i + 3 < n) && key_d1(score_key(v.w)) >= t1) << (4 * qq + 3);
     }
-    if (lane == 0) sm.wa[warp] = mine;
-    __syncthreads();
-    if (warp == 0) warp0_prefix16(sm.wa, sm.wb, &sm.scratch[0]);
-    __syncthreads();
-    // write pass: only the steps that hold candidates
-    uint32_t pos = count + sm.wb[warp];
-    for (int j = 0; j < STEPS; ++j) {
-      const uint32_t bal = sm.masks[warp][j];
-      if (bal == 0u) continue;  // warp-uniform
-      if ((bal >> lane) & 1u) {
-        const int i = seg0 + 32 * j + lane;
-        const uint32_t key = score_key(sm.st.sc[i]);
-        const uint32_t at = pos + __popc(bal & lt);
-        const uint2 e = make_uint2(key, (uint32_t)(rb - s0 + i));
-        if (at < (uint32_t)kCandCap)
-          sm.cand[at] = e;
-        else
-          spill[at] = e;
-      }
-      pos += __popc(bal);
+    uint32_t total;
+    uint32_t pos = count + block_excl_scan<kRowThreads>((uint32_t)__popc(bits), sm.scratch, total);
+    while (bits) {
+      const int i = base + __ffs(bits) - 1;
+      bits &= bits - 1u;
+      const uint32_t key = score_key(sm.u.tk.sc[i]);
+      const uint2 e = make_uint2(key, (uint32_t)(rb - s0 + i));
+      if (pos < (uint32_t)kCandCap)
+        sm.u.tk.cand[pos] = e;
+      else
+        spill[pos] = e;
+      if (key_d1(key) == t1) atomicAdd(&sm.h2[key_d2(key)], 1u);
+      ++pos;
     }
-    count += sm.scratch[0];
+    count += total;
   }
   __syncthreads();
   auto cand_at = [&](uint32_t i) -> uint2 {
-    return (i < (uint32_t)kCandCap) ? sm.cand[i] : spill[i];
+    return (i < (uint32_t)kCandCap) ? sm.u.tk.cand[i] : spill[i];
   };
-  // digit-2 histogram of the candidates exactly at t1 (few atomics)
-  for (uint32_t i = tid; i < count; i += kRowThreads) {
-    const uint32_t k = cand_at(i).x;
-    if (key_d1(k) == t1) atomicAdd(&sm.h2[key_d2(k)], 1u);
-  }
-  __syncthreads();
 
   // 2. digit-2 threshold from the cluster's histograms
   cluster_threshold<D, CL, kBins2>(sm, cluster, r1, sm.thr + 2);
@@ -300,34 +282,27 @@ __device__ void row_topk(RowSmem<D> &sm, const RowParams &p, cg::cluster_group &
     r3 = r2 - sm.thr[3];
   }
 
-  // 4. classify: warp w takes candidates [count*w/16, count*(w+1)/16)
-  const uint32_t c0 = (uint32_t)(((uint64_t)count * warp) / kRowWarps);
-  const uint32_t c1 = (uint32_t)(((uint64_t)count * (warp + 1)) / kRowWarps);
+  // 4. classify: thread t takes the contiguous candidates [t*per, t*per +
+  //    per).  Block prefixes of the (above, tie) counts give each thread
+  //    the counts before it; the CTA totals go to every rank.  Ties
+  //    are taken in index order while the cluster-wide tie rank stays below
+  //    r3, so the ties taken before a thread are min(ties before it, r3 -
+  //    this CTA's tie base): no second prefix is needed.
+  const uint32_t per = (count + kRowThreads - 1) / kRowThreads;
+  const uint32_t i0 = min(count, per * (uint32_t)tid), i1 = min(count, i0 + per);
   uint32_t n_above = 0, n_tie = 0;
-  for (uint32_t i = c0 + lane; i < c1; i += 32) {
+  for (uint32_t i = i0; i < i1; ++i) {
     const uint32_t cls = cand_class(cand_at(i).x, t1, t2, t3, need3);
     n_above += (cls == 2u);
     n_tie += (cls == 1u);
   }
-  n_above = __reduce_add_sync(0xffffffffu, n_above);
-  n_tie = __reduce_add_sync(0xffffffffu, n_tie);
-  if (lane == 0) {
-    sm.wa[warp] = n_above;
-    sm.wb[warp] = n_tie;
-  }
-  __syncthreads();
-  if (warp == 0) {
-    uint32_t tot_tie;
-    warp0_prefix16(sm.wb, sm.wd, &tot_tie);  // tie prefix per warp
-    const uint32_t v = (lane < kRowWarps) ? sm.wa[lane] : 0u;
-    const uint32_t tot_above = __reduce_add_sync(0xffffffffu, v);
-    tot_tie = __shfl_sync(0xffffffffu, tot_tie, 31);
-    // push this CTA's counts to every rank
-    if (lane < CL) {
-      uint32_t *dst = cluster.map_shared_rank(&sm.cnt_all[0][0], lane);
-      dst[2 * c] = tot_above;
-      dst[2 * c + 1] = tot_tie;
-    }
+  uint32_t tot_above, tot_tie;
+  const uint32_t above_before = block_excl_scan<kRowThreads>(n_above, sm.scratch, tot_above);
+  const uint32_t tie_before = block_excl_scan<kRowThreads>(n_tie, sm.scratch, tot_tie);
+  if (tid < CL) {  // push this CTA's counts to every rank
+    uint32_t *dst = cluster.map_shared_rank(&sm.cnt_all[0][0], tid);
+    dst[2 * c] = tot_above;
+    dst[2 * c + 1] = tot_tie;
   }
   cluster.sync();  // every rank's (above, tie) counts are in cnt_all
   if (warp == 0) {
@@ -337,51 +312,30 @@ __device__ void row_topk(RowSmem<D> &sm, const RowParams &p, cg::cluster_group &
     const uint32_t take = (tb >= r3) ? 0u : min(ties, r3 - tb);
     const uint32_t sel = above + take;
     const uint32_t ob = warp_incl_scan(sel) - sel;
-    const uint32_t ob_c = __shfl_sync(0xffffffffu, ob, c);
-    const uint32_t tb_c = __shfl_sync(0xffffffffu, tb, c);
-    // per-warp offsets inside this CTA: warp w selects its above-class
-    // candidates plus its ties whose CTA-wide rank stays below r3 - tb_c
-    uint32_t wsel = 0;
-    if (lane < kRowWarps) {
-      const uint32_t tie_before = tb_c + sm.wd[lane];
-      const uint32_t wt = sm.wb[lane];
-      const uint32_t wtake = (tie_before >= r3) ? 0u : min(wt, r3 - tie_before);
-      wsel = sm.wa[lane] + wtake;
+    if (lane == c) {
+      sm.out_base = ob;
+      sm.tie_base = tb;
+      sm.sel_count = sel;
     }
-    const uint32_t wo = warp_incl_scan(wsel) - wsel;
-    if (lane < kRowWarps) sm.wc[lane] = ob_c + wo;  // output position of that warp's first
-    if (lane == 0) {
-      sm.out_base = ob_c;
-      sm.tie_base = tb_c;
-    }
-    const uint32_t total_sel = __shfl_sync(0xffffffffu, wo + wsel, kRowWarps - 1);
-    if (lane == 0) sm.sel_count = total_sel;
   }
   __syncthreads();
-  // write: warp w walks its candidates in order again
+  // write this thread's selected candidates in index order
   {
-    uint32_t pos = sm.wc[warp];                     // output row position
-    uint32_t tie_rank = sm.tie_base + sm.wd[warp];  // CTA-wide tie rank of the next tie
-    const uint32_t ob = sm.out_base;
-    for (uint32_t i0 = c0; i0 < c1; i0 += 32) {
-      const uint32_t i = i0 + lane;
-      uint2 e = make_uint2(0u, 0u);
-      uint32_t cls = 0u;
-      if (i < c1) {
-        e = cand_at(i);
-        cls = cand_class(e.x, t1, t2, t3, need3);
-      }
-      const uint32_t tbal = __ballot_sync(0xffffffffu, cls == 1u);
-      const bool take = (cls == 2u) || (cls == 1u && tie_rank + __popc(tbal & lt) < r3);
-      const uint32_t sb = __ballot_sync(0xffffffffu, take);
+    const uint32_t ob = sm.out_base, tb = sm.tie_base;
+    const uint32_t room = tb >= r3 ? 0u : r3 - tb;  // ties this CTA may still take
+    uint32_t tie_rank = tie_before;                 // CTA-local rank of the next tie
+    uint32_t at = ob + above_before + min(tie_before, room);
+    for (uint32_t i = i0; i < i1; ++i) {
+      const uint2 e = cand_at(i);
+      const uint32_t cls = cand_class(e.x, t1, t2, t3, need3);
+      bool take = cls == 2u;
+      if (cls == 1u) take = tie_rank++ < room;
       if (take) {
-        const uint32_t at = pos + __popc(sb & lt);
         const int32_t n = (int32_t)(s0 + e.y);
         if (at < (uint32_t)p.topk) orow[at] = n;
         if (at - ob < (uint32_t)kSelCap) sm.sel[at - ob] = n;
+        ++at;
       }
-      pos += __popc(sb);
-      tie_rank += __popc(tbal);
     }
   }
   if (c == CL - 1)
@@ -393,224 +347,6 @@ __device__ void row_topk(RowSmem<D> &sm, const RowParams &p, cg::cluster_group &
 // ---------------------------------------------------------------------------
 // Attention on tensor cores (mma.sync m16n8k16, bf16 x bf16 -> fp32).
 // ---------------------------------------------------------------------------
-__device__ __forceinline__ void mma_bf16(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2,
-                                         uint32_t a3, uint32_t b0, uint32_t b1) {
-  asm volatile(
-      "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, "
-      "{%8,%9}, {%0,%1,%2,%3};"
-      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
-      : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
-}
-
-__device__ __forceinline__ uint32_t lds32(const uint16_t *p) {
-  return *reinterpret_cast<const uint32_t *>(p);
-}
-
-// fp32 pair -> (hi, lo) packed bf16 pairs with x ~= hi + lo.
-__device__ __forceinline__ void split_bf16x2(float x0, float x1, uint32_t &hi, uint32_t &lo) {
-  const __nv_bfloat162 h = __floats2bfloat162_rn(x0, x1);
-  const float2 hf = __bfloat1622float2(h);
-  const __nv_bfloat162 l = __floats2bfloat162_rn(x0 - hf.x, x1 - hf.y);
-  hi = *reinterpret_cast<const uint32_t *>(&h);
-  lo = *reinterpret_cast<const uint32_t *>(&l);
-}
-
-// 8 E2M1 codes (one 32-bit word, element 2i in the low nibble of byte i) ->
-// 8 exact bf16 values (as 4 packed pairs, lower element in the low half).
-__device__ __forceinline__ void e2m1x8_to_bf16(uint32_t word, uint32_t (&o)[4]) {
-  uint32_t h[4];
-  asm("{\n\t.reg .b8 b0, b1, b2, b3;\n\t"
-      "mov.b32 {b0, b1, b2, b3}, %4;\n\t"
-      "cvt.rn.f16x2.e2m1x2 %0, b0;\n\t"
-      "cvt.rn.f16x2.e2m1x2 %1, b1;\n\t"
-      "cvt.rn.f16x2.e2m1x2 %2, b2;\n\t"
-      "cvt.rn.f16x2.e2m1x2 %3, b3;\n\t}"
-      : "=r"(h[0]), "=r"(h[1]), "=r"(h[2]), "=r"(h[3])
-      : "r"(word));
-#pragma unroll
-  for (int i = 0; i < 4; ++i) {
-    const float2 f = __half22float2(*reinterpret_cast<const __half2 *>(&h[i]));
-    const __nv_bfloat162 b = __floats2bfloat162_rn(f.x, f.y);  // exact: <= 3 significant bits
-    o[i] = *reinterpret_cast<const uint32_t *>(&b);
-  }
-}
-
-__device__ __forceinline__ void cp_async16(void *smem_dst, const void *gmem_src) {
-  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(smem_u32(smem_dst)),
-               "l"(gmem_src)
-               : "memory");
-}
-__device__ __forceinline__ void cp_async_wait_all() {
-  asm volatile("cp.async.commit_group;\n\tcp.async.wait_group 0;" ::: "memory");
-}
-
-// Write one key of a chunk into shared memory: kv (keys) and vv (values) are
-// EP/2 packed bf16 pairs for elements [part*EP, part*EP + EP) of key j.
-template <int D>
-__device__ __forceinline__ void store_key_part(RowSmem<D> &sm, int j, int part,
-                                               const uint32_t *kv, const uint32_t *vv) {
-  constexpr int EP = D / 8;
-#pragma unroll
-  for (int u = 0; u < EP / 8; ++u)
-    *reinterpret_cast<uint4 *>(&sm.kb[j][part * EP + 8 * u]) =
-        make_uint4(kv[4 * u], kv[4 * u + 1], kv[4 * u + 2], kv[4 * u + 3]);
-#pragma unroll
-  for (int i = 0; i < EP / 2; ++i) {
-    sm.vt[part * EP + 2 * i][j] = (uint16_t)(vv[i] & 0xffffu);
-    sm.vt[part * EP + 2 * i + 1][j] = (uint16_t)(vv[i] >> 16);
-  }
-}
-
-// Window rows [row0, row0 + nkeys) -> chunk buffers (bf16 as stored, scale 1).
-template <int D>
-__device__ void load_window_chunk(RowSmem<D> &sm, const RowParams &p, int64_t row0, int nkeys) {
-  constexpr int EP = D / 8;  // 512 threads = 64 keys x 8 parts
-  const int tid = threadIdx.x, j = tid % kChunkKeys, part = tid / kChunkKeys;
-  uint32_t kv[EP / 2], vv[EP / 2];
-  const bool ok = j < nkeys;
-  if (ok) {
-    const uint4 *kp = reinterpret_cast<const uint4 *>(p.win_k + (row0 + j) * D + part * EP);
-    const uint4 *vp = reinterpret_cast<const uint4 *>(p.win_v + (row0 + j) * D + part * EP);
-#pragma unroll
-    for (int u = 0; u < EP / 8; ++u) {
-      const uint4 k4 = kp[u], v4 = vp[u];
-      kv[4 * u] = k4.x, kv[4 * u + 1] = k4.y, kv[4 * u + 2] = k4.z, kv[4 * u + 3] = k4.w;
-      vv[4 * u] = v4.x, vv[4 * u + 1] = v4.y, vv[4 * u + 2] = v4.z, vv[4 * u + 3] = v4.w;
-    }
-  } else {
-#pragma unroll
-    for (int i = 0; i < EP / 2; ++i) kv[i] = vv[i] = 0u;
-  }
-  if (EP == 16 || (part & 1) == 0) sm.ks[j][(part * EP) / 16] = 1.0f;
-  if (part == 0) sm.valid[j] = ok;
-  store_key_part<D>(sm, j, part, kv, vv);
-}
-
-// Gathered entries [b0, b0 + nkeys) of the raw batch -> chunk buffers
-// (E2M1 values as exact bf16, group scales kept apart).
-template <int D>
-__device__ void load_entry_chunk(RowSmem<D> &sm, const RowParams &p, int b0, int nkeys) {
-  constexpr int EP = D / 8;
-  const int tid = threadIdx.x, j = tid % kChunkKeys, part = tid / kChunkKeys;
-  uint32_t kv[EP / 2];
-  const int slot = b0 + j;
-  const int32_t n = (j < nkeys) ? sm.raw_idx[slot] : -1;
-  const bool ok = n >= 0 && (int64_t)n < p.N;
-  float s = 0.0f;
-  if (ok) {
-    s = sm.st.raw.scales[slot][(part * EP) / 16];
-    if constexpr (EP == 16) {
-      const uint2 cw = *reinterpret_cast<const uint2 *>(&sm.st.raw.codes[slot][part * 8]);
-      uint32_t o0[4], o1[4];
-      e2m1x8_to_bf16(cw.x, o0);
-      e2m1x8_to_bf16(cw.y, o1);
-#pragma unroll
-      for (int i = 0; i < 4; ++i) {
-        kv[i] = o0[i];
-        kv[4 + i] = o1[i];
-      }
-    } else {
-      const uint32_t cw = *reinterpret_cast<const uint32_t *>(&sm.st.raw.codes[slot][part * 4]);
-      uint32_t o0[4];
-      e2m1x8_to_bf16(cw, o0);
-#pragma unroll
-      for (int i = 0; i < 4; ++i) kv[i] = o0[i];
-    }
-  } else {
-#pragma unroll
-    for (int i = 0; i < EP / 2; ++i) kv[i] = 0u;
-  }
-  if (EP == 16 || (part & 1) == 0) sm.ks[j][(part * EP) / 16] = s;
-  if (part == 0) sm.valid[j] = ok;
-  store_key_part<D>(sm, j, part, kv, kv);
-}
-
-// One head pass's running softmax state (per thread: output fragment of the
-// PV warps, max/sum of the head owned by this warp).
-struct AttnState {
-  float o[4];
-  float m, l;
-};
-
-// Logits, online softmax and PV update of the chunk now in the buffers.
-template <int D>
-__device__ void attend_chunk(RowSmem<D> &sm, const RowParams &p, AttnState &st, int nh) {
-  constexpr int G = D / 16;
-  constexpr int PV_WARPS = D / 8;  // warp w owns output dims [8w, 8w + 8)
-  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  const int gid = lane >> 2, tig = lane & 3;
-  (void)tid;
-  // logits: warp w < 8 owns keys [8w, 8w + 8)
-  if (warp < kChunkKeys / 8) {
-    float sacc[4] = {0.0f, 0.0f, 0.0f, 0.0f};
-    const int key0 = 8 * warp + 2 * tig;  // this thread's two key columns
-#pragma unroll
-    for (int g = 0; g < G; ++g) {
-      float d4[4] = {0.0f, 0.0f, 0.0f, 0.0f};
-      const uint32_t a0 = lds32(&sm.qb[gid][16 * g + 2 * tig]);
-      const uint32_t a1 = lds32(&sm.qb[gid + 8][16 * g + 2 * tig]);
-      const uint32_t a2 = lds32(&sm.qb[gid][16 * g + 8 + 2 * tig]);
-      const uint32_t a3 = lds32(&sm.qb[gid + 8][16 * g + 8 + 2 * tig]);
-      const uint32_t b0 = lds32(&sm.kb[8 * warp + gid][16 * g + 2 * tig]);
-      const uint32_t b1 = lds32(&sm.kb[8 * warp + gid][16 * g + 8 + 2 * tig]);
-      mma_bf16(d4, a0, a1, a2, a3, b0, b1);
-      const float s0 = sm.ks[key0][g], s1 = sm.ks[key0 + 1][g];
-      sacc[0] = fmaf(d4[0], s0, sacc[0]);
-      sacc[1] = fmaf(d4[1], s1, sacc[1]);
-      sacc[2] = fmaf(d4[2], s0, sacc[2]);
-      sacc[3] = fmaf(d4[3], s1, sacc[3]);
-    }
-    const bool v0 = sm.valid[key0], v1 = sm.valid[key0 + 1];
-    sm.s[gid][key0] = v0 ? sacc[0] * p.q_scale : -INFINITY;
-    sm.s[gid][key0 + 1] = v1 ? sacc[1] * p.q_scale : -INFINITY;
-    sm.s[gid + 8][key0] = v0 ? sacc[2] * p.q_scale : -INFINITY;
-    sm.s[gid + 8][key0 + 1] = v1 ? sacc[3] * p.q_scale : -INFINITY;
-  }
-  __syncthreads();
-  // online softmax: warp h owns head h (padding heads get zero weights)
-  {
-    const int h = warp;
-    const float z0 = sm.s[h][lane], z1 = sm.s[h][lane + 32];
-    const float new_m = fmaxf(st.m, warp_max(fmaxf(z0, z1)));
-    float p0 = 0.0f, p1 = 0.0f, corr = 1.0f;
-    if (h < nh && new_m != -INFINITY) {
-      p0 = exp2f(z0 - new_m);
-      p1 = exp2f(z1 - new_m);
-      corr = exp2f(st.m - new_m);  // 0 when the running max is -inf
-      st.l = st.l * corr + warp_sum(p0 + p1);
-      st.m = new_m;
-    }
-    sm.s[h][lane] = p0;
-    sm.s[h][lane + 32] = p1;
-    if (lane == 0) sm.corr[h] = corr;
-  }
-  __syncthreads();
-  // values: warp w < D/8 owns output dims [8w, 8w + 8) in scale group w/2
-  if (warp < PV_WARPS) {
-    const int g = warp >> 1;
-    const float c0 = sm.corr[gid], c1 = sm.corr[gid + 8];
-    st.o[0] *= c0;
-    st.o[1] *= c0;
-    st.o[2] *= c1;
-    st.o[3] *= c1;
-#pragma unroll
-    for (int kk = 0; kk < kChunkKeys / 16; ++kk) {
-      const int k0 = 16 * kk + 2 * tig, k1 = k0 + 8;
-      const float sa = sm.ks[k0][g], sb = sm.ks[k0 + 1][g];
-      const float sc = sm.ks[k1][g], sd = sm.ks[k1 + 1][g];
-      uint32_t ah[4], al[4];
-      split_bf16x2(sm.s[gid][k0] * sa, sm.s[gid][k0 + 1] * sb, ah[0], al[0]);
-      split_bf16x2(sm.s[gid + 8][k0] * sa, sm.s[gid + 8][k0 + 1] * sb, ah[1], al[1]);
-      split_bf16x2(sm.s[gid][k1] * sc, sm.s[gid][k1 + 1] * sd, ah[2], al[2]);
-      split_bf16x2(sm.s[gid + 8][k1] * sc, sm.s[gid + 8][k1 + 1] * sd, ah[3], al[3]);
-      const uint32_t b0 = lds32(&sm.vt[8 * warp + gid][k0]);
-      const uint32_t b1 = lds32(&sm.vt[8 * warp + gid][k1]);
-      mma_bf16(st.o, ah[0], ah[1], ah[2], ah[3], b0, b1);
-      mma_bf16(st.o, al[0], al[1], al[2], al[3], b0, b1);
-    }
-  }
-}
-
 template <int D>
 __device__ void load_q(RowSmem<D> &sm, const RowParams &p, int64_t r, int h0, int nh) {
   // 16-byte pieces: 16 heads x D/8 pieces
@@ -623,97 +359,98 @@ __device__ void load_q(RowSmem<D> &sm, const RowParams &p, int64_t r, int h0, in
   }
 }
 
-// Window rows of this CTA for one head pass.
+// Attention of one head pass: this CTA's window rows and its entries (its
+// own selection `sel`, else the given index slots [lo, hi)), cut into
+// 16-key chunks that kAttnWarps warps take in turn, each with its own
+// running state; the CTA's merged partial of head h then goes to the owner
+// CTA h % CL, which merges the CL partials after one cluster barrier.
 template <int D, int CL>
-__device__ void attend_window(RowSmem<D> &sm, const RowParams &p, AttnState &st, int64_t r,
-                              int c, int nh) {
+__device__ void row_attend(RowSmem<D> &sm, const RowParams &p, cg::cluster_group &cluster,
+                           int64_t r, int c, int h0, int nh, bool from_sel, int64_t lo,
+                           int64_t hi, int64_t sel_base) {
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int64_t b = r / p.T, t = r % p.T;
   const int w_lo = (p.W * c) / CL, w_hi = (p.W * (c + 1)) / CL;
-  const int64_t row0 = b * ((int64_t)p.W - 1 + p.T) + t + w_lo;
-  for (int k0 = 0; k0 < w_hi - w_lo; k0 += kChunkKeys) {
-    __syncthreads();  // chunk buffers free (and q written)
-    load_window_chunk<D>(sm, p, row0 + k0, min(kChunkKeys, w_hi - w_lo - k0));
-    __syncthreads();
-    attend_chunk<D>(sm, p, st, nh);
-  }
-}
-
-// Selected entries [lo, hi) of this CTA's list for one head pass: gathered
-// in batches of kRawCap with async copies, then attended chunk by chunk.
-// `from_sel`: indices come from sm.sel (own selection, beyond kSelCap from
-// the output row) or, when false, straight from the given index row.
-template <int D>
-__device__ void attend_selected(RowSmem<D> &sm, const RowParams &p, AttnState &st, int64_t r,
-                                int64_t lo, int64_t hi, bool from_sel, int64_t sel_base,
-                                int nh) {
-  const int tid = threadIdx.x;
-  const int64_t b = r / p.T;
+  const int nwin = w_hi - w_lo;
+  const int64_t nsel = hi - lo;
+  const int64_t cw = (nwin + ar::kChunk - 1) / ar::kChunk;
+  const int64_t ce = p.N > 0 ? (nsel + ar::kChunk - 1) / ar::kChunk : 0;
   const int32_t *irow = p.idx + r * (int64_t)p.topk;
-  constexpr int CCH = D / 32;                  // 16-byte code chunks per entry
-  constexpr int SCH = (D / 16 * 4 + 15) / 16;  // 16-byte scale chunks per entry
-  for (int64_t bb = lo; bb < hi; bb += kRawCap) {
-    const int nb = (int)min64(kRawCap, hi - bb);
-    __syncthreads();  // raw buffers free
-    for (int i = tid; i < nb; i += kRowThreads) {
-      const int64_t k = bb + i;  // position in this CTA's list / the index row
-      int32_t n;
-      if (from_sel)
-        n = (k - lo < kSelCap) ? sm.sel[k - lo] : irow[sel_base + k - lo];
+  const uint8_t *cseq = p.codes + b * p.N * (D / 2);
+  const float *sseq = p.scales + b * p.N * (D / 16);
+  const int64_t wrow0 = b * ((int64_t)p.W - 1 + p.T) + t + w_lo;
+  __syncthreads();  // top-k buffers dead, query in place
+  if (warp < kAttnWarps) {
+    ar::WarpArea<D> &wa = sm.u.aw[warp];
+    ar::WarpState<D> st;
+    ar::state_init(st);
+    const int64_t nch = cw + ce;
+    auto entry_of = [&](int64_t ch) -> int32_t {  // this lane's key of entry chunk ch
+      const int64_t k = (ch - cw) * ar::kChunk + (lane & 15);
+      if (k >= nsel) return -1;
+      if (from_sel) return (k < kSelCap) ? sm.sel[k] : irow[sel_base + k];
+      return irow[lo + k];
+    };
+    // this warp's first entry chunk is gathered before its window chunks run
+    int64_t ech = warp;
+    while (ech < cw) ech += kAttnWarps;
+    uint32_t mask_cur = 0u;
+    if (ech < nch) mask_cur = ar::gather_entries<D>(wa, 0, entry_of(ech), p.N, cseq, sseq);
+    for (int64_t ch = warp; ch < cw; ch += kAttnWarps) {
+      const int j0 = (int)ch * ar::kChunk;
+      const uint32_t mask = ar::load_window_rows<D>(wa, p.win_k, p.win_v, wrow0 + j0,
+                                                    min(ar::kChunk, nwin - j0));
+      ar::attend_chunk16<D>(wa, sm.qb, st, mask, true, nullptr, p.q_scale);
+      __syncwarp();
+    }
+    // entry chunks, the next one gathered while the current one is used
+    for (int it = 0; ech < nch; ++it, ech += kAttnWarps) {
+      const int sb = it & 1;
+      uint32_t mask_next = 0u;
+      const bool more = ech + kAttnWarps < nch;
+      if (more) mask_next = ar::gather_entries<D>(wa, sb ^ 1, entry_of(ech + kAttnWarps), p.N, cseq, sseq);
+      if (more)
+        ar::cp_wait<1>();
       else
-        n = irow[k];
-      const bool ok = n >= 0 && (int64_t)n < p.N;
-      if (n >= 0 && !ok) raise_status(kStatusBadIndex);
-      sm.raw_idx[i] = ok ? n : -1;
-      if (ok) {
-        const int64_t row = b * p.N + n;
-        const uint8_t *cp = p.codes + row * (D / 2);
-        const float *sp = p.scales + row * (D / 16);
-#pragma unroll
-        for (int u = 0; u < CCH; ++u) cp_async16(&sm.st.raw.codes[i][16 * u], cp + 16 * u);
-#pragma unroll
-        for (int u = 0; u < SCH; ++u) cp_async16(&sm.st.raw.scales[i][4 * u], sp + 4 * u);
-      }
+        ar::cp_wait<0>();
+      __syncwarp();
+      ar::convert_entries<D>(wa, sb);
+      __syncwarp();
+      ar::attend_chunk16<D>(wa, sm.qb, st, mask_cur, false, wa.s.scales[sb], p.q_scale);
+      __syncwarp();
+      mask_cur = mask_next;
     }
-    cp_async_wait_all();
-    __syncthreads();
-    for (int k0 = 0; k0 < nb; k0 += kChunkKeys) {
-      if (k0 > 0) __syncthreads();  // previous chunk consumed
-      load_entry_chunk<D>(sm, p, k0, min(kChunkKeys, nb - k0));
-      __syncthreads();
-      attend_chunk<D>(sm, p, st, nh);
-    }
+    ar::store_state<D>(wa, st);
   }
-}
-
-// Push this CTA's partial of heads h0..h0+nh-1 to the owners, barrier, merge
-// the heads this CTA owns.
-template <int D, int CL>
-__device__ void merge_heads(RowSmem<D> &sm, const RowParams &p, cg::cluster_group &cluster,
-                            const AttnState &st, int64_t r, int h0, int nh) {
-  constexpr int PV_WARPS = D / 8;
-  constexpr int DL = D / 32;
-  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-  const int gid = lane >> 2, tig = lane & 3;
-  const int c = (int)cluster.block_rank();
-  // head h's partial goes to CTA h % CL, inbox slot (h / CL) * CL + c
-  if (warp < PV_WARPS) {
-    const int d0 = 8 * warp + 2 * tig;
+  __syncthreads();
+  // per head: the max over the warps and each warp's factor
+  for (int i = tid; i < nh * kAttnWarps; i += kRowThreads) {
+    const int h = i / kAttnWarps, w = i % kAttnWarps;
+    float M = -INFINITY;
 #pragma unroll
-    for (int half = 0; half < 2; ++half) {
-      const int h = gid + 8 * half;
-      float *dst = cluster.map_shared_rank(&sm.inbox[0][0], h % CL) + ((h / CL) * CL + c) * (D + 2);
-      dst[2 + d0] = st.o[2 * half];
-      dst[2 + d0 + 1] = st.o[2 * half + 1];
-    }
+    for (int v = 0; v < kAttnWarps; ++v) M = fmaxf(M, sm.u.aw[v].merge.m[h]);
+    sm.mf[h][w] = M == -INFINITY ? 0.0f : exp2f(sm.u.aw[w].merge.m[h] - M);
+    if (w == 0) sm.mf[h][kAttnWarps] = M;
   }
-  if (lane == 0) {  // warp h holds the max and sum of head h
-    const int h = warp;
+  __syncthreads();
+  // this CTA's partial of each head (max, sum, acc) -> inbox slot
+  // (h / CL) * CL + c of the owner CTA h % CL
+  for (int i = tid; i < nh * (D + 2); i += kRowThreads) {
+    const int h = i / (D + 2), e = i % (D + 2);
+    float v = 0.0f;
+    if (e == 0) {
+      v = sm.mf[h][kAttnWarps];
+    } else {
+#pragma unroll
+      for (int w = 0; w < kAttnWarps; ++w)
+        v = fmaf(e == 1 ? sm.u.aw[w].merge.l[h] : sm.u.aw[w].merge.o[h][e - 2], sm.mf[h][w], v);
+    }
     float *dst = cluster.map_shared_rank(&sm.inbox[0][0], h % CL) + ((h / CL) * CL + c) * (D + 2);
-    dst[0] = st.m;
-    dst[1] = st.l;
+    dst[e] = v;
   }
   cluster.sync();
-  // merge: warp k merges head h = c + k*CL from CL partials in the inbox
+  // merge: warp k merges head h = c + k*CL from the CL partials in the inbox
+  constexpr int DL = D / 32;
   const int h = c + warp * CL;
   if (warp < kHeads / CL && h < nh) {
     const float *slot = &sm.inbox[warp * CL][0];
@@ -747,7 +484,6 @@ __device__ void merge_heads(RowSmem<D> &sm, const RowParams &p, cg::cluster_grou
   }
 }
 
-// grid.x = rows * CL, cluster (CL, 1, 1).
 template <int D, int CL>
 __global__ void __launch_bounds__(kRowThreads, 1) row_cluster_kernel(const RowParams p) {
   extern __shared__ __align__(128) unsigned char row_smem_raw[];
@@ -765,20 +501,19 @@ __global__ void __launch_bounds__(kRowThreads, 1) row_cluster_kernel(const RowPa
   const int64_t s1 = (c == CL - 1) ? V : (((V * (c + 1)) / CL) & ~int64_t(15));
   const bool topk_here = p.do_topk && K > 0;
 
+  // Every CTA of the cluster must be running before any of them writes into
+  // another's shared memory: arrive now, wait before the first such write.
+  asm volatile("barrier.cluster.arrive.relaxed.aligned;" ::: "memory");
   if (tid == 0) {
     mbar_init(&sm.bar, 1);
     fence_barrier_init();
   }
   __syncthreads();
-  // Prologue, independent of the scan that produced the scores: the query and
-  // the window part of attention.  With programmatic dependent launch this
-  // overlaps the scan's tail.
+  // Prologue, independent of the scan that produced the scores: the query.
+  // With programmatic dependent launch this overlaps the scan's tail.
   for (int i = tid; i < kBins2; i += kRowThreads) sm.h2[i] = 0u;
-  AttnState st{{0.0f, 0.0f, 0.0f, 0.0f}, -INFINITY, 0.0f};
-  if (p.do_attn) {
-    load_q<D>(sm, p, r, 0, min(kHeads, p.H));
-    attend_window<D, CL>(sm, p, st, r, c, min(kHeads, p.H));
-  }
+  if (p.do_attn) load_q<D>(sm, p, r, 0, min(kHeads, p.H));
+  asm volatile("barrier.cluster.wait.aligned;" ::: "memory");
   pdl_wait_primary();  // the scores and histograms are complete from here on
   if (topk_here && tid == 0) {
     const int n0 = (int)min64(kStageScores, s1 - s0);
@@ -787,7 +522,7 @@ __global__ void __launch_bounds__(kRowThreads, 1) row_cluster_kernel(const RowPa
     mbar_arrive_expect_tx(&sm.bar, bytes);
     bulk_g2s(sm.h1, p.hist1 + r_local * kBins1, kBins1 * 4, &sm.bar);
     if (bulk && n0 > 0)
-      bulk_g2s(sm.st.sc, p.scores + r_local * p.score_stride + s0,
+      bulk_g2s(sm.u.tk.sc, p.scores + r_local * p.score_stride + s0,
                (uint32_t)(((n0 + 3) & ~3) * 4), &sm.bar);
   }
 
@@ -825,16 +560,8 @@ __global__ void __launch_bounds__(kRowThreads, 1) row_cluster_kernel(const RowPa
         cluster.sync();  // the previous merge read this CTA's inbox
         __syncthreads();
         load_q<D>(sm, p, r, h0, nh);
-        st = AttnState{{0.0f, 0.0f, 0.0f, 0.0f}, -INFINITY, 0.0f};
-        attend_window<D, CL>(sm, p, st, r, c, nh);
       }
-      if (p.do_topk) {
-        attend_selected<D>(sm, p, st, r, lo, hi, true, sel_base, nh);
-      } else {
-        attend_selected<D>(sm, p, st, r, lo, hi, false, 0, nh);
-      }
-      __syncthreads();
-      merge_heads<D, CL>(sm, p, cluster, st, r, h0, nh);
+      row_attend<D, CL>(sm, p, cluster, r, c, h0, nh, p.do_topk != 0, lo, hi, sel_base);
     }
   }
   if (abort && tid == 0 && phases > 0)  // let a late bulk copy land before exit
