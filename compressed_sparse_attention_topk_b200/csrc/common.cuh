@@ -178,8 +178,10 @@ __device__ __forceinline__ uint32_t block_excl_scan(uint32_t v, uint32_t *scratc
 
 // Radix threshold over a histogram of NBINS counts (in shared or global
 // memory): the largest bin t with sum(hist[t..]) >= need, and the count of
-// elements strictly above it.  need >= 1 and sum(hist) >= need required.
-// Result in out[0] (bin) and out[1] (count above).  Contains __syncthreads().
+// elements strictly above it.  When sum(hist) < need (only after an aborted
+// producer) the result is bin 0 with the count above it, so that every CTA
+// reading the same histogram still takes the same decisions.  Result in
+// out[0] (bin) and out[1] (count above).  Contains __syncthreads().
 template <int THREADS, int NBINS>
 __device__ void radix_threshold(const uint32_t *hist, uint32_t need, uint32_t *scratch,
                                 uint32_t *out) {
@@ -197,8 +199,15 @@ __device__ void radix_threshold(const uint32_t *hist, uint32_t need, uint32_t *s
     local[i] = hist[hi - 1 - i];
     s += local[i];
   }
+  if (tid == THREADS - 1) {  // default (sum < need): bin 0; bins [1, hi) of this thread counted below
+    uint32_t a = 0;
+    for (int i = 0; i < BPT - 1; ++i) a += local[i];
+    out[0] = 0u;
+    out[1] = a;  // completed by the scan below
+  }
   uint32_t total;
   uint32_t above = block_excl_scan<THREADS>(s, scratch, total);
+  if (tid == THREADS - 1 && total < need) out[1] += above;
   if (above < need && above + s >= need) {
     uint32_t acc = above;
 #pragma unroll

@@ -120,7 +120,7 @@ TopkWs topk_ws_layout(void *base, int64_t R, int64_t N) {
   };
   const size_t o_scores = take(size_t(R) * score_stride(N) * 4);
   const size_t o_cand = take(size_t(R) * N * 8);
-  const size_t o_hist = take(size_t(R) * kBins1 * 4);
+  const size_t o_hist = take(size_t(R) * kHistStride * 4);
   char *p = static_cast<char *>(base);
   w.scores = reinterpret_cast<float *>(p + o_scores);
   w.cand = reinterpret_cast<uint2 *>(p + o_cand);
@@ -623,7 +623,7 @@ csa2_status run_index_topk(const int8_t *q_idx, const float *w, const int8_t *k_
 
   for (int64_t row0 = 0; row0 < rows; row0 += R) {
     const int64_t nr = std::min<int64_t>(R, rows - row0);
-    if (cudaMemsetAsync(L.hist1, 0, size_t(nr) * kBins1 * 4, st) != cudaSuccess)
+    if (cudaMemsetAsync(L.hist1, 0, size_t(nr) * kHistStride * 4, st) != cudaSuccess)
       return CSA2_ERR_CUDA;
     const int64_t stride = score_out ? N : score_stride(N);
     float *scores = score_out ? score_out + row0 * N : L.scores;

@@ -25,6 +25,9 @@
 namespace csa2 {
 
 constexpr int kScanThreads = 256;
+// Per-row histogram rows in global memory: kBins1 counters (zeroed before
+// the scan), padded to keep rows 16-byte aligned.
+constexpr int kHistStride = kBins1 + 4;
 
 template <int DI, int HI>
 struct ScanShape {
@@ -44,7 +47,7 @@ __device__ __forceinline__ int chunk_xor(int t) {
   return (NCH == 1) ? 0 : (t / (8 / NCH)) % NCH;
 }
 
-// grid = (G slices, rows).
+// grid = (G slices, rows).  hist1: [rows][kHistStride], zeroed.
 template <int DI, int HI>
 __global__ void __launch_bounds__(kScanThreads, 2)
     index_scan_kernel(const int8_t *__restrict__ q_idx, const float *__restrict__ w,
@@ -192,7 +195,7 @@ __global__ void __launch_bounds__(kScanThreads, 2)
   }
 
   __syncthreads();
-  uint32_t *grow = hist1 + r_local * kBins1;
+  uint32_t *grow = hist1 + r_local * kHistStride;
   for (int i = tid; i < kBins1; i += kScanThreads) {
     const uint32_t v = sh_hist[i];
     if (v) atomicAdd(grow + i, v);

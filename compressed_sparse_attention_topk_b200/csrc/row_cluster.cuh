@@ -17,19 +17,19 @@
 // score slice in shared memory with bulk copies, then
 //   1. finds the digit-1 threshold t1 (largest digit whose suffix count
 //      reaches k) and lists the elements of its slice with digit 1 >= t1,
-//      in index order (each warp walks a contiguous segment: a count pass,
-//      one prefix over warps, a write pass), histogramming digit 2 of the
-//      elements exactly at t1;
+//      in index order (each thread masks a contiguous run, one block
+//      prefix, then each thread writes its run's candidates), histogramming
+//      digit 2 of the elements exactly at t1;
 //   2. reduces the cluster's digit-2 histograms (CTA c sums bin slice c of
-//      every rank; every CTA then locates the threshold slice from the
-//      slice totals and reads only that slice) -> t2;
+//      every rank and pushes the sums to every rank; every CTA then finds
+//      t2 locally) -> t2;
 //   3. only when the boundary bucket (t1, t2) holds more elements than still
 //      needed: the same for digit 3 -> t3;
 //   4. classifies the candidates as above the threshold key or equal to
 //      it.  Equal keys are equal scores; they are taken in index order
 //      (lower index first) up to the count still needed.  Prefix sums over
-//      ranks and warps give every warp its offset in the output row, so the
-//      indices come out ascending.
+//      ranks and threads give every thread its offset in the output row, so
+//      the indices come out ascending.
 //
 // Attention: each CTA attends over an even share of the window rows and over
 // the entries it selected itself (with given indices, an even share of the
@@ -74,7 +74,7 @@ struct RowParams {
   // top-k
   const float *scores;      // [rows_local, score_stride] (this launch's rows)
   int64_t score_stride;
-  const uint32_t *hist1;    // [rows_local, kBins1]
+  const uint32_t *hist1;    // [rows_local, kHistStride] (digit-1 histogram first)
   uint2 *cand;              // [rows_local, N] candidate overflow regions
   int64_t N;
   int32_t T;
@@ -388,8 +388,11 @@ __device__ void row_attend(RowSmem<D> &sm, const RowParams &p, cg::cluster_group
     auto entry_of = [&](int64_t ch) -> int32_t {  // this lane's key of entry chunk ch
       const int64_t k = (ch - cw) * ar::kChunk + (lane & 15);
       if (k >= nsel) return -1;
-      if (from_sel) return (k < kSelCap) ? sm.sel[k] : irow[sel_base + k];
-      return irow[lo + k];
+      if (from_sel) {
+        if (k < kSelCap) return sm.sel[k];
+        return (sel_base + k < p.topk) ? irow[sel_base + k] : -1;
+      }
+      return (lo + k < p.topk) ? irow[lo + k] : -1;
     };
     // this warp's first entry chunk is gathered before its window chunks run
     int64_t ech = warp;
@@ -520,7 +523,7 @@ __global__ void __launch_bounds__(kRowThreads, 1) row_cluster_kernel(const RowPa
     uint32_t bytes = kBins1 * 4;
     if (bulk && n0 > 0) bytes += (uint32_t)(((n0 + 3) & ~3) * 4);
     mbar_arrive_expect_tx(&sm.bar, bytes);
-    bulk_g2s(sm.h1, p.hist1 + r_local * kBins1, kBins1 * 4, &sm.bar);
+    bulk_g2s(sm.h1, p.hist1 + r_local * kHistStride, kBins1 * 4, &sm.bar);
     if (bulk && n0 > 0)
       bulk_g2s(sm.u.tk.sc, p.scores + r_local * p.score_stride + s0,
                (uint32_t)(((n0 + 3) & ~3) * 4), &sm.bar);
