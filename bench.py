@@ -74,6 +74,26 @@ def measured_peaks():
     return FALLBACK_HBM_GBS, "fallback"
 
 
+def pack_into_one_buffer(layers, keys, dev):
+    """Move layers[l][k] (k in keys) into one uint8 device buffer, each tensor
+    at a 256-byte aligned offset, and replace them by views of it (same dtype
+    and shape).  Returns the buffer and the bytes it holds."""
+    import torch
+    plan, off = [], 0
+    for l, d in enumerate(layers):
+        for k in keys:
+            nb = d[k].numel() * d[k].element_size()
+            plan.append((l, k, off, nb))
+            off += (nb + 255) // 256 * 256
+    buf = torch.zeros(off, dtype=torch.uint8, device=dev)
+    for l, k, o, nb in plan:
+        t = layers[l][k]
+        v = buf[o:o + nb].view(t.dtype).view(t.shape)
+        v.copy_(t)
+        layers[l][k] = v
+    return buf, off
+
+
 def scan_source_sha() -> str:
     h = hashlib.sha256()
     for f in ("index_scan.cuh", "common.cuh"):
@@ -256,6 +276,13 @@ def run_gpu(args, w0):
         d["lse"] = torch.empty((w0.B, w0.H), dtype=torch.float32, device=dev)
         tens.append(d)
     torch.cuda.synchronize()
+    # Per-token inputs and per-step results of all layers live as views of one
+    # device buffer each (256-byte aligned slots), so a step moves them with
+    # one host->device and one device->host copy, as a serving loop would.
+    in_keys = ("q", "q_idx", "w", "win_k", "win_v")
+    out_keys = ("out", "lse", "idx")
+    dev_in, _ = pack_into_one_buffer(tens, in_keys, dev)
+    dev_out, _ = pack_into_one_buffer(tens, out_keys, dev)
     dims = csa2.make_dims(w0.B, w0.T, w0.H, w0.D, w0.N, w0.H_I, w0.d_I, w0.topk, w0.W,
                           w0.n_prior, w0.ratio, w0.sm_scale)
     group = csa2.LayerGroup(list(w0.modes), tens, dims)
@@ -358,13 +385,10 @@ def run_gpu(args, w0):
     launches_per_step = len(recs) / args.steps
 
     # ---- e2e: pinned host inputs -> device, hot path, results -> host ----
-    in_keys = ("q", "q_idx", "w", "win_k", "win_v")
-    out_keys = ("out", "lse", "idx")
-    host_in = [{k: tens[l][k].cpu().pin_memory() for k in in_keys} for l in range(w0.L)]
-    host_out = [{k: torch.empty_like(tens[l][k], device="cpu").pin_memory() for k in out_keys}
-                for l in range(w0.L)]
-    h2d = sum(t.numel() * t.element_size() for d in host_in for t in d.values())
-    d2h = sum(t.numel() * t.element_size() for d in host_out for t in d.values())
+    host_in = dev_in.cpu().pin_memory()
+    host_out = torch.empty_like(dev_out, device="cpu").pin_memory()
+    h2d = host_in.numel()
+    d2h = host_out.numel()
 
     def e2e_steps(K):
         res = []
@@ -373,9 +397,7 @@ def run_gpu(args, w0):
             flush()
             a, b = ev(), ev()
             a.record(stream)
-            for l in range(w0.L):
-                for k in in_keys:
-                    tens[l][k].copy_(host_in[l][k], non_blocking=True)
+            dev_in.copy_(host_in, non_blocking=True)
             b.record(stream)
             segs = [(a, b)]
             for l in range(w0.L):
@@ -385,9 +407,7 @@ def run_gpu(args, w0):
                 a.record(stream)
                 graphs[l].replay()
                 if l == w0.L - 1:
-                    for ll in range(w0.L):
-                        for k in out_keys:
-                            host_out[ll][k].copy_(tens[ll][k], non_blocking=True)
+                    host_out.copy_(dev_out, non_blocking=True)
                 b.record(stream)
                 segs.append((a, b))
             res.append(segs)
