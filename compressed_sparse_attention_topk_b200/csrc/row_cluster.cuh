@@ -65,10 +65,10 @@ namespace cg = cooperative_groups;
 constexpr int kRowThreads = 512;
 constexpr int kRowWarps = kRowThreads / 32;
 constexpr int kStageScores = 16384;  // scores staged in shared memory per round
-constexpr int kCandCap = 4096;       // candidates kept in shared memory
+constexpr int kCandCap = 2048;       // candidates kept in shared memory (more spill to global)
 constexpr int kSelCap = 4096;        // selected indices kept in shared memory
 constexpr int kHeads = 16;           // heads per pass (the MMA's M)
-constexpr int kAttnWarps = 8;        // warps that run attention chunks
+constexpr int kAttnWarps = 7;        // warps that run attention chunks
 
 struct RowParams {
   // top-k
@@ -101,8 +101,7 @@ struct RowSmem {
   union {
     struct {  // top-k working set
       float sc[kStageScores];                                    // staged score slice
-      uint2 cand[kCandCap];                                      // candidates (key, index - slice start)
-      uint32_t masks[kRowWarps][kStageScores / kRowWarps / 32];  // per-warp ballots of a round
+      uint2 cand[kCandCap];    // candidates (key, index - slice start); more spill to global
     } tk;
     ar::WarpArea<D> aw[kAttnWarps];  // attention: per-warp chunk buffers, then partial states
   } u;
@@ -112,7 +111,6 @@ struct RowSmem {
   uint32_t full[kBins2];        // cluster-wide histogram (reduced slices pushed by owners)
   uint32_t cnt_all[32][2];      // every rank's (above, tie) counts (pushed)
   int32_t sel[kSelCap];         // this CTA's selected indices, ascending
-  uint32_t wa[kRowWarps], wb[kRowWarps], wc[kRowWarps], wd[kRowWarps];
   uint16_t qb[kHeads][D + 8];   // query of the head pass, bf16
   float inbox[kHeads][D + 2];   // pushed partials (m, l, acc) of the heads this CTA merges
   float mf[kHeads][kAttnWarps + 1];  // per head: each attention warp's factor, then the max
@@ -173,17 +171,6 @@ __device__ void cluster_threshold(RowSmem<D> &sm, cg::cluster_group &cluster, ui
   __syncthreads();
 }
 
-// Exclusive prefix of one value per warp (sm.* arrays of kRowWarps), done by
-// warp 0; returns nothing, writes the prefix into `dst` and the total into
-// dst_total.  Caller synchronises before and after.
-__device__ __forceinline__ void warp0_prefix16(const uint32_t *src, uint32_t *dst,
-                                               uint32_t *dst_total) {
-  const int lane = threadIdx.x & 31;
-  const uint32_t v = (lane < kRowWarps) ? src[lane] : 0u;
-  const uint32_t incl = warp_incl_scan(v);
-  if (lane < kRowWarps) dst[lane] = incl - v;
-  if (lane == 31) *dst_total = incl;
-}
 
 template <int D, int CL>
 __device__ void row_topk(RowSmem<D> &sm, const RowParams &p, cg::cluster_group &cluster,
