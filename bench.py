@@ -483,8 +483,9 @@ def run_gpu(args, w0):
 
 
 def run_prefill(args, w0):
-    """Supplementary measurement of a chunked-prefill layer (index + top-k
-    over the visible prefix of every query, then attention), one GPU."""
+    """Supplementary measurement of one layer with several query tokens per
+    sequence (a chunked prefill, or multi-token decode): index + top-k over
+    the visible entries of every query, then attention; one GPU."""
     import torch
     import compressed_sparse_attention_topk_b200 as csa2
     torch.cuda.set_device(0)
@@ -529,7 +530,8 @@ def run_prefill(args, w0):
         c, s_ = per.get(name, (0, 0.0))
         per[name] = (c + 1, s_ + m)
     print(json.dumps({
-        "metric": "CSA2 chunked-prefill tokens/s per layer (supplementary)",
+        "metric": ("CSA2 chunked-prefill tokens/s per layer (supplementary)" if w0.n_prior >= 0
+                   else "CSA2 multi-token decode tokens/s per layer (supplementary)"),
         "value": w0.B * w0.T / (ms * 1e-3), "unit": "tokens/s/layer", "ms_per_layer": ms,
         "steps": args.steps, "config": {"workload": w0.name, "T": w0.T, "N": w0.N,
                                           "n_prior": w0.n_prior, "topk": w0.topk},

@@ -176,6 +176,40 @@ ScanLaunch pick_scan(int32_t d_I, int32_t H_I) {
   return nullptr;
 }
 
+template <int DI, int HI, int TQ>
+void launch_scan_group(dim3 grid, cudaStream_t st, const int8_t *q_idx, const float *w,
+                       const int8_t *k_idx, int32_t T, int64_t N, int64_t n_prior, int32_t ratio,
+                       int64_t row0, float *scores, int64_t stride, uint32_t *hist1,
+                       int write_masked) {
+  using S = ScanGroupShape<DI, HI, TQ>;
+  static bool done[256] = {false};
+  int dev = 0;
+  cudaGetDevice(&dev);
+  if (dev < 0 || dev >= 256 || !done[dev]) {
+    set_smem_attr(index_scan_group_kernel<DI, HI, TQ>, S::SMEM, false);
+    if (dev >= 0 && dev < 256) done[dev] = true;
+  }
+  index_scan_group_kernel<DI, HI, TQ><<<grid, S::THREADS, S::SMEM, st>>>(
+      q_idx, w, k_idx, T, N, n_prior, ratio, row0, scores, stride, hist1, write_masked);
+}
+
+// Several query rows per sequence (2 <= T <= 8, d_I <= 64): one scan of the
+// keys serves all of them.
+ScanLaunch pick_scan_group(int32_t d_I, int32_t H_I, int32_t T) {
+  if (T < 2 || T > 8 || d_I > 64) return nullptr;
+#define CSA2_SG_CASE(DI, HI)                                                    \
+  if (d_I == DI && H_I == HI) {                                                 \
+    if (T <= 2) return &launch_scan_group<DI, HI, 2>;                           \
+    if (T <= 4) return &launch_scan_group<DI, HI, 4>;                           \
+    return &launch_scan_group<DI, HI, 8>;                                       \
+  }
+  CSA2_SG_CASE(16, 1) CSA2_SG_CASE(16, 2) CSA2_SG_CASE(16, 4) CSA2_SG_CASE(16, 8)
+  CSA2_SG_CASE(32, 1) CSA2_SG_CASE(32, 2) CSA2_SG_CASE(32, 4) CSA2_SG_CASE(32, 8)
+  CSA2_SG_CASE(64, 1) CSA2_SG_CASE(64, 2) CSA2_SG_CASE(64, 4) CSA2_SG_CASE(64, 8)
+#undef CSA2_SG_CASE
+  return nullptr;
+}
+
 // ---- the per-row cluster kernel -------------------------------------------
 template <int D, int CL>
 csa2_status launch_row_cl(const RowParams &p, int64_t nr, cudaStream_t st) {
@@ -613,12 +647,15 @@ csa2_status run_index_topk(const int8_t *q_idx, const float *w, const int8_t *k_
     return run_attn(att->q, att->codes, att->scales, idx_out, att->win_k, att->win_v, B, T,
                     att->H, att->D, N, topk, att->W, att->sm_scale, att->out, att->lse, st);
   }
-  const int64_t R = topk_rows_per_pass(rows, N);
-  const TopkWs L0 = topk_ws_layout(nullptr, R, N);
+  const int64_t R0 = topk_rows_per_pass(rows, N);
+  const TopkWs L0 = topk_ws_layout(nullptr, R0, N);
   if (!ws || ws_bytes < L0.bytes || !aligned(ws, 16)) return CSA2_ERR_WORKSPACE;
-  const TopkWs L = topk_ws_layout(ws, R, N);
+  const TopkWs L = topk_ws_layout(ws, R0, N);
   const ScanLaunch scan = pick_scan(d_I, H_I);
   if (!scan) return CSA2_ERR_UNSUPPORTED;
+  // several rows per sequence: whole sequences per pass, one shared scan each
+  const ScanLaunch scan_group = pick_scan_group(d_I, H_I, T);
+  const int64_t R = (scan_group && R0 >= T) ? R0 / T * T : R0;
   const int sms = device_sms();
 
   for (int64_t row0 = 0; row0 < rows; row0 += R) {
@@ -629,13 +666,15 @@ csa2_status run_index_topk(const int8_t *q_idx, const float *w, const int8_t *k_
     float *scores = score_out ? score_out + row0 * N : L.scores;
     // scan: about two CTAs per SM in total (the slices of a row are balanced
     // to 16 keys), at least 256 keys per CTA
-    const int64_t g_want = std::max<int64_t>(1, (2 * sms + nr / 2) / nr);
+    const bool grouped = scan_group && R >= T;  // passes hold whole sequences
+    const int64_t units = grouped ? nr / T : nr;  // CTA groups: sequences or rows
+    const int64_t g_want = std::max<int64_t>(1, (2 * sms + units / 2) / units);
     const int64_t g_max = std::max<int64_t>(1, N / 256);
     const int G = (int)std::min(g_want, g_max);
     {
       TraceScope ts("index_scan", st);
-      scan(dim3(G, (unsigned)nr), st, q_idx, w, k_idx, T, N, n_prior, ratio, row0, scores,
-           stride, L.hist1, score_out != nullptr);
+      (grouped ? scan_group : scan)(dim3(G, (unsigned)units), st, q_idx, w, k_idx, T, N, n_prior,
+                                    ratio, row0, scores, stride, L.hist1, score_out != nullptr);
     }
     if (after_launch() != CSA2_OK) return CSA2_ERR_CUDA;
     RowParams p{};

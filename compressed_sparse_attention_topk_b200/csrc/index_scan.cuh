@@ -17,8 +17,8 @@
 // threads of a 128-byte shared-memory phase hit 8 different 16-byte bank
 // groups, and holds its index-query chunks pre-permuted the same way, so the
 // dot product needs no data-dependent register indexing.  The score's top
-// radix digit goes to a shared-memory histogram (warp-aggregated), merged
-// into the row's global histogram at the end for the top-k selection.
+// radix digit goes to a shared-memory histogram, merged into the row's
+// global histogram at the end for the top-k selection.
 #pragma once
 #include "common.cuh"
 
@@ -61,7 +61,7 @@ __global__ void __launch_bounds__(kScanThreads, 2)
   __shared__ uint32_t sh_hist[kBins1];
   __shared__ __align__(16) int4 sh_q[S::QREG ? 1 : HI * NCH];
 
-  const int tid = threadIdx.x, lane = tid & 31;
+  const int tid = threadIdx.x;
   const int64_t r_local = blockIdx.y, r = row0 + r_local;
   const int64_t b = r / T, t = r % T;
   const int G = gridDim.x, g = blockIdx.x;
@@ -167,12 +167,9 @@ __global__ void __launch_bounds__(kScanThreads, 2)
         score = __fadd_rn(acc, 0.0f);
         srow[tbase + kl] = score;
       }
-      const uint32_t bin = key_d1(score_key(score));
-      const uint32_t active = __ballot_sync(0xffffffffu, valid);
-      if (valid) {
-        const uint32_t peers = __match_any_sync(active, bin);
-        if (lane == __ffs(peers) - 1) atomicAdd(&sh_hist[bin], __popc(peers));
-      }
+      // plain shared-memory reduction (a warp-aggregating match costs more
+      // on its narrow issue pipe than the bin conflicts it saves)
+      if (valid) atomicAdd(&sh_hist[key_d1(score_key(score))], 1u);
     }
   }
   if (abort_it >= 0) {
@@ -199,6 +196,196 @@ __global__ void __launch_bounds__(kScanThreads, 2)
   for (int i = tid; i < kBins1; i += kScanThreads) {
     const uint32_t v = sh_hist[i];
     if (v) atomicAdd(grow + i, v);
+  }
+}
+
+}  // namespace csa2
+
+namespace csa2 {
+
+// ---------------------------------------------------------------------------
+// Several queries of one sequence (multi-token decode, e.g. a few draft
+// tokens verified together): the CTAs of a sequence stream its keys once and
+// score every query row of the sequence against each key, so the key bytes
+// per token fall by the number of rows.  Two warps per query row: warp 2t+i
+// scores half of every key tile against row t, with the row's index query in
+// registers (pre-permuted by the lane's chunk rotation, as above), so shared
+// memory serves only key chunks.  Same score, histogram and slice rules as
+// index_scan_kernel; row t sees n < V_t.
+// grid = (G slices, sequences of the pass); block = 64 * TQ threads; rows of
+// sequence b are b*T .. b*T + T - 1 (T <= TQ); hist1 rows per query row.
+// ---------------------------------------------------------------------------
+template <int DI, int HI, int TQ>
+struct ScanGroupShape {
+  static_assert(DI <= 64, "16 KiB key tiles");
+  static constexpr int THREADS = 64 * TQ;
+  static constexpr int NCH = DI / 16;
+  static constexpr int TILE_KEYS = 16384 / DI;            // 16 KiB tiles
+  static constexpr int TILE_BYTES = 16384;
+  static constexpr int KPL = TILE_KEYS / 64;              // keys per lane and tile
+  static constexpr int STAGES = 4;
+  static constexpr bool QREG = HI * NCH <= 16;            // index query fits in registers
+  static constexpr size_t HIST_BYTES = size_t(TQ) * kBins1 * 4;
+  static constexpr size_t SMEM = size_t(STAGES) * TILE_BYTES + HIST_BYTES;
+};
+
+template <int DI, int HI, int TQ>
+__global__ void __launch_bounds__(64 * TQ, TQ <= 4 ? 2 : 1)
+    index_scan_group_kernel(const int8_t *__restrict__ q_idx, const float *__restrict__ w,
+                            const int8_t *__restrict__ k_idx, int32_t T, int64_t N,
+                            int64_t n_prior, int32_t ratio, int64_t row0,
+                            float *__restrict__ scores, int64_t score_stride,
+                            uint32_t *__restrict__ hist1, int write_masked) {
+  using S = ScanGroupShape<DI, HI, TQ>;
+  constexpr int NCH = S::NCH, STAGES = S::STAGES, TK = S::TILE_KEYS, THREADS = S::THREADS;
+  extern __shared__ __align__(128) unsigned char smem_tiles[];
+  uint32_t *sh_hist = reinterpret_cast<uint32_t *>(smem_tiles + STAGES * S::TILE_BYTES);
+  __shared__ uint64_t full_bar[STAGES];
+  __shared__ __align__(16) int4 sh_q[S::QREG ? 1 : TQ][S::QREG ? 1 : HI * NCH];
+
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int t = warp >> 1;          // this warp's query row within the sequence
+  const int half = warp & 1;        // and its half of every key tile
+  const bool row_live = t < T;
+  const int64_t gl = blockIdx.y;    // sequence within the pass
+  const int64_t rl0 = gl * T;       // its first row within the pass
+  const int64_t b = (row0 + rl0) / T;
+  const int G = gridDim.x, g = blockIdx.x;
+
+  int64_t V = N;   // the group's largest visible count (visibility grows with t)
+  int64_t Vt = N;  // this warp's row
+  if (n_prior >= 0) {
+    V = n_prior + (int64_t)T / ratio;
+    if (V > N) V = N;
+    Vt = n_prior + (int64_t)(t + 1) / ratio;
+    if (Vt > N) Vt = N;
+  }
+  const int64_t n0 = ((V * g) / G) & ~int64_t(15);
+  const int64_t n1 = (g == G - 1) ? V : (((V * (g + 1)) / G) & ~int64_t(15));
+  const int ntiles = (int)((n1 - n0 + TK - 1) / TK);
+  const int8_t *src = k_idx + (b * N + n0) * DI;
+
+  pdl_allow_dependents();
+  for (int i = tid; i < TQ * kBins1; i += THREADS) sh_hist[i] = 0u;
+  if (tid == 0) {
+    for (int s = 0; s < STAGES; ++s) mbar_init(&full_bar[s], 1);
+    fence_barrier_init();
+  }
+  // this row's index query (registers, pre-permuted; or shared memory) and weights
+  const int x = chunk_xor<NCH>(lane);
+  const int64_t r = b * T + (row_live ? t : 0);
+  int4 qreg[S::QREG ? HI * NCH : 1];
+  const int4 *qrow = reinterpret_cast<const int4 *>(q_idx + r * HI * DI);
+  if constexpr (S::QREG) {
+#pragma unroll
+    for (int h = 0; h < HI; ++h)
+#pragma unroll
+      for (int c = 0; c < NCH; ++c) qreg[h * NCH + c] = qrow[h * NCH + (c ^ x)];
+  } else {
+    for (int i = tid; i < TQ * HI * NCH; i += THREADS) {
+      const int tt = i / (HI * NCH), j = i % (HI * NCH);
+      sh_q[tt][j] = (tt < T) ? reinterpret_cast<const int4 *>(q_idx + (b * T + tt) * HI * DI)[j]
+                             : make_int4(0, 0, 0, 0);
+    }
+  }
+  float wh[HI];
+#pragma unroll
+  for (int h = 0; h < HI; ++h) wh[h] = w[r * HI + h];
+  __syncthreads();
+  if (tid == 0) {
+    for (int s = 0; s < STAGES && s < ntiles; ++s) {
+      const int64_t keys = min64(TK, n1 - n0 - (int64_t)s * TK);
+      const uint32_t bytes = (uint32_t)(keys * DI);
+      mbar_arrive_expect_tx(&full_bar[s], bytes);
+      bulk_g2s(smem_tiles + s * S::TILE_BYTES, src + (int64_t)s * TK * DI, bytes, &full_bar[s]);
+    }
+  }
+
+  float *srow = scores + (rl0 + (row_live ? t : 0)) * score_stride;
+  uint32_t *hrow = sh_hist + (row_live ? t : 0) * kBins1;
+  int abort_it = -1;
+  for (int it = 0; it < ntiles; ++it) {
+    const int s = it % STAGES;
+    const bool ok = mbar_wait_bounded(&full_bar[s], (uint32_t)(it / STAGES) & 1u);
+    if (__syncthreads_or(!ok)) {
+      abort_it = it;
+      break;
+    }
+    if (tid == 0 && it >= 1 && it - 1 + STAGES < ntiles) {
+      const int nt = it - 1 + STAGES, ps = (it - 1) % STAGES;
+      const int64_t keys = min64(TK, n1 - n0 - (int64_t)nt * TK);
+      const uint32_t bytes = (uint32_t)(keys * DI);
+      asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+      mbar_arrive_expect_tx(&full_bar[ps], bytes);
+      bulk_g2s(smem_tiles + ps * S::TILE_BYTES, src + (int64_t)nt * TK * DI, bytes,
+               &full_bar[ps]);
+    }
+    if (!row_live) continue;  // warp-uniform; the warp still takes every barrier
+    const unsigned char *tile = smem_tiles + s * S::TILE_BYTES;
+    const int64_t tbase = n0 + (int64_t)it * TK;
+    const int tkeys = (int)min64(TK, n1 - tbase);
+#pragma unroll
+    for (int j = 0; j < S::KPL; ++j) {
+      const int kl = half * (TK / 2) + j * 32 + lane;
+      const int64_t n = tbase + kl;
+      const bool vis = kl < tkeys && n < Vt;
+      float score = 0.0f;
+      if (vis) {
+        const unsigned char *krow = tile + kl * DI;
+        int dot[HI];
+#pragma unroll
+        for (int h = 0; h < HI; ++h) dot[h] = 0;
+#pragma unroll
+        for (int c = 0; c < NCH; ++c) {
+          const int4 kv = *reinterpret_cast<const int4 *>(krow + ((c ^ x) << 4));
+#pragma unroll
+          for (int h = 0; h < HI; ++h) {
+            int4 qv;
+            if constexpr (S::QREG)
+              qv = qreg[h * NCH + c];
+            else
+              qv = sh_q[t][h * NCH + (c ^ x)];
+            dot[h] = __dp4a(kv.x, qv.x, dot[h]);
+            dot[h] = __dp4a(kv.y, qv.y, dot[h]);
+            dot[h] = __dp4a(kv.z, qv.z, dot[h]);
+            dot[h] = __dp4a(kv.w, qv.w, dot[h]);
+          }
+        }
+        float acc = 0.0f;
+#pragma unroll
+        for (int h = 0; h < HI; ++h) acc = __fadd_rn(acc, __fmul_rn(wh[h], __int2float_rn(dot[h])));
+        score = __fadd_rn(acc, 0.0f);
+        srow[n] = score;
+        // plain shared-memory reduction: with a few rows per key the
+        // warp-aggregation of the single-row scan (match) would bound the
+        // kernel on its narrow issue pipe
+        atomicAdd(&hrow[key_d1(score_key(score))], 1u);
+      }
+    }
+  }
+  if (abort_it >= 0) {
+    if (tid == 0) {
+      const int upto = min(ntiles, max(abort_it - 1, 0) + STAGES);
+      for (int k = 0; k < STAGES && k < upto; ++k) {
+        const int last = k + ((upto - 1 - k) / STAGES) * STAGES;
+        mbar_wait_bounded(&full_bar[k], (uint32_t)(last / STAGES) & 1u);
+      }
+    }
+    __syncthreads();
+    return;
+  }
+  // entries a row may not see: -inf when scores are requested
+  if (write_masked && row_live && Vt < N) {
+    const int64_t m0 = Vt + ((N - Vt) * g) / G, m1 = Vt + ((N - Vt) * (g + 1)) / G;
+    for (int64_t n = m0 + half * 32 + lane; n < m1; n += 64) srow[n] = -__int_as_float(0x7f800000);
+  }
+  __syncthreads();
+  for (int tt = 0; tt < T && tt < TQ; ++tt) {
+    uint32_t *grow = hist1 + (rl0 + tt) * kHistStride;
+    for (int i = tid; i < kBins1; i += THREADS) {
+      const uint32_t v = sh_hist[tt * kBins1 + i];
+      if (v) atomicAdd(grow + i, v);
+    }
   }
 }
 

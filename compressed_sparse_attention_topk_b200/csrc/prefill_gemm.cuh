@@ -677,7 +677,7 @@ __global__ void __launch_bounds__(kThetaThreads) pf_theta_kernel(const ThetaPara
 // the row to the fallback.  One CTA of kSelThreads per row.
 // ---------------------------------------------------------------------------
 template <int DI, int HI>
-__global__ void __launch_bounds__(kSelThreads) pf_select_kernel(const SelParams p) {
+__global__ void __launch_bounds__(kSelThreads, 2) pf_select_kernel(const SelParams p) {
   extern __shared__ __align__(16) unsigned char sel_smem_raw[];
   SelSmem<DI, HI> &sm = *reinterpret_cast<SelSmem<DI, HI> *>(sel_smem_raw);
   uint32_t *cidx = reinterpret_cast<uint32_t *>(sel_smem_raw + sel_head_bytes<DI, HI>());
@@ -699,7 +699,7 @@ __global__ void __launch_bounds__(kSelThreads) pf_select_kernel(const SelParams 
   // candidates in ascending entry order: thread u owns a contiguous,
   // 16-byte aligned range of mask words; the first kWordsCached of them stay
   // in registers between the count and the extraction
-  constexpr int kWordsCached = 32;
+  constexpr int kWordsCached = 16;
   const uint32_t *brow = p.bits + (int64_t)lt * p.bits_pitch;
   const int64_t nw = (V + 31) / 32;
   const int64_t wpt = ((nw + kSelThreads - 1) / kSelThreads + 3) & ~int64_t(3);
@@ -755,20 +755,20 @@ __global__ void __launch_bounds__(kSelThreads) pf_select_kernel(const SelParams 
   __syncthreads();
   bool fail = overflow;
   if (!fail) {
-    // exact scores, four candidates per thread in flight; count those
+    // exact scores, two candidates per thread in flight; count those
     // certified above every entry left out
     const double U = ((double)p.tau[lt] - 1.0) / p.sigma[lt] + p.err[lt];
     const int8_t *kseq = p.k_idx + (int64_t)p.b * p.N * DI;
     uint32_t above = 0;
-    for (uint32_t i0 = tid; i0 < C; i0 += 4 * kSelThreads) {
-      float s[4];
+    for (uint32_t i0 = tid; i0 < C; i0 += 2 * kSelThreads) {
+      float s[2];
 #pragma unroll
-      for (int u = 0; u < 4; ++u) {
+      for (int u = 0; u < 2; ++u) {
         const uint32_t i = i0 + u * kSelThreads;
         s[u] = i < C ? exact_score<DI, HI>(kseq + (int64_t)cidx[i] * DI, sm.q, sm.w) : 0.0f;
       }
 #pragma unroll
-      for (int u = 0; u < 4; ++u) {
+      for (int u = 0; u < 2; ++u) {
         const uint32_t i = i0 + u * kSelThreads;
         if (i < C) {
           ckey[i] = score_key(s[u]);

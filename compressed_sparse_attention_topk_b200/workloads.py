@@ -81,7 +81,12 @@ PREFILL = Workload("prefill_t4096_nprior262144", B=1, T=4096, H=16, D=128, N=262
                    H_I=4, d_I=64, topk=2048, W=128, seed=5, modes=((FULL, 0, 0),),
                    n_prior=262144, ratio=4)
 
-ALL = {w.name: w for w in (TINY, DECODE, GROUP, LONG, PREFILL)}
+# Multi-token decode: 5 query tokens per sequence (draft tokens verified
+# together) at the 1M-context shape; every token sees all N entries.
+MTP5 = Workload("mtp5_decode_1m_b4_n262144", B=4, T=5, H=16, D=128, N=262144, H_I=4, d_I=64,
+                topk=2048, W=128, seed=6, modes=((FULL, 0, 0), (REINDEX, 0, 1)))
+
+ALL = {w.name: w for w in (TINY, DECODE, GROUP, LONG, PREFILL, MTP5)}
 
 _TENSOR_IDS = {"entries": 1, "k_idx": 2, "q_idx": 3, "w": 4, "q": 5, "win_k": 6, "win_v": 7,
                "outliers": 8}

@@ -203,6 +203,32 @@ def test_prefill_tensor_core_misleading_sample(where):
     _check_index(q, w, k, topk, check_scores=False)
 
 
+# ---------------------------------------------------------------------------
+# Several query rows per sequence (2 <= T <= 8, d_I <= 64): one shared key
+# scan scores every row of the sequence.
+# ---------------------------------------------------------------------------
+
+@pytest.mark.parametrize("T", [2, 3, 5, 8])
+@pytest.mark.parametrize("d_I,H_I", [(32, 4), (64, 4), (64, 1), (16, 8)])
+def test_multi_query_shared_scan(T, d_I, H_I):
+    q, w, k = _index_case(3, T, H_I, d_I, 9001, seed=100 * T + d_I + H_I)
+    _check_index(q, w, k, 300)                     # scores bit-exact too
+    _check_index(q, w, k, 300, check_scores=False)
+
+
+def test_multi_query_shared_scan_visibility():
+    B, T, n_prior, ratio = 2, 7, 5000, 2         # each row sees a different prefix
+    N = n_prior + T // ratio
+    q, w, k = _index_case(B, T, 4, 64, N, seed=77)
+    _check_index(q, w, k, 1024, n_prior=n_prior, ratio=ratio)
+
+
+def test_multi_token_decode_workload_full_size():
+    """5 query tokens per sequence at the 1M-context shape (B=4, N=262,144,
+    Full + Reindex): shared scans, per-row top-k, attention; every row."""
+    _run_group_and_compare(wl.MTP5)
+
+
 @pytest.mark.parametrize("wl_name", ["tiny_decode_n1024", "decode_b32_n131072"])
 def test_index_topk_workload(wl_name):
     w0 = wl.ALL[wl_name]
