@@ -74,6 +74,29 @@ def measured_peaks():
     return FALLBACK_HBM_GBS, "fallback"
 
 
+def dist_env():
+    """(world size, rank, local rank) of a torchrun launch; (1, 0, 0) alone."""
+    return (int(os.environ.get("WORLD_SIZE", "1")), int(os.environ.get("RANK", "0")),
+            int(os.environ.get("LOCAL_RANK", "0")))
+
+
+def max_over_ranks(dist, values, device):
+    """Element-wise maximum over all ranks of per-rank device times (ms).
+    Every rank calls it with the same number of values, in the same order."""
+    if dist is None:
+        return [float(v) for v in values]
+    import torch
+    t = torch.tensor([float(v) for v in values], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return [float(x) for x in t.tolist()]
+
+
+def job_tokens_per_s(world, steps, B, T, L, total_ms):
+    """Whole-job throughput: the tokens x layers of every rank (independent
+    replicas) over the slowest rank's device time."""
+    return world * steps * B * T * L / (total_ms * 1e-3)
+
+
 def pack_into_one_buffer(layers, keys, dev):
     """Move layers[l][k] (k in keys) into one uint8 device buffer, each tensor
     at a 256-byte aligned offset, and replace them by views of it (same dtype
@@ -191,7 +214,7 @@ def oracle_sample(w0, seconds: float, min_runs: int = 1):
 
 
 def run_reference(args, w0):
-    rank = int(os.environ.get("RANK", "0"))
+    _, rank, _ = dist_env()
     if rank != 0:
         return 0
     import oracle
@@ -236,9 +259,7 @@ def run_gpu(args, w0):
     import torch
     import compressed_sparse_attention_topk_b200 as csa2
 
-    world = int(os.environ.get("WORLD_SIZE", "1"))
-    rank = int(os.environ.get("RANK", "0"))
-    local = int(os.environ.get("LOCAL_RANK", "0"))
+    world, rank, local = dist_env()
     dist = None
     if world > 1:
         import datetime
@@ -366,11 +387,8 @@ def run_gpu(args, w0):
     step_ms = timed_steps(args.steps)
     torch.cuda.synchronize()
     wall_s = time.perf_counter() - w_t0
-    total_ms = float(sum(step_ms))
+    total_ms = max_over_ranks(dist, [float(sum(step_ms))], dev)[0]
     if dist:
-        t = torch.tensor([total_ms], dtype=torch.float64, device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        total_ms = float(t.item())
         dist.barrier()
 
     # ---- per-kernel device times (trace on; second timed pass) ----
@@ -415,20 +433,15 @@ def run_gpu(args, w0):
         return [sum(a.elapsed_time(b) for a, b in s) for s in res]
 
     e2e_steps(3)
-    e2e_ms = float(sum(e2e_steps(args.steps)))
-    if dist:
-        t = torch.tensor([e2e_ms], dtype=torch.float64, device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        e2e_ms = float(t.item())
+    e2e_ms = max_over_ranks(dist, [float(sum(e2e_steps(args.steps)))], dev)[0]
     clk = clocks.stop()
 
     status = csa2.get_device_status()
     if status:
         raise RuntimeError(f"device status word set: {status}")
 
-    tokens_layers = world * args.steps * w0.B * w0.T * w0.L
-    value = tokens_layers / (total_ms * 1e-3)
-    e2e_value = tokens_layers / (e2e_ms * 1e-3)
+    value = job_tokens_per_s(world, args.steps, w0.B, w0.T, w0.L, total_ms)
+    e2e_value = job_tokens_per_s(world, args.steps, w0.B, w0.T, w0.L, e2e_ms)
 
     ab = algorithmic_bytes(w0)
     peak, peak_kind = measured_peaks()
