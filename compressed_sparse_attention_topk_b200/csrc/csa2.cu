@@ -56,6 +56,17 @@ void trace_clear() {
   g_trace_n = 0;
 }
 
+// Records an event on `st`; while `st` is being captured into a CUDA graph
+// the record becomes an event-record node of the graph (timed on every
+// replay) instead of a capture-internal dependency.
+inline void trace_record(cudaEvent_t ev, cudaStream_t st) {
+  cudaStreamCaptureStatus cs = cudaStreamCaptureStatusNone;
+  if (cudaStreamIsCapturing(st, &cs) == cudaSuccess && cs == cudaStreamCaptureStatusActive)
+    cudaEventRecordWithFlags(ev, st, cudaEventRecordExternal);
+  else
+    cudaEventRecord(ev, st);
+}
+
 // Brackets one launch: records `start` on construction and `stop` on
 // destruction when the trace is on and has room.
 struct TraceScope {
@@ -73,10 +84,10 @@ struct TraceScope {
     r.name = name;
     rec = &r;
     ++g_trace_n;
-    cudaEventRecord(r.start, st);
+    trace_record(r.start, st);
   }
   ~TraceScope() {
-    if (rec) cudaEventRecord(rec->stop, st);
+    if (rec) trace_record(rec->stop, st);
   }
 };
 
@@ -1056,8 +1067,11 @@ int32_t csa2_trace_count(void) { return (int32_t)g_trace_n; }
 csa2_status csa2_trace_get(int32_t i, const char **name, float *ms) {
   if (i < 0 || (size_t)i >= g_trace_n || !name || !ms) return CSA2_ERR_INVALID_ARG;
   const TraceRecord &r = g_trace[i];
-  if (cudaEventSynchronize(r.stop) != cudaSuccess) return CSA2_ERR_CUDA;
-  if (cudaEventElapsedTime(ms, r.start, r.stop) != cudaSuccess) return CSA2_ERR_CUDA;
+  if (cudaEventSynchronize(r.stop) != cudaSuccess ||
+      cudaEventElapsedTime(ms, r.start, r.stop) != cudaSuccess) {
+    cudaGetLastError();  // a failed query must not be reported by the next launch
+    return CSA2_ERR_CUDA;
+  }
   *name = r.name;
   return CSA2_OK;
 }
