@@ -105,10 +105,10 @@ struct RowSmem {
     } tk;
     ar::WarpArea<D> aw[kAttnWarps];  // attention: per-warp chunk buffers, then partial states
   } u;
-  uint32_t h1[kBins1];          // staged digit-1 histogram
-  uint32_t h2[kBins2];          // own digit-2 (then digit-3) histogram
-  uint32_t hin[kBins2];         // bin slice this CTA owns, one row per source rank (pushed)
-  uint32_t full[kBins2];        // cluster-wide histogram (reduced slices pushed by owners)
+  alignas(16) uint32_t h1[kBins1];    // staged digit-1 histogram
+  alignas(16) uint32_t h2[kBins2];    // own digit-2 (then digit-3) histogram
+  alignas(16) uint32_t hin[kBins2];   // bin slice this CTA owns, one row per source rank (pushed)
+  alignas(16) uint32_t full[kBins2];  // cluster-wide histogram (reduced slices pushed by owners)
   uint32_t cnt_all[32][2];      // every rank's (above, tie) counts (pushed)
   int32_t sel[kSelCap];         // this CTA's selected indices, ascending
   uint16_t qb[kHeads][D + 8];   // query of the head pass, bf16
@@ -142,28 +142,39 @@ __device__ __forceinline__ uint32_t cand_class(uint32_t k, uint32_t t1, uint32_t
 
 // Cluster-wide histogram of NB bins (each CTA's own counts in sm.h2) ->
 // the largest bin t whose cluster-wide suffix count reaches `need`, the
-// count strictly above it and the count of bin t, in out[0..2].  Push-based:
-// every CTA stores bin slice j of its histogram into CTA j's `hin`; after a
-// barrier CTA j reduces its slice and stores it into every CTA's `full`;
-// after a second barrier each CTA finds the threshold locally.  Callers make
-// sure no CTA still reads its `hin` or `full` from an earlier use.
+// count strictly above it and the count of bin t, in out[0..2].  Push-based,
+// in 16-byte pieces of 4 bins: every CTA stores bin slice j of its histogram
+// into CTA j's `hin`; after a barrier CTA j reduces its slice (thread u sums
+// 4 bins over the CL sources and stores them into the `full` of CTA u / G4)
+// ; after a second barrier each CTA finds the threshold locally.  Callers
+// make sure no CTA still reads its `hin` or `full` from an earlier use.
 template <int D, int CL, int NB>
 __device__ void cluster_threshold(RowSmem<D> &sm, cg::cluster_group &cluster, uint32_t need,
                                   uint32_t *out) {
   constexpr int BPC = NB / CL;  // bins owned by each CTA
+  constexpr int G4 = BPC / 4;   // 4-bin pieces owned by each CTA
+  static_assert(BPC % 4 == 0, "16-byte pieces");
   const int tid = threadIdx.x;
   const int c = (int)cluster.block_rank();
-  for (int i = tid; i < NB; i += kRowThreads) {
-    const int owner = i / BPC;
-    cluster.map_shared_rank(&sm.hin[0], owner)[c * BPC + (i - owner * BPC)] = sm.h2[i];
+  for (int q = tid; q < NB / 4; q += kRowThreads) {
+    const int i = 4 * q, owner = i / BPC;
+    const uint4 v = *reinterpret_cast<const uint4 *>(&sm.h2[i]);
+    *reinterpret_cast<uint4 *>(cluster.map_shared_rank(&sm.hin[0], owner) + c * BPC +
+                               (i - owner * BPC)) = v;
   }
   cluster.sync();
-  for (int b = tid; b < BPC; b += kRowThreads) {
-    uint32_t s = 0;
+  for (int u = tid; u < G4 * CL; u += kRowThreads) {
+    const int g = u % G4, j = u / G4;
+    uint4 s = make_uint4(0u, 0u, 0u, 0u);
 #pragma unroll
-    for (int j = 0; j < CL; ++j) s += sm.hin[j * BPC + b];
-#pragma unroll
-    for (int j = 0; j < CL; ++j) cluster.map_shared_rank(&sm.full[0], j)[c * BPC + b] = s;
+    for (int src = 0; src < CL; ++src) {
+      const uint4 v = *reinterpret_cast<const uint4 *>(&sm.hin[src * BPC + 4 * g]);
+      s.x += v.x;
+      s.y += v.y;
+      s.z += v.z;
+      s.w += v.w;
+    }
+    *reinterpret_cast<uint4 *>(cluster.map_shared_rank(&sm.full[0], j) + c * BPC + 4 * g) = s;
   }
   cluster.sync();
   radix_threshold<kRowThreads, NB>(sm.full, need, sm.scratch, out);
@@ -198,6 +209,12 @@ __device__ void row_topk(RowSmem<D> &sm, const RowParams &p, cg::cluster_group &
   //    one block prefix over the counts, then each thread writes its
   //    candidates and histograms digit 2 of those exactly at t1.
   static_assert(kStageScores == 32 * kRowThreads, "one 32-bit mask per thread and round");
+  // digit 1 >= t1  <=>  key >= t1 << 21  <=>  score >= f1, the smallest
+  // score with that key (keys are monotone in the score; no -0 or NaN);
+  // for t1 <= 3 every key above the NaN patterns qualifies: f1 = -inf
+  const uint32_t k1 = t1 << 21;
+  const float f1 = (t1 <= 3u) ? -__int_as_float(0x7f800000)
+                              : __uint_as_float((k1 & 0x80000000u) ? (k1 & 0x7fffffffu) : ~k1);
   uint32_t count = 0;
   for (int64_t rb = s0; rb < s1; rb += kStageScores) {
     const int n = (int)min64(kStageScores, s1 - rb);
@@ -223,11 +240,11 @@ __device__ void row_topk(RowSmem<D> &sm, const RowParams &p, cg::cluster_group &
       const int qq = (q + tid) & 7;
       const int i = base + 4 * qq;
       const float4 v = *reinterpret_cast<const float4 *>(&sm.u.tk.sc[i]);
-      bits |= (uint32_t)((i + 0 < n) && key_d1(score_key(v.x)) >= t1) << (4 * qq + 0);
-      bits |= (uint32_t)((i + 1 < n) && key_d1(score_key(v.y)) >= t1) << (4 * qq + 1);
-      bits |= (uint32_t)((i + 2 < n) && key_d1(score_key(v.z)) >= t1) << (4 * qq + 2);
-      bits |= (uint32_t)((i + 3 < n) && key_d1(score_key(v.w)) >= t1) << (4 * qq + 3);
+      bits |= ((uint32_t)(v.x >= f1) | ((uint32_t)(v.y >= f1) << 1) |
+               ((uint32_t)(v.z >= f1) << 2) | ((uint32_t)(v.w >= f1) << 3))
+              << (4 * qq);
     }
+    if (n < kStageScores) bits &= (base >= n) ? 0u : (base + 32 <= n ? ~0u : (1u << (n - base)) - 1u);
     uint32_t total;
     uint32_t pos = count + block_excl_scan<kRowThreads>((uint32_t)__popc(bits), sm.scratch, total);
     while (bits) {
@@ -283,9 +300,18 @@ __device__ void row_topk(RowSmem<D> &sm, const RowParams &p, cg::cluster_group &
     n_above += (cls == 2u);
     n_tie += (cls == 1u);
   }
-  uint32_t tot_above, tot_tie;
-  const uint32_t above_before = block_excl_scan<kRowThreads>(n_above, sm.scratch, tot_above);
-  const uint32_t tie_before = block_excl_scan<kRowThreads>(n_tie, sm.scratch, tot_tie);
+  uint32_t tot_above, tot_tie, above_before, tie_before;
+  if (count < 65536u) {  // both counts in one prefix (16 bits each)
+    uint32_t tot;
+    const uint32_t pre = block_excl_scan<kRowThreads>(n_above | (n_tie << 16), sm.scratch, tot);
+    above_before = pre & 0xffffu;
+    tie_before = pre >> 16;
+    tot_above = tot & 0xffffu;
+    tot_tie = tot >> 16;
+  } else {
+    above_before = block_excl_scan<kRowThreads>(n_above, sm.scratch, tot_above);
+    tie_before = block_excl_scan<kRowThreads>(n_tie, sm.scratch, tot_tie);
+  }
   if (tid < CL) {  // push this CTA's counts to every rank
     uint32_t *dst = cluster.map_shared_rank(&sm.cnt_all[0][0], tid);
     dst[2 * c] = tot_above;

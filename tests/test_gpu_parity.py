@@ -120,6 +120,23 @@ def test_topk_heavy_ties_at_boundary(levels):
     _check_index(q, w, k, 1000)
 
 
+def test_topk_crowded_into_few_slices():
+    # The top-k sits in the last 3,000 entries (their head-0 dot product is
+    # |q_0|^2): the candidate lists of those slices stop above the row's
+    # threshold digit, so the selection has to work from the score rows.
+    q, w, k = _index_case(2, 1, 4, 64, 60000, seed=11)
+    for b in range(2):
+        k[b, -3000:, :] = q[b, 0, 0, :]
+    _check_index(q, w, k, 2048)
+
+
+@pytest.mark.parametrize("N", [4096, 70000, 262144])
+def test_topk_candidate_lists_many_slices(N):
+    # one row: the scan splits it into up to ~2 slices per SM, each emitting a list
+    q, w, k = _index_case(1, 1, 4, 64, N, seed=N)
+    _check_index(q, w, k, 2048)
+
+
 def test_topk_empty_store():
     q, w, k = _index_case(2, 1, 4, 64, 0, seed=1)
     idx = csa2.index_topk(dev(q), dev(w), torch.empty((2, 0, 64), dtype=torch.int8,
