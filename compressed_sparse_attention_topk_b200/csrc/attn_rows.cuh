@@ -44,7 +44,7 @@ struct Params {
 };
 
 template <int D>
-struct WarpArea {
+struct alignas(16) WarpArea {
   static constexpr int CB = D / 2;                  // code bytes per entry
   static constexpr int SB = D / 4;                  // scale bytes per entry
   static constexpr int PIECES = (CB + SB) / 16;     // 16-byte pieces per entry
@@ -56,7 +56,7 @@ struct WarpArea {
       uint16_t vt[kChunk][D + 8];                   // window values (bf16)
     } s;
     struct {
-      float o[kHeads][D];                           // partial output for the merge
+      alignas(16) float o[kHeads][D];               // partial output for the merge
       float m[kHeads], l[kHeads];
     } merge;
   };

@@ -68,7 +68,7 @@ constexpr int kStageScores = 16384;  // scores staged in shared memory per round
 constexpr int kCandCap = 2048;       // candidates kept in shared memory (more spill to global)
 constexpr int kSelCap = 4096;        // selected indices kept in shared memory
 constexpr int kHeads = 16;           // heads per pass (the MMA's M)
-constexpr int kAttnWarps = 7;        // warps that run attention chunks
+constexpr int kAttnWarps = 10;       // warps that run attention chunks
 
 struct RowParams {
   // top-k
@@ -112,8 +112,11 @@ struct RowSmem {
   uint32_t cnt_all[32][2];      // every rank's (above, tie) counts (pushed)
   int32_t sel[kSelCap];         // this CTA's selected indices, ascending
   uint16_t qb[kHeads][D + 8];   // query of the head pass, bf16
-  float inbox[kHeads][D + 2];   // pushed partials (m, l, acc) of the heads this CTA merges
+  // pushed partials of the heads this CTA merges: (m, l, -, -, acc[D])
+  alignas(16) float inbox[kHeads][D + 4];
   float mf[kHeads][kAttnWarps + 1];  // per head: each attention warp's factor, then the max
+  float fac[kHeads];            // final merge: factor of each inbox slot
+  float mrg_m[kHeads], mrg_l[kHeads];  // final merge: max and sum of each merged head
   uint32_t scratch[40];
   uint32_t thr[8];
   uint32_t cnt[4];  // [1] above-threshold, [2] equal-to-threshold, [3] reduced-slice total
@@ -450,53 +453,69 @@ __device__ void row_attend(RowSmem<D> &sm, const RowParams &p, cg::cluster_group
   }
   __syncthreads();
   // this CTA's partial of each head (max, sum, acc) -> inbox slot
-  // (h / CL) * CL + c of the owner CTA h % CL
-  for (int i = tid; i < nh * (D + 2); i += kRowThreads) {
-    const int h = i / (D + 2), e = i % (D + 2);
-    float v = 0.0f;
-    if (e == 0) {
-      v = sm.mf[h][kAttnWarps];
+  // (h / CL) * CL + c of the owner CTA h % CL, in 16-byte pieces: (m, l)
+  // first, then the accumulator
+  constexpr int U = D / 4 + 1;
+  for (int i = tid; i < nh * U; i += kRowThreads) {
+    const int h = i / U, q = i % U;
+    float4 v = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
+    if (q == 0) {
+#pragma unroll
+      for (int w = 0; w < kAttnWarps; ++w) v.y = fmaf(sm.u.aw[w].merge.l[h], sm.mf[h][w], v.y);
+      v.x = sm.mf[h][kAttnWarps];
     } else {
 #pragma unroll
-      for (int w = 0; w < kAttnWarps; ++w)
-        v = fmaf(e == 1 ? sm.u.aw[w].merge.l[h] : sm.u.aw[w].merge.o[h][e - 2], sm.mf[h][w], v);
+      for (int w = 0; w < kAttnWarps; ++w) {
+        const float4 o = *reinterpret_cast<const float4 *>(&sm.u.aw[w].merge.o[h][4 * (q - 1)]);
+        const float f = sm.mf[h][w];
+        v.x = fmaf(o.x, f, v.x);
+        v.y = fmaf(o.y, f, v.y);
+        v.z = fmaf(o.z, f, v.z);
+        v.w = fmaf(o.w, f, v.w);
+      }
     }
-    float *dst = cluster.map_shared_rank(&sm.inbox[0][0], h % CL) + ((h / CL) * CL + c) * (D + 2);
-    dst[e] = v;
+    float *dst = cluster.map_shared_rank(&sm.inbox[0][0], h % CL) +
+                 ((h / CL) * CL + c) * (D + 4) + 4 * q;
+    *reinterpret_cast<float4 *>(dst) = v;
   }
   cluster.sync();
-  // merge: warp k merges head h = c + k*CL from the CL partials in the inbox
-  constexpr int DL = D / 32;
-  const int h = c + warp * CL;
-  if (warp < kHeads / CL && h < nh) {
+  // merge of head h = c + k*CL (k < kHeads / CL) from its CL partials in
+  // slots [k*CL, k*CL + CL): warp k finds the max, the factors and the sum,
+  // then one thread per (head, dim) sums the weighted partials
+  constexpr int KH = kHeads / CL;
+  if (warp < KH) {
+    const int h = c + warp * CL;
     const float *slot = &sm.inbox[warp * CL][0];
-    const float m = (lane < CL) ? slot[lane * (D + 2)] : -INFINITY;
-    const float l = (lane < CL) ? slot[lane * (D + 2) + 1] : 0.0f;
+    const float m = (lane < CL) ? slot[lane * (D + 4)] : -INFINITY;
+    const float l = (lane < CL) ? slot[lane * (D + 4) + 1] : 0.0f;
     const float M = warp_max(l > 0.0f ? m : -INFINITY);
-    float *op = p.out + (r * p.H + h0 + h) * (int64_t)D;
-    if (M == -INFINITY) {
-#pragma unroll
-      for (int i = 0; i < DL; ++i) op[lane + 32 * i] = 0.0f;
-      if (p.lse && lane == 0) p.lse[r * p.H + h0 + h] = -INFINITY;
-    } else {
-      const float f = (l > 0.0f) ? exp2f(m - M) : 0.0f;
-      const float L = warp_sum(l * f);
-      float a[DL];
-#pragma unroll
-      for (int i = 0; i < DL; ++i) a[i] = 0.0f;
-#pragma unroll
-      for (int j = 0; j < CL; ++j) {
-        const float fj = __shfl_sync(0xffffffffu, f, j);
-        if (fj != 0.0f) {
-#pragma unroll
-          for (int i = 0; i < DL; ++i) a[i] = fmaf(slot[j * (D + 2) + 2 + lane + 32 * i], fj, a[i]);
-        }
-      }
-      const float inv = 1.0f / L;
-#pragma unroll
-      for (int i = 0; i < DL; ++i) op[lane + 32 * i] = a[i] * inv;
-      if (p.lse && lane == 0) p.lse[r * p.H + h0 + h] = (M + log2f(L)) * 0.69314718055994530942f;
+    const float f = (M != -INFINITY && l > 0.0f) ? exp2f(m - M) : 0.0f;
+    const float L = warp_sum(l * f);
+    if (lane < CL) sm.fac[warp * CL + lane] = f;
+    if (lane == 0) {
+      sm.mrg_m[warp] = M;
+      sm.mrg_l[warp] = L;
+      if (p.lse && h < nh)
+        p.lse[r * p.H + h0 + h] =
+            M == -INFINITY ? -INFINITY : (M + log2f(L)) * 0.69314718055994530942f;
     }
+  }
+  __syncthreads();
+  for (int i = tid; i < KH * D; i += kRowThreads) {
+    const int k = i / D, e = i % D, h = c + k * CL;
+    if (h >= nh) continue;
+    float *op = p.out + (r * p.H + h0 + h) * (int64_t)D;
+    if (sm.mrg_m[k] == -INFINITY) {
+      op[e] = 0.0f;
+      continue;
+    }
+    float a = 0.0f;
+#pragma unroll
+    for (int j = 0; j < CL; ++j) {
+      const float fj = sm.fac[k * CL + j];
+      if (fj != 0.0f) a = fmaf(sm.inbox[k * CL + j][4 + e], fj, a);
+    }
+    op[e] = a * (1.0f / sm.mrg_l[k]);
   }
 }
 
