@@ -86,6 +86,48 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t *bar, uint32_t parity) {
   return ok != 0;
 }
 
+// The same wait with cluster-scope acquire: data that other CTAs of the
+// cluster delivered with st.async (below) is visible once the phase is seen
+// complete.
+__device__ __forceinline__ bool mbar_try_wait_cluster(uint64_t *bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(smem_u32(bar)), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+
+// Shared-memory address of `p` (an address of this CTA's shared memory) in
+// CTA `rank` of the cluster.
+__device__ __forceinline__ uint32_t cluster_addr(const void *p, uint32_t rank) {
+  uint32_t a;
+  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(a) : "r"(smem_u32(p)), "r"(rank));
+  return a;
+}
+
+// Stores into the shared memory of CTA `rank` (at the offset of `dst` here)
+// whose bytes are counted on the mbarrier at the offset of `bar` in that
+// CTA (st.async with complete_tx): the receiver announces the bytes it
+// expects and waits for its own barrier, no cluster-wide barrier involved.
+__device__ __forceinline__ void st_async_v4(void *dst, uint4 v, uint64_t *bar, uint32_t rank) {
+  asm volatile(
+      "st.async.shared::cluster.mbarrier::complete_tx::bytes.v4.b32 [%0], {%1, %2, %3, %4}, [%5];"
+      ::"r"(cluster_addr(dst, rank)), "r"(v.x), "r"(v.y), "r"(v.z), "r"(v.w),
+        "r"(cluster_addr(bar, rank))
+      : "memory");
+}
+__device__ __forceinline__ void st_async_v2(void *dst, uint32_t a, uint32_t b, uint64_t *bar,
+                                            uint32_t rank) {
+  asm volatile(
+      "st.async.shared::cluster.mbarrier::complete_tx::bytes.v2.b32 [%0], {%1, %2}, [%3];"
+      ::"r"(cluster_addr(dst, rank)), "r"(a), "r"(b), "r"(cluster_addr(bar, rank))
+      : "memory");
+}
+
 // Wait for the given phase parity for at most ~2^32 cycles (about 2 s);
 // on timeout record it in the status word and return false.  The clock is
 // read only once the phase is found incomplete: a clock read costs as much
@@ -94,6 +136,18 @@ __device__ __forceinline__ bool mbar_wait_bounded(uint64_t *bar, uint32_t parity
   if (mbar_try_wait(bar, parity)) return true;
   const long long start = clock64();
   while (!mbar_try_wait(bar, parity)) {
+    if (clock64() - start > (1ll << 32)) {
+      raise_status(kStatusWaitTimeout);
+      return false;
+    }
+  }
+  return true;
+}
+
+__device__ __forceinline__ bool mbar_wait_cluster_bounded(uint64_t *bar, uint32_t parity) {
+  if (mbar_try_wait_cluster(bar, parity)) return true;
+  const long long start = clock64();
+  while (!mbar_try_wait_cluster(bar, parity)) {
     if (clock64() - start > (1ll << 32)) {
       raise_status(kStatusWaitTimeout);
       return false;

@@ -109,7 +109,7 @@ struct RowSmem {
   alignas(16) uint32_t h2[kBins2];    // own digit-2 (then digit-3) histogram
   alignas(16) uint32_t hin[kBins2];   // bin slice this CTA owns, one row per source rank (pushed)
   alignas(16) uint32_t full[kBins2];  // cluster-wide histogram (reduced slices pushed by owners)
-  uint32_t cnt_all[32][2];      // every rank's (above, tie) counts (pushed)
+  alignas(8) uint32_t cnt_all[32][2];      // every rank's (above, tie) counts (pushed)
   int32_t sel[kSelCap];         // this CTA's selected indices, ascending
   uint16_t qb[kHeads][D + 8];   // query of the head pass, bf16
   // pushed partials of the heads this CTA merges: (m, l, -, -, acc[D])
@@ -122,6 +122,9 @@ struct RowSmem {
   uint32_t cnt[4];  // [1] above-threshold, [2] equal-to-threshold, [3] reduced-slice total
   uint32_t sel_base, sel_count, out_base, tie_base;
   uint64_t bar;
+  // exchange barriers, one per delivery (bytes counted by st.async):
+  // digit-2 slices, digit-2 sums, digit-3 slices, digit-3 sums, counts, partials
+  uint64_t xbar[6];
 };
 
 __device__ __forceinline__ int64_t row_visible(int64_t N, int64_t n_prior, int32_t ratio,
@@ -146,26 +149,33 @@ __device__ __forceinline__ uint32_t cand_class(uint32_t k, uint32_t t1, uint32_t
 // Cluster-wide histogram of NB bins (each CTA's own counts in sm.h2) ->
 // the largest bin t whose cluster-wide suffix count reaches `need`, the
 // count strictly above it and the count of bin t, in out[0..2].  Push-based,
-// in 16-byte pieces of 4 bins: every CTA stores bin slice j of its histogram
-// into CTA j's `hin`; after a barrier CTA j reduces its slice (thread u sums
-// 4 bins over the CL sources and stores them into the `full` of CTA u / G4)
-// ; after a second barrier each CTA finds the threshold locally.  Callers
-// make sure no CTA still reads its `hin` or `full` from an earlier use.
+// in 16-byte pieces of 4 bins delivered by st.async: every CTA stores bin
+// slice j of its histogram into CTA j's `hin` (counted on bar_in); CTA j,
+// once its NB * 4 bytes are in, reduces its slice (thread u sums 4 bins over
+// the CL sources) and stores the sums into the `full` of every CTA (counted
+// on bar_full); each CTA finds the threshold once its own `full` is
+// complete.  No cluster-wide barrier: a CTA reduces only after every CTA has
+// delivered to it, i.e. after every CTA is done with the previous use of
+// `full`; callers make sure the same holds for `hin`.
 template <int D, int CL, int NB>
 __device__ void cluster_threshold(RowSmem<D> &sm, cg::cluster_group &cluster, uint32_t need,
-                                  uint32_t *out) {
+                                  uint32_t *out, uint64_t *bar_in, uint64_t *bar_full,
+                                  bool &abort) {
   constexpr int BPC = NB / CL;  // bins owned by each CTA
   constexpr int G4 = BPC / 4;   // 4-bin pieces owned by each CTA
   static_assert(BPC % 4 == 0, "16-byte pieces");
   const int tid = threadIdx.x;
   const int c = (int)cluster.block_rank();
+  if (tid == 0) {
+    mbar_arrive_expect_tx(bar_in, NB * 4);
+    mbar_arrive_expect_tx(bar_full, NB * 4);
+  }
   for (int q = tid; q < NB / 4; q += kRowThreads) {
     const int i = 4 * q, owner = i / BPC;
     const uint4 v = *reinterpret_cast<const uint4 *>(&sm.h2[i]);
-    *reinterpret_cast<uint4 *>(cluster.map_shared_rank(&sm.hin[0], owner) + c * BPC +
-                               (i - owner * BPC)) = v;
+    st_async_v4(&sm.hin[c * BPC + (i - owner * BPC)], v, bar_in, (uint32_t)owner);
   }
-  cluster.sync();
+  if (!mbar_wait_cluster_bounded(bar_in, 0)) abort = true;
   for (int u = tid; u < G4 * CL; u += kRowThreads) {
     const int g = u % G4, j = u / G4;
     uint4 s = make_uint4(0u, 0u, 0u, 0u);
@@ -177,9 +187,9 @@ __device__ void cluster_threshold(RowSmem<D> &sm, cg::cluster_group &cluster, ui
       s.z += v.z;
       s.w += v.w;
     }
-    *reinterpret_cast<uint4 *>(cluster.map_shared_rank(&sm.full[0], j) + c * BPC + 4 * g) = s;
+    st_async_v4(&sm.full[c * BPC + 4 * g], s, bar_full, (uint32_t)j);
   }
-  cluster.sync();
+  if (!mbar_wait_cluster_bounded(bar_full, 0)) abort = true;
   radix_threshold<kRowThreads, NB>(sm.full, need, sm.scratch, out);
   if (tid == 0) out[2] = sm.full[out[0]];
   __syncthreads();
@@ -270,7 +280,7 @@ __device__ void row_topk(RowSmem<D> &sm, const RowParams &p, cg::cluster_group &
   };
 
   // 2. digit-2 threshold from the cluster's histograms
-  cluster_threshold<D, CL, kBins2>(sm, cluster, r1, sm.thr + 2);
+  cluster_threshold<D, CL, kBins2>(sm, cluster, r1, sm.thr + 2, &sm.xbar[0], &sm.xbar[1], abort);
   const uint32_t t2 = sm.thr[2], r2 = r1 - sm.thr[3];
   const bool need3 = sm.thr[4] > r2;
 
@@ -284,7 +294,7 @@ __device__ void row_topk(RowSmem<D> &sm, const RowParams &p, cg::cluster_group &
       if (key_d1(k) == t1 && key_d2(k) == t2) atomicAdd(&sm.h2[key_d3(k)], 1u);
     }
     __syncthreads();
-    cluster_threshold<D, CL, kBins3>(sm, cluster, r2, sm.thr + 2);
+    cluster_threshold<D, CL, kBins3>(sm, cluster, r2, sm.thr + 2, &sm.xbar[2], &sm.xbar[3], abort);
     t3 = sm.thr[2];
     r3 = r2 - sm.thr[3];
   }
@@ -315,12 +325,10 @@ __device__ void row_topk(RowSmem<D> &sm, const RowParams &p, cg::cluster_group &
     above_before = block_excl_scan<kRowThreads>(n_above, sm.scratch, tot_above);
     tie_before = block_excl_scan<kRowThreads>(n_tie, sm.scratch, tot_tie);
   }
-  if (tid < CL) {  // push this CTA's counts to every rank
-    uint32_t *dst = cluster.map_shared_rank(&sm.cnt_all[0][0], tid);
-    dst[2 * c] = tot_above;
-    dst[2 * c + 1] = tot_tie;
-  }
-  cluster.sync();  // every rank's (above, tie) counts are in cnt_all
+  // this CTA's counts to every rank; wait for every rank's
+  if (tid == 0) mbar_arrive_expect_tx(&sm.xbar[4], CL * 8);
+  if (tid < CL) st_async_v2(&sm.cnt_all[c][0], tot_above, tot_tie, &sm.xbar[4], (uint32_t)tid);
+  if (!mbar_wait_cluster_bounded(&sm.xbar[4], 0)) abort = true;
   if (warp == 0) {
     const uint32_t above = (lane < CL) ? sm.cnt_all[lane][0] : 0u;
     const uint32_t ties = (lane < CL) ? sm.cnt_all[lane][1] : 0u;
@@ -454,8 +462,13 @@ __device__ void row_attend(RowSmem<D> &sm, const RowParams &p, cg::cluster_group
   __syncthreads();
   // this CTA's partial of each head (max, sum, acc) -> inbox slot
   // (h / CL) * CL + c of the owner CTA h % CL, in 16-byte pieces: (m, l)
-  // first, then the accumulator
+  // first, then the accumulator, delivered by st.async and counted on the
+  // owner's partials barrier (the owner expects CL pieces per head it merges)
   constexpr int U = D / 4 + 1;
+  if (tid == 0) {
+    const int owned = nh > c ? (nh - 1 - c) / CL + 1 : 0;
+    mbar_arrive_expect_tx(&sm.xbar[5], (uint32_t)(owned * CL * (D + 4) * 4));
+  }
   for (int i = tid; i < nh * U; i += kRowThreads) {
     const int h = i / U, q = i % U;
     float4 v = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
@@ -474,11 +487,14 @@ __device__ void row_attend(RowSmem<D> &sm, const RowParams &p, cg::cluster_group
         v.w = fmaf(o.w, f, v.w);
       }
     }
-    float *dst = cluster.map_shared_rank(&sm.inbox[0][0], h % CL) +
-                 ((h / CL) * CL + c) * (D + 4) + 4 * q;
-    *reinterpret_cast<float4 *>(dst) = v;
+    st_async_v4(&sm.inbox[(h / CL) * CL + c][4 * q],
+                make_uint4(__float_as_uint(v.x), __float_as_uint(v.y), __float_as_uint(v.z),
+                           __float_as_uint(v.w)),
+                &sm.xbar[5], (uint32_t)(h % CL));
   }
-  cluster.sync();
+  // the partials of the heads this CTA merges (CL sources each); a wait
+  // that gives up is recorded in the status word
+  mbar_wait_cluster_bounded(&sm.xbar[5], (uint32_t)(h0 / kHeads) & 1u);
   // merge of head h = c + k*CL (k < kHeads / CL) from its CL partials in
   // slots [k*CL, k*CL + CL): warp k finds the max, the factors and the sum,
   // then one thread per (head, dim) sums the weighted partials
@@ -536,14 +552,16 @@ __global__ void __launch_bounds__(kRowThreads, 1) row_cluster_kernel(const RowPa
   const int64_t s1 = (c == CL - 1) ? V : (((V * (c + 1)) / CL) & ~int64_t(15));
   const bool topk_here = p.do_topk && K > 0;
 
-  // Every CTA of the cluster must be running before any of them writes into
-  // another's shared memory: arrive now, wait before the first such write.
-  asm volatile("barrier.cluster.arrive.relaxed.aligned;" ::: "memory");
+  // Every CTA of the cluster must be running, with its barriers initialised,
+  // before any of them writes into another's shared memory: arrive once the
+  // barriers are set up, wait before the first such write.
   if (tid == 0) {
     mbar_init(&sm.bar, 1);
+    for (int k = 0; k < 6; ++k) mbar_init(&sm.xbar[k], 1);
     fence_barrier_init();
   }
   __syncthreads();
+  asm volatile("barrier.cluster.arrive.relaxed.aligned;" ::: "memory");
   // Prologue, independent of the scan that produced the scores: the query.
   // With programmatic dependent launch this overlaps the scan's tail.
   for (int i = tid; i < kBins2; i += kRowThreads) sm.h2[i] = 0u;
