@@ -86,14 +86,28 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t *bar, uint32_t parity) {
   return ok != 0;
 }
 
-// The same wait with cluster-scope acquire: data that other CTAs of the
+// Non-blocking tests of a phase: a thread that polls with test_wait is never
+// suspended, so it sees the phase complete as soon as it does (a try_wait
+// that suspends the thread can resume it well after completion).  The
+// cluster form acquires at cluster scope: data that other CTAs of the
 // cluster delivered with st.async (below) is visible once the phase is seen
 // complete.
-__device__ __forceinline__ bool mbar_try_wait_cluster(uint64_t *bar, uint32_t parity) {
+__device__ __forceinline__ bool mbar_test_wait(uint64_t *bar, uint32_t parity) {
   uint32_t ok;
   asm volatile(
       "{\n\t.reg .pred p;\n\t"
-      "mbarrier.try_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2;\n\t"
+      "mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(smem_u32(bar)), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+__device__ __forceinline__ bool mbar_test_wait_cluster(uint64_t *bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.test_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2;\n\t"
       "selp.u32 %0, 1, 0, p;\n\t}"
       : "=r"(ok)
       : "r"(smem_u32(bar)), "r"(parity)
@@ -128,14 +142,14 @@ __device__ __forceinline__ void st_async_v2(void *dst, uint32_t a, uint32_t b, u
       : "memory");
 }
 
-// Wait for the given phase parity for at most ~2^32 cycles (about 2 s);
-// on timeout record it in the status word and return false.  The clock is
-// read only once the phase is found incomplete: a clock read costs as much
-// as ~150 cycles on the waiting thread's path.
+// Wait for the given phase parity for at most ~2^32 cycles (about 2 s),
+// polling without suspension; on timeout record it in the status word and
+// return false.  The clock is read only once the phase is found incomplete:
+// a clock read costs as much as ~150 cycles on the waiting thread's path.
 __device__ __forceinline__ bool mbar_wait_bounded(uint64_t *bar, uint32_t parity) {
-  if (mbar_try_wait(bar, parity)) return true;
+  if (mbar_test_wait(bar, parity)) return true;
   const long long start = clock64();
-  while (!mbar_try_wait(bar, parity)) {
+  while (!mbar_test_wait(bar, parity)) {
     if (clock64() - start > (1ll << 32)) {
       raise_status(kStatusWaitTimeout);
       return false;
@@ -144,10 +158,13 @@ __device__ __forceinline__ bool mbar_wait_bounded(uint64_t *bar, uint32_t parity
   return true;
 }
 
+// Wait for a barrier that other CTAs of the cluster complete with st.async
+// (below), with cluster-scope acquire: the bytes they stored into this CTA's
+// shared memory are visible once the phase is seen complete.
 __device__ __forceinline__ bool mbar_wait_cluster_bounded(uint64_t *bar, uint32_t parity) {
-  if (mbar_try_wait_cluster(bar, parity)) return true;
+  if (mbar_test_wait_cluster(bar, parity)) return true;
   const long long start = clock64();
-  while (!mbar_try_wait_cluster(bar, parity)) {
+  while (!mbar_test_wait_cluster(bar, parity)) {
     if (clock64() - start > (1ll << 32)) {
       raise_status(kStatusWaitTimeout);
       return false;
