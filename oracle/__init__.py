@@ -67,8 +67,11 @@ def _load():
                                         P, i64, P, P]
         lib.orc_validate_modes.argtypes = [P, i32]
         lib.orc_group_cache_bytes.argtypes = [P, i32, i64, i64, i64, P]
+        lib.orc_block_pool.argtypes = [P, i64, i32, i32, P, P]
+        lib.orc_pool_topk.argtypes = [P, P, P, i32, i32, i64, P, i64, i32, P]
         for name in ("orc_pack_fp4", "orc_unpack_fp4", "orc_topk_row", "orc_index_topk",
-                     "orc_sparse_attn", "orc_validate_modes", "orc_group_cache_bytes"):
+                     "orc_sparse_attn", "orc_validate_modes", "orc_group_cache_bytes",
+                     "orc_block_pool", "orc_pool_topk"):
             getattr(lib, name).restype = ctypes.c_int
         _lib = lib
     return _lib
@@ -161,6 +164,32 @@ def index_topk(q_idx, w, k_idx, topk, n_prior=-1, ratio=4, rows=None, want_score
                                   ratio, topk, _ptr(rows_arr), nrows, _ptr(idx), _ptr(scores)),
            "index_topk")
     return (idx, scores) if want_scores else idx
+
+
+# --- hierarchical indexer (candidate pool of a Full layer) ---------------------
+
+def block_pool(scores: np.ndarray, block: int, n_blocks: int) -> np.ndarray:
+    """A Full layer's visible scores fp32 [V] -> the pool's positions int32,
+    ascending: every visible position of the n_blocks best blocks of `block`
+    consecutive positions (block score = its largest score; ties to the
+    lower block)."""
+    scores = _c(scores, np.float32)
+    out = np.empty(block * n_blocks, np.int32)
+    n = np.zeros(1, np.int64)
+    _check(_load().orc_block_pool(_ptr(scores), scores.shape[0], block, n_blocks, _ptr(out),
+                                  _ptr(n)), "block_pool")
+    return out[: int(n[0])].copy()
+
+
+def pool_topk(q: np.ndarray, w: np.ndarray, keys: np.ndarray, pool: np.ndarray, k: int) -> np.ndarray:
+    """One query row (q int8 [H_I, d_I], w fp32 [H_I]) over the pool's
+    positions of keys int8 [N, d_I]: top-k positions, ascending, -1 padded."""
+    q, w, keys, pool = _c(q, np.int8), _c(w, np.float32), _c(keys, np.int8), _c(pool, np.int32)
+    H_I, d_I = q.shape
+    out = np.empty(k, np.int32)
+    _check(_load().orc_pool_topk(_ptr(q), _ptr(w), _ptr(keys), H_I, d_I, keys.shape[0],
+                                 _ptr(pool), pool.shape[0], k, _ptr(out)), "pool_topk")
+    return out
 
 
 # --- attention --------------------------------------------------------------

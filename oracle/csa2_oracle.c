@@ -446,3 +446,107 @@ int orc_group_cache_bytes(const int32_t *modes, int32_t L, int64_t entries,
     *bytes_out = bits / 8u;
     return ORC_OK;
 }
+
+/* ------------------------------------------------------------------------ */
+/* Hierarchical sparse indexing.  [P3] section 5 ("Hierarchical Sparse      */
+/* Indexing"): an earlier Full layer searches broadly and keeps a candidate */
+/* pool -- the example keeps 2,048 blocks of eight positions, 16,384        */
+/* candidates -- and later Reindex layers search only within that pool.    */
+/* Readings (the pages give no formula):                                    */
+/*  - a block is `block` consecutive compressed positions, block j covering */
+/*    [j*block, (j+1)*block); the last block holds only visible positions;  */
+/*  - a block's score is the largest of the Full layer's index scores over  */
+/*    its visible positions; blocks are ranked by that score, ties to the   */
+/*    lower block index, and the best n_blocks are kept (all of them when   */
+/*    fewer are visible);                                                   */
+/*  - the pool lists the kept blocks' positions in ascending order;         */
+/*  - a Reindex layer scores only the pool's positions with its own index   */
+/*    query (same score as above) and keeps their top-k with the same tie   */
+/*    rule, ascending output and -1 padding.                                */
+/* ------------------------------------------------------------------------ */
+
+typedef struct {
+    float score;
+    int64_t j;
+} orc_block;
+
+static int orc_block_cmp(const void *pa, const void *pb)
+{
+    const orc_block *a = (const orc_block *)pa, *b = (const orc_block *)pb;
+    if (a->score > b->score)
+        return -1;
+    if (a->score < b->score)
+        return 1;
+    return (a->j < b->j) ? -1 : (a->j > b->j) ? 1 : 0;
+}
+
+/* scores[0..V): a Full layer's visible index scores.  Writes the pool to
+ * pool_out[0..n_blocks*block) (-1 after its *pool_len entries). */
+int orc_block_pool(const float *scores, int64_t V, int32_t block, int32_t n_blocks,
+                   int32_t *pool_out, int64_t *pool_len)
+{
+    if (!pool_out || !pool_len || V < 0 || block <= 0 || n_blocks <= 0 || (V > 0 && !scores))
+        return ORC_EINVAL;
+    const int64_t nb = (V + block - 1) / block;
+    orc_block *b = (orc_block *)malloc((size_t)(nb > 0 ? nb : 1) * sizeof(orc_block));
+    unsigned char *kept = (unsigned char *)calloc((size_t)(nb > 0 ? nb : 1), 1);
+    if (!b || !kept) {
+        free(b);
+        free(kept);
+        return ORC_ENOMEM;
+    }
+    for (int64_t j = 0; j < nb; ++j) {
+        const int64_t n0 = j * block, n1 = (n0 + block < V) ? n0 + block : V;
+        float best = scores[n0];
+        for (int64_t n = n0 + 1; n < n1; ++n)
+            if (scores[n] > best)
+                best = scores[n];
+        b[j].score = best;
+        b[j].j = j;
+    }
+    qsort(b, (size_t)nb, sizeof(orc_block), orc_block_cmp);
+    const int64_t m = nb < n_blocks ? nb : n_blocks;
+    for (int64_t i = 0; i < m; ++i)
+        kept[b[i].j] = 1;
+    int64_t len = 0;
+    for (int64_t n = 0; n < V; ++n)
+        if (kept[n / block])
+            pool_out[len++] = (int32_t)n;
+    for (int64_t i = len; i < (int64_t)n_blocks * block; ++i)
+        pool_out[i] = -1;
+    *pool_len = len;
+    free(b);
+    free(kept);
+    return ORC_OK;
+}
+
+/* Top-k of one query row over a pool of positions.  q: [H_I, d_I] int8,
+ * w: [H_I], keys: [N, d_I] int8, pool[0..pool_len) ascending positions
+ * (each < N).  idx_out[0..k): kept positions, ascending, -1 padded. */
+int orc_pool_topk(const int8_t *q, const float *w, const int8_t *keys, int32_t H_I, int32_t d_I,
+                  int64_t N, const int32_t *pool, int64_t pool_len, int32_t k, int32_t *idx_out)
+{
+    if (!q || !w || !keys || !idx_out || H_I <= 0 || d_I <= 0 || N < 0 || pool_len < 0 ||
+        k <= 0 || (pool_len > 0 && !pool))
+        return ORC_EINVAL;
+    orc_cand *c = (orc_cand *)malloc((size_t)(pool_len > 0 ? pool_len : 1) * sizeof(orc_cand));
+    if (!c)
+        return ORC_ENOMEM;
+    for (int64_t i = 0; i < pool_len; ++i) {
+        if (pool[i] < 0 || pool[i] >= N) {
+            free(c);
+            return ORC_ERANGE;
+        }
+        orc_index_score_row(q, w, keys + (int64_t)pool[i] * d_I, H_I, d_I, 1, &c[i].score);
+        c[i].n = pool[i];
+    }
+    qsort(c, (size_t)pool_len, sizeof(orc_cand), orc_cand_cmp);
+    const int64_t m = pool_len < k ? pool_len : k;
+    for (int64_t i = 0; i < m; ++i)
+        idx_out[i] = (int32_t)c[i].n;
+    qsort(idx_out, (size_t)m, sizeof(int32_t), orc_i32_cmp);
+    for (int64_t i = m; i < k; ++i)
+        idx_out[i] = -1;
+    free(c);
+    return ORC_OK;
+}
