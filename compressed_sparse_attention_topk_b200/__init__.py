@@ -31,7 +31,8 @@ EXPORTED = (
     "csa2_sparse_attn_decode", "csa2_sparse_attn_prefill", "csa2_validate_modes",
     "csa2_group_cache_bytes", "csa2_layer_group_workspace_size", "csa2_layer_group_run",
     "csa2_get_device_status", "csa2_trace_enable", "csa2_trace_count", "csa2_trace_get",
-    "csa2_layer_run", "csa2_index_topk_noalloc",
+    "csa2_layer_run", "csa2_index_topk_noalloc", "csa2_index_pool_workspace_size",
+    "csa2_index_pool", "csa2_pool_topk_workspace_size", "csa2_pool_topk",
 )
 
 
@@ -91,6 +92,10 @@ def lib() -> ctypes.CDLL:
         "csa2_layer_run": ([P, P, i32, i32, P, P, sz, P], i32),
         "csa2_index_topk_noalloc": ([P, P, P, i32, i32, i32, i32, i64, i64, i32, i32, P, P, P],
                                     i32),
+        "csa2_index_pool_workspace_size": ([i32, i32, i32, i64, i32, i32], sz),
+        "csa2_index_pool": ([P, P, P, i32, i32, i32, i64, i32, i32, P, P, sz, P], i32),
+        "csa2_pool_topk_workspace_size": ([i32, i32, i32], sz),
+        "csa2_pool_topk": ([P, P, P, i32, i32, i32, i64, P, i32, i32, P, P, sz, P], i32),
         "csa2_get_device_status": ([P, P], i32),
         "csa2_trace_enable": ([i32], i32),
         "csa2_trace_count": ([], i32),
@@ -208,6 +213,56 @@ def index_topk(q_idx, w, k_idx, topk: int, n_prior: int = -1, ratio: int = 4, id
                                  ratio, topk, _ptr(idx_out), _ptr(scores), _ptr(ws), ws.numel(),
                                  _stream()), "csa2_index_topk")
     return (idx_out, scores) if want_scores else idx_out
+
+
+# --- hierarchical indexer -----------------------------------------------------
+
+def index_pool_workspace_size(B, H_I, d_I, N, block, n_blocks) -> int:
+    return int(lib().csa2_index_pool_workspace_size(B, H_I, d_I, N, block, n_blocks))
+
+
+def index_pool(q_idx, w, k_idx, block: int = 8, n_blocks: int = 2048, ws=None):
+    """Candidate pool of each sequence's Full-layer query: q_idx int8
+    [B,H_I,d_I], w fp32 [B,H_I], k_idx int8 [B,N,d_I] -> int32
+    [B, n_blocks*block] positions ascending, then -1."""
+    torch = _torch()
+    q_idx = _dev(q_idx, "q_idx", torch.int8)
+    w = _dev(w, "w", torch.float32)
+    k_idx = _dev(k_idx, "k_idx", torch.int8)
+    B, H_I, d_I = q_idx.shape
+    N = k_idx.shape[1]
+    pool = torch.empty((B, n_blocks * block), dtype=torch.int32, device=q_idx.device)
+    if ws is None:
+        ws = workspace(index_pool_workspace_size(B, H_I, d_I, N, block, n_blocks))
+    _check(lib().csa2_index_pool(_ptr(q_idx), _ptr(w), _ptr(k_idx), B, H_I, d_I, N, block,
+                                 n_blocks, _ptr(pool), _ptr(ws), ws.numel(), _stream()),
+           "csa2_index_pool")
+    return pool
+
+
+def pool_topk_workspace_size(B, P, topk) -> int:
+    return int(lib().csa2_pool_topk_workspace_size(B, P, topk))
+
+
+def pool_topk(q_idx, w, k_idx, pool, topk: int, ws=None):
+    """Top-k of each sequence's query within its pool (int32 [B, P],
+    positions ascending then -1) -> int32 [B, topk] positions ascending,
+    then -1."""
+    torch = _torch()
+    q_idx = _dev(q_idx, "q_idx", torch.int8)
+    w = _dev(w, "w", torch.float32)
+    k_idx = _dev(k_idx, "k_idx", torch.int8)
+    pool = _dev(pool, "pool", torch.int32)
+    B, H_I, d_I = q_idx.shape
+    N = k_idx.shape[1]
+    P = pool.shape[1]
+    out = torch.empty((B, topk), dtype=torch.int32, device=q_idx.device)
+    if ws is None:
+        ws = workspace(pool_topk_workspace_size(B, P, topk))
+    _check(lib().csa2_pool_topk(_ptr(q_idx), _ptr(w), _ptr(k_idx), B, H_I, d_I, N, _ptr(pool), P,
+                                topk, _ptr(out), _ptr(ws), ws.numel(), _stream()),
+           "csa2_pool_topk")
+    return out
 
 
 # --- attention ----------------------------------------------------------------

@@ -11,6 +11,7 @@
 #include "common.cuh"
 #include "index_scan.cuh"
 #include "pack.cuh"
+#include "pool.cuh"
 #include "prefill_gemm.cuh"
 #include "row_cluster.cuh"
 
@@ -722,6 +723,185 @@ csa2_status run_index_topk(const int8_t *q_idx, const float *w, const int8_t *k_
 }
 
 // ---------------------------------------------------------------------------
+// Hierarchical indexer (pool.cuh): the pool of a Full row, the top-k of a
+// Reindex row within a pool.  Decode shape: one query per sequence.
+// ---------------------------------------------------------------------------
+constexpr int32_t kPoolMaxBlock = 64;
+constexpr int64_t kPoolMaxLen = 65536;
+
+struct PoolWs {
+  TopkWs t;         // full-row scores, their histograms, candidate overflow
+  float *bscores;   // [R, round4(nb)] block maxima
+  uint32_t *bhist;  // [R, kHistStride] their digit-1 histograms
+  int32_t *bidx;    // [B, n_blocks] kept blocks
+  size_t bytes;
+};
+
+PoolWs pool_ws_layout(void *base, int64_t R, int64_t B, int64_t N, int32_t block,
+                      int32_t n_blocks) {
+  PoolWs w{};
+  w.t = topk_ws_layout(base, R, N);
+  size_t off = w.t.bytes;
+  auto take = [&](size_t bytes) {
+    size_t o = off;
+    off += align_up(bytes, 256);
+    return o;
+  };
+  const int64_t nb = ceil_div(N, block);
+  const size_t o_bs = take(size_t(R) * size_t((nb + 3) & ~int64_t(3)) * 4);
+  const size_t o_bh = take(size_t(R) * kHistStride * 4);
+  const size_t o_bi = take(size_t(B) * n_blocks * 4);
+  char *p = static_cast<char *>(base);
+  w.bscores = reinterpret_cast<float *>(p + o_bs);
+  w.bhist = reinterpret_cast<uint32_t *>(p + o_bh);
+  w.bidx = reinterpret_cast<int32_t *>(p + o_bi);
+  w.bytes = off;
+  return w;
+}
+
+struct PoolTopkWs {
+  TopkWs t;     // pool scores, their histograms, candidate overflow
+  int32_t *sel; // [B, topk] selected pool slots
+  size_t bytes;
+};
+
+PoolTopkWs pool_topk_ws_layout(void *base, int64_t R, int64_t B, int64_t P, int32_t topk) {
+  PoolTopkWs w{};
+  w.t = topk_ws_layout(base, R, P);
+  const size_t o = w.t.bytes;
+  w.sel = reinterpret_cast<int32_t *>(static_cast<char *>(base) + o);
+  w.bytes = o + align_up(size_t(B) * topk * 4, 256);
+  return w;
+}
+
+csa2_status check_pool_common(const int8_t *q_idx, const float *w, const int8_t *k_idx,
+                              int32_t B, int32_t H_I, int32_t d_I, int64_t N) {
+  if (B < 0 || N < 0 || H_I < 1 || d_I < 1 || d_I % 16 != 0) return CSA2_ERR_INVALID_ARG;
+  if (!scan_shape_supported(H_I, d_I) || N >= (int64_t(1) << 31) - 1 || B > 65535)
+    return CSA2_ERR_UNSUPPORTED;
+  if (B == 0) return CSA2_OK;
+  if (!q_idx || !w || (N > 0 && !k_idx)) return CSA2_ERR_INVALID_ARG;
+  if (!aligned(q_idx, 16) || (k_idx && !aligned(k_idx, 16)) || !aligned(w, 4))
+    return CSA2_ERR_INVALID_ARG;
+  return CSA2_OK;
+}
+
+csa2_status run_index_pool(const int8_t *q_idx, const float *w, const int8_t *k_idx, int32_t B,
+                           int32_t H_I, int32_t d_I, int64_t N, int32_t block, int32_t n_blocks,
+                           int32_t *pool_out, void *ws, size_t ws_bytes, cudaStream_t st) {
+  const int64_t P = int64_t(n_blocks) * block;
+  if (N == 0) {  // nothing stored: an empty pool
+    return cudaMemsetAsync(pool_out, 0xff, size_t(B) * P * 4, st) == cudaSuccess ? CSA2_OK
+                                                                                : CSA2_ERR_CUDA;
+  }
+  const int64_t rows = B;
+  const int64_t R = topk_rows_per_pass(rows, N);
+  const PoolWs L0 = pool_ws_layout(nullptr, R, B, N, block, n_blocks);
+  if (!ws || ws_bytes < L0.bytes || !aligned(ws, 16)) return CSA2_ERR_WORKSPACE;
+  const PoolWs L = pool_ws_layout(ws, R, B, N, block, n_blocks);
+  const ScanLaunch scan = pick_scan(d_I, H_I);
+  if (!scan) return CSA2_ERR_UNSUPPORTED;
+  const int sms = device_sms();
+  const int64_t nb = ceil_div(N, block);
+  const int64_t bstride = (nb + 3) & ~int64_t(3);
+  for (int64_t row0 = 0; row0 < rows; row0 += R) {
+    const int64_t nr = std::min<int64_t>(R, rows - row0);
+    // the Full row's scores over the whole store
+    if (cudaMemsetAsync(L.t.hist1, 0, size_t(nr) * kHistStride * 4, st) != cudaSuccess)
+      return CSA2_ERR_CUDA;
+    const int64_t g_want = std::max<int64_t>(1, (2 * sms + nr / 2) / nr);
+    const int G = (int)std::min(g_want, std::max<int64_t>(1, N / 256));
+    {
+      TraceScope ts("index_scan", st);
+      scan(dim3(G, (unsigned)nr), st, q_idx, w, k_idx, 1, N, -1, 1, row0, L.t.scores,
+           score_stride(N), L.t.hist1, 0);
+    }
+    if (after_launch() != CSA2_OK) return CSA2_ERR_CUDA;
+    // block maxima and their histogram
+    if (cudaMemsetAsync(L.bhist, 0, size_t(nr) * kHistStride * 4, st) != cudaSuccess)
+      return CSA2_ERR_CUDA;
+    {
+      TraceScope ts("pool_block_max", st);
+      block_max_kernel<<<dim3((unsigned)ceil_div(nb, kPoolThreads), (unsigned)nr), kPoolThreads,
+                         0, st>>>(L.t.scores, score_stride(N), N, block, L.bscores, bstride,
+                                  L.bhist);
+    }
+    if (after_launch() != CSA2_OK) return CSA2_ERR_CUDA;
+    // the best n_blocks blocks, ascending
+    RowParams p{};
+    p.scores = L.bscores;
+    p.score_stride = bstride;
+    p.hist1 = L.bhist;
+    p.cand = L.t.cand;
+    p.N = nb;
+    p.T = 1;
+    p.n_prior = -1;
+    p.ratio = 1;
+    p.row0 = row0;
+    p.topk = n_blocks;
+    p.idx = L.bidx;
+    p.do_topk = 1;
+    if (launch_row(p, 64, nr, st) != CSA2_OK) return CSA2_ERR_CUDA;
+  }
+  {
+    TraceScope ts("pool_expand", st);
+    expand_pool_kernel<<<dim3((unsigned)ceil_div(P, kPoolThreads), (unsigned)B), kPoolThreads, 0,
+                         st>>>(L.bidx, n_blocks, block, N, pool_out);
+  }
+  return after_launch();
+}
+
+csa2_status run_pool_topk(const int8_t *q_idx, const float *w, const int8_t *k_idx, int32_t B,
+                          int32_t H_I, int32_t d_I, int64_t N, const int32_t *pool, int32_t P,
+                          int32_t topk, int32_t *idx_out, void *ws, size_t ws_bytes,
+                          cudaStream_t st) {
+  if (P == 0) {  // an empty pool selects nothing
+    return cudaMemsetAsync(idx_out, 0xff, size_t(B) * topk * 4, st) == cudaSuccess
+               ? CSA2_OK
+               : CSA2_ERR_CUDA;
+  }
+  const int64_t rows = B;
+  const int64_t R = topk_rows_per_pass(rows, P);
+  const PoolTopkWs L0 = pool_topk_ws_layout(nullptr, R, B, P, topk);
+  if (!ws || ws_bytes < L0.bytes || !aligned(ws, 16)) return CSA2_ERR_WORKSPACE;
+  const PoolTopkWs L = pool_topk_ws_layout(ws, R, B, P, topk);
+  const int64_t pstride = score_stride(P);
+  for (int64_t row0 = 0; row0 < rows; row0 += R) {
+    const int64_t nr = std::min<int64_t>(R, rows - row0);
+    if (cudaMemsetAsync(L.t.hist1, 0, size_t(nr) * kHistStride * 4, st) != cudaSuccess)
+      return CSA2_ERR_CUDA;
+    {
+      TraceScope ts("pool_scan", st);
+      pool_scan_kernel<<<dim3((unsigned)ceil_div(P, kPoolThreads), (unsigned)nr), kPoolThreads, 0,
+                         st>>>(q_idx + row0 * H_I * d_I, w + row0 * H_I,
+                               N > 0 ? k_idx + row0 * N * d_I : k_idx, H_I, d_I, N,
+                               pool + row0 * P, P, L.t.scores, pstride, L.t.hist1);
+    }
+    if (after_launch() != CSA2_OK) return CSA2_ERR_CUDA;
+    RowParams p{};
+    p.scores = L.t.scores;
+    p.score_stride = pstride;
+    p.hist1 = L.t.hist1;
+    p.cand = L.t.cand;
+    p.N = P;
+    p.T = 1;
+    p.n_prior = -1;
+    p.ratio = 1;
+    p.row0 = row0;
+    p.topk = topk;
+    p.idx = L.sel;
+    p.do_topk = 1;
+    if (launch_row(p, 64, nr, st) != CSA2_OK) return CSA2_ERR_CUDA;
+  }
+  {
+    TraceScope ts("pool_map", st);
+    map_pool_kernel<<<dim3((unsigned)ceil_div(topk, kPoolThreads), (unsigned)B), kPoolThreads, 0,
+                      st>>>(L.sel, topk, pool, P, N, idx_out);
+  }
+  return after_launch();
+}
+
+// ---------------------------------------------------------------------------
 // Attention with given indices.
 // ---------------------------------------------------------------------------
 csa2_status check_attn_args(const uint16_t *q, const uint8_t *codes, const float *scales,
@@ -913,6 +1093,48 @@ csa2_status csa2_index_topk(const int8_t *q_idx, const float *w, const int8_t *k
   if (rc != CSA2_OK || int64_t(B) * T == 0) return rc;
   return run_index_topk(q_idx, w, k_idx, B, T, H_I, d_I, N, n_prior, ratio, topk, idx_out,
                         score_out, nullptr, ws, ws_bytes, as_stream(stream));
+}
+
+size_t csa2_index_pool_workspace_size(int32_t B, int32_t H_I, int32_t d_I, int64_t N,
+                                      int32_t block, int32_t n_blocks) {
+  if (B < 0 || N < 0 || block < 1 || block > kPoolMaxBlock || n_blocks < 1 ||
+      int64_t(n_blocks) * block > kPoolMaxLen || !scan_shape_supported(H_I, d_I))
+    return 0;
+  const int64_t R = topk_rows_per_pass(B, N);
+  return pool_ws_layout(nullptr, R, B, N, block, n_blocks).bytes;
+}
+
+csa2_status csa2_index_pool(const int8_t *q_idx, const float *w, const int8_t *k_idx, int32_t B,
+                            int32_t H_I, int32_t d_I, int64_t N, int32_t block, int32_t n_blocks,
+                            int32_t *pool_out, void *ws, size_t ws_bytes, void *stream) {
+  if (block < 1 || n_blocks < 1) return CSA2_ERR_INVALID_ARG;
+  if (block > kPoolMaxBlock || int64_t(n_blocks) * block > kPoolMaxLen)
+    return CSA2_ERR_UNSUPPORTED;
+  csa2_status rc = check_pool_common(q_idx, w, k_idx, B, H_I, d_I, N);
+  if (rc != CSA2_OK || B == 0) return rc;
+  if (!pool_out || !aligned(pool_out, 4)) return CSA2_ERR_INVALID_ARG;
+  return run_index_pool(q_idx, w, k_idx, B, H_I, d_I, N, block, n_blocks, pool_out, ws, ws_bytes,
+                        as_stream(stream));
+}
+
+size_t csa2_pool_topk_workspace_size(int32_t B, int32_t P, int32_t topk) {
+  if (B < 0 || P < 0 || P > kPoolMaxLen || topk < 1 || topk > 65536) return 0;
+  const int64_t R = topk_rows_per_pass(B, P);
+  return pool_topk_ws_layout(nullptr, R, B, P, topk).bytes;
+}
+
+csa2_status csa2_pool_topk(const int8_t *q_idx, const float *w, const int8_t *k_idx, int32_t B,
+                           int32_t H_I, int32_t d_I, int64_t N, const int32_t *pool, int32_t P,
+                           int32_t topk, int32_t *idx_out, void *ws, size_t ws_bytes,
+                           void *stream) {
+  if (P < 0 || topk < 1) return CSA2_ERR_INVALID_ARG;
+  if (P > kPoolMaxLen || topk > 65536) return CSA2_ERR_UNSUPPORTED;
+  csa2_status rc = check_pool_common(q_idx, w, k_idx, B, H_I, d_I, N);
+  if (rc != CSA2_OK || B == 0) return rc;
+  if (!idx_out || !aligned(idx_out, 4) || (P > 0 && (!pool || !aligned(pool, 4))))
+    return CSA2_ERR_INVALID_ARG;
+  return run_pool_topk(q_idx, w, k_idx, B, H_I, d_I, N, pool, P, topk, idx_out, ws, ws_bytes,
+                       as_stream(stream));
 }
 
 size_t csa2_sparse_attn_workspace_size(int32_t B, int32_t T, int32_t H, int32_t D, int32_t topk,

@@ -168,6 +168,60 @@ csa2_status csa2_index_topk_noalloc(const int8_t *q_idx, const float *w, const i
                                     int32_t *idx_out, float *score_out, void *stream);
 
 /* ---------------------------------------------------------------------- */
+/* Hierarchical indexer: a Full layer's candidate pool, a Reindex layer's  */
+/* top-k within it                                                         */
+/* ---------------------------------------------------------------------- */
+
+/* "Inference-Efficient LLMs: How Sparse Compute and Compressed Memory
+ * Work", section 5 ("Hierarchical Sparse Indexing"): an earlier Full layer
+ * searches the whole context and keeps a candidate pool (the example: 2,048
+ * blocks of eight positions, 16,384 candidates); later Reindex layers
+ * search only within that pool.  This library's reading: block j covers
+ * positions [j*block, (j+1)*block) (the last block only those < N); a
+ * block's score is the largest index score (as in csa2_index_topk) among
+ * its positions; the best n_blocks blocks are kept, ties to the lower block;
+ * the pool lists their positions ascending.  Decode shape: one query per
+ * sequence. */
+
+/* Workspace bytes for csa2_index_pool (0 on invalid or unsupported sizes). */
+size_t csa2_index_pool_workspace_size(int32_t B, int32_t H_I, int32_t d_I, int64_t N,
+                                      int32_t block, int32_t n_blocks);
+
+/* The pool of each sequence's Full-layer query.
+ *   q_idx    device, int8 [B, H_I, d_I]
+ *   w        device, fp32 [B, H_I]
+ *   k_idx    device, int8 [B, N, d_I]   (16-byte aligned)
+ *   pool_out device, int32 [B, n_blocks * block]   (output) the kept
+ *            positions ascending, then -1 (fewer when fewer blocks exist, or
+ *            when the last block is partial)
+ *   ws       device workspace of ws_bytes >= csa2_index_pool_workspace_size
+ * Supported: the index shapes of csa2_index_topk, 1 <= block <= 64,
+ * n_blocks * block <= 65536, B <= 65535. */
+csa2_status csa2_index_pool(const int8_t *q_idx, const float *w, const int8_t *k_idx, int32_t B,
+                            int32_t H_I, int32_t d_I, int64_t N, int32_t block, int32_t n_blocks,
+                            int32_t *pool_out, void *ws, size_t ws_bytes, void *stream);
+
+/* Workspace bytes for csa2_pool_topk (0 on invalid or unsupported sizes). */
+size_t csa2_pool_topk_workspace_size(int32_t B, int32_t P, int32_t topk);
+
+/* Top-k of each sequence's (Reindex-layer) query within its pool: the
+ * index score of every pool position, then the min(topk, positions) best,
+ * ties to the lower position, ascending, then -1.
+ *   q_idx, w, k_idx as for csa2_index_pool (the Reindex layer's query, the
+ *            store's index keys)
+ *   pool     device, int32 [B, P]: positions ascending, then -1 entries (as
+ *            written by csa2_index_pool); an entry >= N counts as -1 and is
+ *            recorded in the device status word (bad index)
+ *   idx_out  device, int32 [B, topk]   (output)
+ *   ws       device workspace of ws_bytes >= csa2_pool_topk_workspace_size
+ * Supported: the index shapes of csa2_index_topk, P <= 65536,
+ * 1 <= topk <= 65536, B <= 65535. */
+csa2_status csa2_pool_topk(const int8_t *q_idx, const float *w, const int8_t *k_idx, int32_t B,
+                           int32_t H_I, int32_t d_I, int64_t N, const int32_t *pool, int32_t P,
+                           int32_t topk, int32_t *idx_out, void *ws, size_t ws_bytes,
+                           void *stream);
+
+/* ---------------------------------------------------------------------- */
 /* Sparse attention over the selected entries + the local window           */
 /* ---------------------------------------------------------------------- */
 

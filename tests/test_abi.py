@@ -121,3 +121,34 @@ def test_group_run_rejects_bad_table_before_launch(lib):
     dims = csa2.make_dims(1, 1, 16, 128, 100, 4, 64, 8, 4)
     rc = lib.csa2_layer_group_run(modes, io, 2, ctypes.byref(dims), None, 0, None)
     assert rc == csa2.CSA2_ERR_INVALID_ARG
+
+
+def test_pool_calls_validate_before_any_launch(lib):
+    P = ctypes.c_void_p
+    fake = P(256)
+    # workspace queries: supported sizes > 0, unsupported or invalid sizes 0
+    assert lib.csa2_index_pool_workspace_size(4, 4, 64, 262144, 8, 2048) > 4 * 262144 * 12
+    assert lib.csa2_index_pool_workspace_size(4, 4, 64, 262144, 65, 16) == 0    # block > 64
+    assert lib.csa2_index_pool_workspace_size(4, 4, 64, 262144, 8, 8193) == 0   # pool > 65,536
+    assert lib.csa2_index_pool_workspace_size(4, 3, 64, 262144, 8, 2048) == 0   # H_I unsupported
+    assert lib.csa2_pool_topk_workspace_size(4, 16384, 2048) > 4 * 16384 * 12
+    assert lib.csa2_pool_topk_workspace_size(4, 70000, 2048) == 0
+    assert lib.csa2_pool_topk_workspace_size(4, 16384, 0) == 0
+    # argument checks
+    rc = lib.csa2_index_pool(fake, fake, fake, 1, 4, 64, 100, 0, 4, fake, fake, 1 << 20, None)
+    assert rc == csa2.CSA2_ERR_INVALID_ARG
+    rc = lib.csa2_index_pool(fake, fake, fake, 1, 4, 64, 100, 128, 4, fake, fake, 1 << 20, None)
+    assert rc == csa2.CSA2_ERR_UNSUPPORTED
+    rc = lib.csa2_index_pool(fake, fake, P(258), 1, 4, 64, 100, 8, 4, fake, fake, 1 << 20, None)
+    assert rc == csa2.CSA2_ERR_INVALID_ARG                      # misaligned keys
+    rc = lib.csa2_pool_topk(fake, fake, fake, 1, 4, 64, 100, fake, 16, 0, fake, fake, 1 << 20,
+                            None)
+    assert rc == csa2.CSA2_ERR_INVALID_ARG                      # topk < 1
+    rc = lib.csa2_pool_topk(fake, fake, fake, 1, 4, 64, 100, None, 16, 8, fake, fake, 1 << 20,
+                            None)
+    assert rc == csa2.CSA2_ERR_INVALID_ARG                      # no pool
+    # no sequences: nothing to do
+    assert lib.csa2_index_pool(None, None, None, 0, 4, 64, 100, 8, 4, None, None, 0,
+                               None) == csa2.CSA2_OK
+    assert lib.csa2_pool_topk(None, None, None, 0, 4, 64, 100, None, 16, 8, None, None, 0,
+                              None) == csa2.CSA2_OK
