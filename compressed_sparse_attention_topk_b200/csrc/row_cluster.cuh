@@ -8,8 +8,12 @@
 // joint softmax, an entry is both key and value and serves every head).
 //
 // One cluster of CL CTAs owns one query row; CTA c owns a contiguous slice
-// of the row's entries.  Cluster barriers order the phases; histograms,
-// counts and softmax partials move through distributed shared memory.
+// of the row's entries.  Histogram slices, counts and softmax partials move
+// between the CTAs by st.async into the receiver's shared memory, each
+// delivery counted in bytes on the receiver's own mbarrier: a CTA waits only
+// for the data it needs, and only the prologue (every CTA running, its
+// barriers initialised) and the step between head passes use a cluster-wide
+// barrier.
 //
 // Top-k: exact radix selection on an order-preserving 32-bit key of the
 // score, digits of 11, 11 and 10 bits.  The scan kernel has histogrammed
@@ -21,7 +25,7 @@
 //      prefix, then each thread writes its run's candidates), histogramming
 //      digit 2 of the elements exactly at t1;
 //   2. reduces the cluster's digit-2 histograms (CTA c sums bin slice c of
-//      every rank and pushes the sums to every rank; every CTA then finds
+//      every rank and delivers the sums to every rank; every CTA then finds
 //      t2 locally) -> t2;
 //   3. only when the boundary bucket (t1, t2) holds more elements than still
 //      needed: the same for digit 3 -> t3;
@@ -47,8 +51,8 @@
 // Window rows use the same path with scale 1 (bf16 keys and values).  The
 // warps' states are merged in shared memory (their buffers alias the dead
 // top-k working set), and each CTA pushes its partial (max, sum, acc) of
-// head h into the shared memory of the CTA that owns h (h mod CL); after one
-// cluster barrier the owners merge locally by log-sum-exp.  Which CTA
+// head h into the shared memory of the CTA that owns h (h mod CL); once its
+// partials are in, each owner merges them locally by log-sum-exp.  Which CTA
 // handles which key does not change the result, so no entry is moved
 // between CTAs.
 #pragma once
