@@ -213,6 +213,21 @@ def oracle_sample(w0, seconds: float, min_runs: int = 1):
     return runs, dt
 
 
+def host_cpu() -> dict:
+    """The host's CPU model and logical core count (for the oracle timings);
+    "unknown" where the system does not say."""
+    model = "unknown"
+    try:
+        with open("/proc/cpuinfo") as f:
+            for ln in f:
+                if ln.startswith("model name"):
+                    model = ln.split(":", 1)[1].strip()
+                    break
+    except OSError:
+        pass
+    return {"cpu_model": model, "nproc": os.cpu_count() or 0}
+
+
 def run_reference(args, w0):
     _, rank, _ = dist_env()
     if rank != 0:
@@ -246,7 +261,7 @@ def run_reference(args, w0):
         "config": {"workload": w0.name, "B": w0.B, "N": w0.N, "layers": w0.L,
                    "topk": w0.topk, "parallelism": "host cores, rank 0 only"},
         "cpu_baseline": {"value": value, "unit": UNIT, "cores": 1, "kind": "oracle",
-                         "sample": sample},
+                         "sample": sample, **host_cpu()},
         "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
     print(json.dumps(line), flush=True)
@@ -489,7 +504,8 @@ def run_gpu(args, w0):
             runs, dt = oracle_sample(w0, args.cpu_seconds)
             cpu = {"value": runs * w0.T * w0.L / dt, "unit": UNIT, "cores": 1, "kind": "oracle",
                    "sample": f"{runs} sequence(s) x {w0.L} layers of the same workload "
-                             f"(N={w0.N}), plain C oracle, single thread, {dt:.1f} s"}
+                             f"(N={w0.N}), plain C oracle, single thread, {dt:.1f} s",
+                   **host_cpu()}
         line = {
             "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world,
             "steps": args.steps, "warmup": args.warmup,
