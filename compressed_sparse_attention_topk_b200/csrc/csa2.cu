@@ -4,6 +4,7 @@
 #include "csa2.h"
 
 #include <algorithm>
+#include <atomic>
 #include <cstdint>
 #include <cstring>
 
@@ -432,11 +433,17 @@ bool make_map_u8(CUtensorMap *m, const void *base, uint64_t d0, uint64_t d1, uin
            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-bool pf_eligible(int32_t T, int32_t H_I, int32_t d_I, int64_t N, int32_t topk,
-                 const float *score_out) {
+// Shapes the tensor-core prefill path serves (host arithmetic only: the
+// workspace query answers the same with or without a GPU driver).
+bool pf_shape_ok(int32_t T, int32_t H_I, int32_t d_I, int64_t N, int32_t topk) {
   return T >= kPfMinT && (d_I == 32 || d_I == 64 || d_I == 128) &&
          scan_shape_supported(H_I, d_I) && N >= 1 && N < (int64_t(1) << 31) - 1 &&
-         4 * int64_t(topk) <= 16384 && score_out == nullptr && encode_tiled() != nullptr;
+         4 * int64_t(topk) <= 16384;
+}
+
+bool pf_eligible(int32_t T, int32_t H_I, int32_t d_I, int64_t N, int32_t topk,
+                 const float *score_out) {
+  return pf_shape_ok(T, H_I, d_I, N, topk) && score_out == nullptr && encode_tiled() != nullptr;
 }
 
 // Key-axis positions per CTA: minimises (waves of CTAs) x (tiles per CTA +
@@ -1080,7 +1087,7 @@ size_t csa2_index_topk_workspace_size(int32_t B, int32_t T, int32_t H_I, int32_t
                                       int32_t topk) {
   if (B < 0 || T < 0 || N < 0 || topk < 1 || !scan_shape_supported(H_I, d_I)) return 0;
   size_t bytes = topk_ws_bytes(B, T, N);
-  if (pf_eligible(T, H_I, d_I, N, topk, nullptr)) bytes = std::max(bytes, pf_ws_bytes(T, N, d_I));
+  if (pf_shape_ok(T, H_I, d_I, N, topk)) bytes = std::max(bytes, pf_ws_bytes(T, N, d_I));
   return bytes;
 }
 
@@ -1311,23 +1318,25 @@ static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocScratch
 namespace {
 
 // Device address of the scratch on the current device, looked up once per
-// device (the name itself is only a host-side stand-in).
+// device (the name itself is only a host-side stand-in).  The address is
+// that of the device's primary context (the one the CUDA runtime uses).
+// Host threads may race on the first lookup: each stores the same address.
 void *noalloc_scratch(csa2_status *rc) {
-  static void *addr[256] = {nullptr};
+  static std::atomic<void *> addr[256];
   int dev = -1;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 256) {
     *rc = CSA2_ERR_CUDA;
     return nullptr;
   }
-  if (!addr[dev]) {
-    void *ptr = nullptr;
-    if (cudaGetSymbolAddress(&ptr, g_noalloc_scratch) != cudaSuccess || !ptr) {
+  void *a = addr[dev].load(std::memory_order_acquire);
+  if (!a) {
+    if (cudaGetSymbolAddress(&a, g_noalloc_scratch) != cudaSuccess || !a) {
       *rc = CSA2_ERR_CUDA;
       return nullptr;
     }
-    addr[dev] = ptr;
+    addr[dev].store(a, std::memory_order_release);
   }
-  return addr[dev];
+  return a;
 }
 
 }  // namespace
@@ -1341,7 +1350,8 @@ csa2_status csa2_index_topk_noalloc(const int8_t *q_idx, const float *w, const i
   csa2_status rc = check_topk_args(q_idx, w, k_idx, B, T, H_I, d_I, N, n_prior, ratio, topk,
                                    idx_out, score_out);
   if (rc != CSA2_OK || int64_t(B) * T == 0) return rc;
-  if (topk_ws_bytes(B, T, N) > kNoAllocScratchBytes) return CSA2_ERR_UNSUPPORTED;
+  if (csa2_index_topk_workspace_size(B, T, H_I, d_I, N, topk) > kNoAllocScratchBytes)
+    return CSA2_ERR_UNSUPPORTED;
   void *ws = noalloc_scratch(&rc);
   if (!ws) return rc;
   return run_index_topk(q_idx, w, k_idx, B, T, H_I, d_I, N, n_prior, ratio, topk, idx_out,

@@ -155,7 +155,9 @@ csa2_status csa2_index_topk(const int8_t *q_idx, const float *w, const int8_t *k
  * nothing itself.  Sizes whose scratch would exceed it
  * (csa2_index_topk_workspace_size(...) > 16 MiB) return CSA2_ERR_UNSUPPORTED
  * before anything is enqueued.  The first call on a device looks up the
- * array's device address and sets kernel attributes; make that first call
+ * array's device address (in the device's primary context, the one the
+ * CUDA runtime uses; calls made under another context of the same device
+ * are not supported) and sets kernel attributes; make that first call
  * before any stream capture.  All calls share the one array and leave their
  * contents in it (the parts that must start at zero are cleared by each
  * call), so calls that overlap on the GPU -- on different streams, or from

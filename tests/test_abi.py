@@ -152,3 +152,22 @@ def test_pool_calls_validate_before_any_launch(lib):
                                None) == csa2.CSA2_OK
     assert lib.csa2_pool_topk(None, None, None, 0, 4, 64, 100, None, 16, 8, None, None, 0,
                               None) == csa2.CSA2_OK
+
+
+def test_noalloc_refuses_by_the_documented_workspace_size(lib):
+    """The allocation-free index + top-k refuses, before any launch, every
+    size whose csa2_index_topk_workspace_size exceeds its 16 MiB scratch --
+    including many-query shapes where only the tensor-core path's scratch
+    is too large."""
+    fake = ctypes.c_void_p(256)
+    limit = 16 << 20
+    # 512 queries over 1,000 entries: the per-row scan would need ~10 MB,
+    # the tensor-core path ~17 MB
+    assert csa2.index_topk_workspace_size(1, 512, 4, 64, 1000, 256) > limit
+    rc = lib.csa2_index_topk_noalloc(fake, fake, fake, 1, 512, 4, 64, 1000, -1, 4, 256, fake,
+                                     None, None)
+    assert rc == csa2.CSA2_ERR_UNSUPPORTED
+    # 4 x 1,000,000 decode entries: ~48 MB
+    rc = lib.csa2_index_topk_noalloc(fake, fake, fake, 4, 1, 4, 64, 1_000_000, -1, 4, 2048,
+                                     fake, None, None)
+    assert rc == csa2.CSA2_ERR_UNSUPPORTED
