@@ -69,9 +69,10 @@ def _load():
         lib.orc_group_cache_bytes.argtypes = [P, i32, i64, i64, i64, P]
         lib.orc_block_pool.argtypes = [P, i64, i32, i32, P, P]
         lib.orc_pool_topk.argtypes = [P, P, P, i32, i32, i64, P, i64, i32, P]
+        lib.orc_append_entry.argtypes = [P, P, P, i32, i32, i32, i64, P, P, P]
         for name in ("orc_pack_fp4", "orc_unpack_fp4", "orc_topk_row", "orc_index_topk",
                      "orc_sparse_attn", "orc_validate_modes", "orc_group_cache_bytes",
-                     "orc_block_pool", "orc_pool_topk"):
+                     "orc_block_pool", "orc_pool_topk", "orc_append_entry"):
             getattr(lib, name).restype = ctypes.c_int
         _lib = lib
     return _lib
@@ -121,6 +122,23 @@ def unpack_fp4(codes: np.ndarray, scales: np.ndarray, D: int) -> np.ndarray:
     _check(_load().orc_unpack_fp4(_ptr(codes), _ptr(scales), codes.shape[0], D, _ptr(out)),
            "unpack_fp4")
     return out
+
+
+def append_entry(src, key, pos, codes, scales, k_idx):
+    """One decode step's entry append, in place: for each sequence b with
+    pos[b] >= 0, src[b] (fp32 [D]) packed to FP4 into row pos[b] of codes
+    [B, N, D/2] / scales [B, N, D/16], and key[b] (int8 [d_I]) into row
+    pos[b] of k_idx [B, N, d_I].  The arrays must be C-contiguous numpy
+    arrays of those dtypes (they are modified)."""
+    src, key, pos = _c(src, np.float32), _c(key, np.int8), _c(pos, np.int64)
+    B, D = src.shape
+    d_I = key.shape[1]
+    N = codes.shape[1]
+    for a, dt in ((codes, np.uint8), (scales, np.float32), (k_idx, np.int8)):
+        if a.dtype != dt or not a.flags["C_CONTIGUOUS"]:
+            raise OracleError("append_entry: stores must be C-contiguous arrays of their dtype")
+    _check(_load().orc_append_entry(_ptr(src), _ptr(key), _ptr(pos), B, D, d_I, N, _ptr(codes),
+                                    _ptr(scales), _ptr(k_idx)), "append_entry")
 
 
 # --- indexer + top-k --------------------------------------------------------

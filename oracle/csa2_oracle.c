@@ -141,6 +141,43 @@ int orc_unpack_fp4(const uint8_t *codes, const float *scales, int64_t rows, int3
 }
 
 /* ------------------------------------------------------------------------ */
+/* Entry append: the per-token write side of the cache.                     */
+/* [P2] "Fast memory, persistent storage and recomputation": the main cache */
+/* entries are stored in a 4-bit floating-point format; [P3] section 6: FP4 */
+/* with per-group scaling.  Reading: when a decode token completes a        */
+/* compressed entry, that entry (its D values as the compressor produced    */
+/* them) is packed with the rule of orc_pack_fp4 into row pos[b] of its     */
+/* sequence's store, and its int8 index key is written into the same row of */
+/* the store's index keys; a sequence with pos[b] < 0 appends nothing.      */
+/* src [B, D] fp32, key [B, d_I] int8, pos [B]; codes [B, N, D/2], scales   */
+/* [B, N, D/16], k_idx [B, N, d_I] are updated in place.  A position >= N   */
+/* is an error: nothing is written and ORC_ERANGE is returned.              */
+/* ------------------------------------------------------------------------ */
+int orc_append_entry(const float *src, const int8_t *key, const int64_t *pos, int32_t B, int32_t D,
+                     int32_t d_I, int64_t N, uint8_t *codes, float *scales, int8_t *k_idx)
+{
+    if (!src || !key || !pos || !codes || !scales || !k_idx || B < 0 || D <= 0 || D % 16 != 0 ||
+        d_I <= 0 || N < 0)
+        return ORC_EINVAL;
+    for (int32_t b = 0; b < B; ++b)
+        if (pos[b] >= N)
+            return ORC_ERANGE;
+    for (int32_t b = 0; b < B; ++b) {
+        const int64_t n = pos[b];
+        if (n < 0)
+            continue;
+        const int64_t row = (int64_t)b * N + n;
+        int rc = orc_pack_fp4(src + (int64_t)b * D, 1, D, codes + row * (D / 2),
+                              scales + row * (D / 16));
+        if (rc != ORC_OK)
+            return rc;
+        for (int32_t i = 0; i < d_I; ++i)
+            k_idx[row * d_I + i] = key[(int64_t)b * d_I + i];
+    }
+    return ORC_OK;
+}
+
+/* ------------------------------------------------------------------------ */
 /* Indexer: a cheap relevance score of every compressed entry.              */
 /* [P1] section 4 ("The indexer"): index heads score the compressed         */
 /* positions before the expensive attention.  Reading: per head h an exact  */
