@@ -70,9 +70,15 @@ def _load():
         lib.orc_block_pool.argtypes = [P, i64, i32, i32, P, P]
         lib.orc_pool_topk.argtypes = [P, P, P, i32, i32, i64, P, i64, i32, P]
         lib.orc_append_entry.argtypes = [P, P, P, i32, i32, i32, i64, P, P, P]
+        lib.orc_pack_mxfp4.argtypes = [P, i64, i32, P, P]
+        lib.orc_unpack_mxfp4.argtypes = [P, P, i64, i32, P]
+        lib.orc_index_score_fp4k_row.argtypes = [P, P, P, P, i32, i32, i64, P]
+        lib.orc_index_score_fp4k_row.restype = None
+        lib.orc_index_topk_fp4k.argtypes = [P, P, P, P, i32, i32, i32, i64, i32, P, P]
         for name in ("orc_pack_fp4", "orc_unpack_fp4", "orc_topk_row", "orc_index_topk",
                      "orc_sparse_attn", "orc_validate_modes", "orc_group_cache_bytes",
-                     "orc_block_pool", "orc_pool_topk", "orc_append_entry"):
+                     "orc_block_pool", "orc_pool_topk", "orc_append_entry",
+                     "orc_pack_mxfp4", "orc_unpack_mxfp4", "orc_index_topk_fp4k"):
             getattr(lib, name).restype = ctypes.c_int
         _lib = lib
     return _lib
@@ -181,6 +187,57 @@ def index_topk(q_idx, w, k_idx, topk, n_prior=-1, ratio=4, rows=None, want_score
     _check(_load().orc_index_topk(_ptr(q_idx), _ptr(w), _ptr(k_idx), B, T, H_I, d_I, N, n_prior,
                                   ratio, topk, _ptr(rows_arr), nrows, _ptr(idx), _ptr(scores)),
            "index_topk")
+    return (idx, scores) if want_scores else idx
+
+
+# --- FP4 index keys (E2M1 with a power-of-two scale per 32 elements) ------------
+
+def pack_mxfp4(src: np.ndarray):
+    """fp32 [rows, d] -> (codes u8 [rows, d/2], biased exponents u8 [rows, d/32])."""
+    src = _c(src, np.float32)
+    rows, d = src.shape
+    codes = np.zeros((rows, d // 2), np.uint8)
+    exps = np.zeros((rows, d // 32), np.uint8)
+    _check(_load().orc_pack_mxfp4(_ptr(src), rows, d, _ptr(codes), _ptr(exps)), "pack_mxfp4")
+    return codes, exps
+
+
+def unpack_mxfp4(codes: np.ndarray, exps: np.ndarray, d: int) -> np.ndarray:
+    codes = _c(codes, np.uint8).reshape(-1, d // 2)
+    exps = _c(exps, np.uint8).reshape(-1, d // 32)
+    out = np.empty((codes.shape[0], d), np.float32)
+    _check(_load().orc_unpack_mxfp4(_ptr(codes), _ptr(exps), codes.shape[0], d, _ptr(out)),
+           "unpack_mxfp4")
+    return out
+
+
+def index_score_fp4k_row(q, w, codes, exps) -> np.ndarray:
+    """q int8 [H_I, d_I], w fp32 [H_I], codes u8 [N, d_I/2], exps u8 [N, d_I/32] -> fp32 [N]."""
+    q, w = _c(q, np.int8), _c(w, np.float32)
+    codes, exps = _c(codes, np.uint8), _c(exps, np.uint8)
+    H_I, d_I = q.shape
+    N = codes.shape[0]
+    out = np.empty(N, np.float32)
+    _load().orc_index_score_fp4k_row(_ptr(q), _ptr(w), _ptr(codes), _ptr(exps), H_I, d_I, N,
+                                     _ptr(out))
+    return out
+
+
+def index_topk_fp4k(q_idx, w, codes, exps, topk, want_scores=False):
+    """Decode rows over FP4 keys: q_idx int8 [B,H_I,d_I] (or [B,1,H_I,d_I]),
+    w fp32 [B,H_I], codes u8 [B,N,d_I/2], exps u8 [B,N,d_I/32] -> idx int32
+    [B, topk] (and scores fp32 [B, N])."""
+    q_idx = _c(q_idx, np.int8)
+    B = q_idx.shape[0]
+    H_I, d_I = q_idx.shape[-2:]
+    q_idx = q_idx.reshape(B, H_I, d_I)
+    w = _c(w, np.float32).reshape(B, H_I)
+    codes, exps = _c(codes, np.uint8), _c(exps, np.uint8)
+    N = codes.shape[1]
+    idx = np.empty((B, topk), np.int32)
+    scores = np.empty((B, N), np.float32) if want_scores else None
+    _check(_load().orc_index_topk_fp4k(_ptr(q_idx), _ptr(w), _ptr(codes), _ptr(exps), B, H_I, d_I,
+                                       N, topk, _ptr(idx), _ptr(scores)), "index_topk_fp4k")
     return (idx, scores) if want_scores else idx
 
 

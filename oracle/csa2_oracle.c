@@ -43,6 +43,8 @@
 #define ORC_ENOMEM 2
 #define ORC_ERANGE 3
 
+int orc_topk_row(const float *scores, int64_t V, int32_t k, int32_t *idx_out);
+
 /* ------------------------------------------------------------------------ */
 /* FP4 (E2M1) storage of the main cache entries, per-group scaling.         */
 /* [P2] "Fast memory, persistent storage and recomputation"; [P3] section 6.*/
@@ -202,6 +204,149 @@ void orc_index_score_row(const int8_t *q, const float *w, const int8_t *keys, in
         }
         out[n] = acc + 0.0f; /* a -0 sum is stored as +0 */
     }
+}
+
+/* ------------------------------------------------------------------------ */
+/* FP4 index keys.  [P3] section 6: V4 already used FP4 for parts of its    */
+/* attention indexing machinery.  Readings (the pages give no format for    */
+/* them): an index key is stored as E2M1 elements with one shared power-of- */
+/* two scale per block of 32 consecutive elements, the scale kept as an     */
+/* 8-bit biased exponent (the OCP Microscaling MXFP4 block format), so a    */
+/* d_I = 64 key takes 32 code bytes + 2 exponent bytes instead of 64 int8   */
+/* bytes.  Packing follows that format's conversion: shared exponent        */
+/* s = floor(log2(amax)) - 2 (2 = the largest E2M1 exponent), clamped to    */
+/* [-127, 127] and stored as s + 127; each element is x / 2^s rounded to    */
+/* the nearest E2M1 value (ties to even, saturating at 6; zero magnitude is */
+/* code 0); an all-zero block stores exponent byte 0 and zero codes.        */
+/* ------------------------------------------------------------------------ */
+
+/* 2^e as an fp32 value (exact for -149 <= e <= 127). */
+static float orc_pow2f(int e)
+{
+    return ldexpf(1.0f, e);
+}
+
+/* src [rows, d] fp32 -> codes [rows, d/2] (element 2i in the low nibble of
+ * byte i), exps [rows, d/32] (biased exponents).  d % 32 == 0. */
+int orc_pack_mxfp4(const float *src, int64_t rows, int32_t d, uint8_t *codes, uint8_t *exps)
+{
+    if (!src || !codes || !exps || rows < 0 || d <= 0 || d % 32 != 0)
+        return ORC_EINVAL;
+    const int32_t nb = d / 32;
+    for (int64_t r = 0; r < rows; ++r) {
+        for (int32_t g = 0; g < nb; ++g) {
+            const float *x = src + r * d + (int64_t)g * 32;
+            float amax = 0.0f;
+            for (int i = 0; i < 32; ++i)
+                if (fabsf(x[i]) > amax)
+                    amax = fabsf(x[i]);
+            uint8_t *cb = codes + r * (d / 2) + (int64_t)g * 16;
+            if (amax == 0.0f) {
+                exps[r * nb + g] = 0;
+                memset(cb, 0, 16);
+                continue;
+            }
+            int ex;
+            frexp((double)amax, &ex); /* amax = m * 2^ex, 0.5 <= m < 1 */
+            int s = (ex - 1) - 2;
+            if (s < -127)
+                s = -127;
+            if (s > 127)
+                s = 127;
+            exps[r * nb + g] = (uint8_t)(s + 127);
+            const float X = orc_pow2f(s);
+            for (int i = 0; i < 32; ++i) {
+                float y = x[i] / X;
+                uint32_t mag = orc_e2m1_round_mag(fabsf(y));
+                uint32_t c = mag;
+                if (mag != 0 && x[i] < 0.0f)
+                    c |= 8u;
+                uint8_t *byte = cb + i / 2;
+                if (i % 2 == 0)
+                    *byte = (uint8_t)((*byte & 0xF0u) | c);
+                else
+                    *byte = (uint8_t)((*byte & 0x0Fu) | (c << 4));
+            }
+        }
+    }
+    return ORC_OK;
+}
+
+/* out[r, i] = E2M1(code[r, i]) * 2^(exps[r, i/32] - 127), one fp32 multiply. */
+int orc_unpack_mxfp4(const uint8_t *codes, const uint8_t *exps, int64_t rows, int32_t d,
+                     float *out)
+{
+    if (!codes || !exps || !out || rows < 0 || d <= 0 || d % 32 != 0)
+        return ORC_EINVAL;
+    for (int64_t r = 0; r < rows; ++r)
+        for (int32_t i = 0; i < d; ++i) {
+            uint8_t byte = codes[r * (d / 2) + i / 2];
+            uint32_t c = (i % 2 == 0) ? (byte & 0x0Fu) : (byte >> 4);
+            out[r * d + i] = orc_e2m1_value(c) * orc_pow2f((int)exps[r * (d / 32) + i / 32] - 127);
+        }
+    return ORC_OK;
+}
+
+/* Index score over FP4 keys.  Reading: per head h and key block g the exact
+ * integer idot = sum_{i in g} q[h,i] * (2 * E2M1(code_i)) (twice the E2M1
+ * value is an integer in {0, +-1, +-2, +-3, +-4, +-6, +-8, +-12}); the
+ * head's dot product is the fp32 sum over blocks in ascending order of
+ * (float)idot * 2^(exp_g - 128) (each multiply and add rounded on its own;
+ * the -128 is the exponent bias 127 plus the factor 2 above); the heads are
+ * then summed with their weights exactly as for int8 keys.
+ * q: [H_I, d_I] int8, w: [H_I], codes: [N, d_I/2], exps: [N, d_I/32] -> out[N]. */
+void orc_index_score_fp4k_row(const int8_t *q, const float *w, const uint8_t *codes,
+                              const uint8_t *exps, int32_t H_I, int32_t d_I, int64_t N, float *out)
+{
+    const int32_t nb = d_I / 32;
+    for (int64_t n = 0; n < N; ++n) {
+        const uint8_t *cb = codes + n * (d_I / 2);
+        float acc = 0.0f;
+        for (int32_t h = 0; h < H_I; ++h) {
+            float dot = 0.0f;
+            for (int32_t g = 0; g < nb; ++g) {
+                int32_t idot = 0;
+                for (int32_t i = 32 * g; i < 32 * g + 32; ++i) {
+                    uint8_t byte = cb[i / 2];
+                    uint32_t c = (i % 2 == 0) ? (byte & 0x0Fu) : (byte >> 4);
+                    int32_t v2 = (int32_t)(2.0f * orc_e2m1_value(c)); /* exact small integer */
+                    idot += (int32_t)q[h * d_I + i] * v2;
+                }
+                float term = (float)idot * orc_pow2f((int)exps[n * nb + g] - 128);
+                dot = dot + term;
+            }
+            float t = w[h] * dot;
+            acc = acc + t;
+        }
+        out[n] = acc + 0.0f;
+    }
+}
+
+/* Index scores + top-k over FP4 keys for all rows of a decode batch (one
+ * query per sequence, every entry visible).  q_idx [B,H_I,d_I], w [B,H_I],
+ * codes [B,N,d_I/2], exps [B,N,d_I/32]; idx_out [B, topk]; scores_out NULL
+ * or [B, N]. */
+int orc_index_topk_fp4k(const int8_t *q_idx, const float *w, const uint8_t *codes,
+                        const uint8_t *exps, int32_t B, int32_t H_I, int32_t d_I, int64_t N,
+                        int32_t topk, int32_t *idx_out, float *scores_out)
+{
+    if (!q_idx || !w || (N > 0 && (!codes || !exps)) || !idx_out || B < 0 || H_I <= 0 ||
+        d_I <= 0 || d_I % 32 != 0 || N < 0 || topk <= 0)
+        return ORC_EINVAL;
+    float *row = (float *)malloc((size_t)(N > 0 ? N : 1) * sizeof(float));
+    if (!row)
+        return ORC_ENOMEM;
+    int rc = ORC_OK;
+    for (int32_t b = 0; b < B && rc == ORC_OK; ++b) {
+        orc_index_score_fp4k_row(q_idx + (int64_t)b * H_I * d_I, w + (int64_t)b * H_I,
+                                 codes + (int64_t)b * N * (d_I / 2), exps + (int64_t)b * N * (d_I / 32),
+                                 H_I, d_I, N, row);
+        if (scores_out)
+            memcpy(scores_out + (int64_t)b * N, row, (size_t)N * sizeof(float));
+        rc = orc_topk_row(row, N, topk, idx_out + (int64_t)b * topk);
+    }
+    free(row);
+    return rc;
 }
 
 /* Number of entries query t of a chunk may see.  Decode (n_prior < 0): all
