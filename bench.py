@@ -44,23 +44,30 @@ FALLBACK_HBM_GBS = 6650.0
 def parse_args():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=50)
+    ap.add_argument("--steps", type=int, default=100)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", default="csa2", choices=["csa2", "reference"])
     ap.add_argument("--workload", default=wl.LONG.name, choices=sorted(wl.ALL))
     ap.add_argument("--cpu-seconds", type=float, default=12.0,
                     help="CPU-baseline budget (oracle on the host cores)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--keys", default="int8", choices=["int8", "fp4"],
+                    help="index key format of the entry stores (fp4: E2M1 with a power-of-two "
+                         "scale per 32 elements; a supplementary line)")
+    ap.add_argument("--append", action="store_true",
+                    help="every step first appends one completed entry per sequence (FP4 "
+                         "entry + int8 key, at the store's last row) in the Full layer")
     ap.add_argument("--profile", action="store_true",
                     help="device-resident steps only (no trace pass, e2e, clocks or CPU "
                          "baseline): the command ncu captures")
     return ap.parse_args()
 
 
-def algorithmic_bytes(w0) -> dict:
+def algorithmic_bytes(w0, key_format: str = "int8") -> dict:
     """Per (sequence, layer, token): index keys scanned + selected FP4 entries
-    gathered (codes + scales) + bf16 window K and V."""
-    keys = w0.N * w0.d_I
+    gathered (codes + scales) + bf16 window K and V.  FP4 index keys take
+    d_I/2 code bytes + d_I/32 exponent bytes per entry."""
+    keys = w0.N * (w0.d_I if key_format == "int8" else w0.d_I // 2 + w0.d_I // 32)
     gather = w0.topk * (w0.D // 2 + w0.D // 4)
     window = 2 * w0.W * w0.D * 2
     return {"keys": keys, "gather": gather, "window": window, "total": keys + gather + window}
@@ -105,6 +112,8 @@ def pack_into_one_buffer(layers, keys, dev):
     plan, off = [], 0
     for l, d in enumerate(layers):
         for k in keys:
+            if k not in d:  # a tensor only some layers hold
+                continue
             nb = d[k].numel() * d[k].element_size()
             plan.append((l, k, off, nb))
             off += (nb + 255) // 256 * 256
@@ -117,22 +126,29 @@ def pack_into_one_buffer(layers, keys, dev):
     return buf, off
 
 
-def scan_source_sha() -> str:
+KERNEL_SOURCES = {
+    "index_scan": ("index_scan.cuh", "common.cuh"),
+    "decode_fused": ("decode_fused.cuh", "attn_rows.cuh", "common.cuh"),
+}
+
+
+def kernel_source_sha(kernel: str) -> str:
     h = hashlib.sha256()
-    for f in ("index_scan.cuh", "common.cuh"):
+    for f in KERNEL_SOURCES[kernel]:
         h.update(open(os.path.join(ROOT, "compressed_sparse_attention_topk_b200", "csrc", f),
                       "rb").read())
     return h.hexdigest()[:16]
 
 
-def ncu_traffic():
-    """DRAM bytes per index-scan launch from a committed ncu summary, only
-    while the kernel source is unchanged since the capture."""
-    p = os.path.join(ROOT, "profiles", "index_scan_traffic.json")
-    if not os.path.exists(p):
+def ncu_traffic(kernel: str):
+    """DRAM bytes per launch of `kernel` from a committed ncu summary
+    (profiles/<kernel>_traffic.json), only while the kernel's source is
+    unchanged since the capture."""
+    p = os.path.join(ROOT, "profiles", f"{kernel}_traffic.json")
+    if kernel not in KERNEL_SOURCES or not os.path.exists(p):
         return None
     d = json.load(open(p))
-    if d.get("source_sha") != scan_source_sha():
+    if d.get("source_sha") != kernel_source_sha(kernel):
         return None
     return d.get("dram_bytes_per_launch_full_size")
 
@@ -306,7 +322,16 @@ def run_gpu(args, w0):
             src = to_dev(lay["entries"])
             d["codes"], d["scales"] = csa2.pack_fp4(src)
             del src
-            d["k_idx"] = to_dev(lay["k_idx"])
+            if args.keys == "fp4":
+                ksrc = to_dev(wl.index_key_sources(w0, len(tens)))
+                d["k_idx"], d["k_exps"] = csa2.pack_index_keys_fp4(ksrc)
+                del ksrc
+            else:
+                d["k_idx"] = to_dev(lay["k_idx"])
+            if args.append:
+                app = wl.append_inputs(w0, 0)
+                d["app_src"], d["app_key"] = to_dev(app["src"]), to_dev(app["key"])
+                d["app_pos"] = torch.full((w0.B,), w0.N - 1, dtype=torch.int64, device=dev)
         d["idx"] = torch.empty((w0.B, 1, w0.topk), dtype=torch.int32, device=dev)
         d["out"] = torch.empty((w0.B, w0.H, w0.D), dtype=torch.float32, device=dev)
         d["lse"] = torch.empty((w0.B, w0.H), dtype=torch.float32, device=dev)
@@ -315,7 +340,15 @@ def run_gpu(args, w0):
     # Per-token inputs and per-step results of all layers live as views of one
     # device buffer each (256-byte aligned slots), so a step moves them with
     # one host->device and one device->host copy, as a serving loop would.
-    in_keys = ("q", "q_idx", "w", "win_k", "win_v")
+    # The per-token inputs are the queries, index queries, head weights and
+    # the new token's window row (K and V of every sequence); the step writes
+    # that row into the window's last slot on the device, and the older
+    # window rows stay resident (a decode loop keeps its window on the GPU).
+    for d in tens:
+        d["new_k"] = d["win_k"][:, -1].clone()
+        d["new_v"] = d["win_v"][:, -1].clone()
+    in_keys = ("q", "q_idx", "w", "new_k", "new_v") + (("app_src", "app_key") if args.append
+                                                        else ())
     out_keys = ("out", "lse", "idx")
     dev_in, _ = pack_into_one_buffer(tens, in_keys, dev)
     dev_out, _ = pack_into_one_buffer(tens, out_keys, dev)
@@ -454,6 +487,8 @@ def run_gpu(args, w0):
     d2h = host_out.numel()
 
     def e2e_steps(K):
+        """K end-to-end steps; per step the device ms of (inputs in + window
+        append, the layers, results out)."""
         res = []
         for _ in range(K):
             torch.cuda._sleep(sleep_cycles)
@@ -461,24 +496,38 @@ def run_gpu(args, w0):
             a, b = ev(), ev()
             a.record(stream)
             dev_in.copy_(host_in, non_blocking=True)
+            for d in tens:
+                d["win_k"][:, -1].copy_(d["new_k"])
+                d["win_v"][:, -1].copy_(d["new_v"])
             b.record(stream)
-            segs = [(a, b)]
+            segs = [("h2d", a, b)]
             for l in range(w0.L):
                 if l > 0:
                     flush()
                 a, b = ev(), ev()
                 a.record(stream)
                 graphs[l].replay()
-                if l == w0.L - 1:
-                    host_out.copy_(dev_out, non_blocking=True)
                 b.record(stream)
-                segs.append((a, b))
+                segs.append(("layers", a, b))
+            a, b = ev(), ev()
+            a.record(stream)
+            host_out.copy_(dev_out, non_blocking=True)
+            b.record(stream)
+            segs.append(("d2h", a, b))
             res.append(segs)
         torch.cuda.synchronize()
-        return [sum(a.elapsed_time(b) for a, b in s) for s in res]
+        out = []
+        for segs in res:
+            d = {"h2d": 0.0, "layers": 0.0, "d2h": 0.0}
+            for name, a, b in segs:
+                d[name] += a.elapsed_time(b)
+            out.append(d)
+        return out
 
     e2e_steps(3)
-    e2e_ms = max_over_ranks(dist, [float(sum(e2e_steps(args.steps)))], dev)[0]
+    e2e_recs = e2e_steps(args.steps)
+    e2e_seg = {k: sum(r[k] for r in e2e_recs) for k in ("h2d", "layers", "d2h")}
+    e2e_ms = max_over_ranks(dist, [float(sum(e2e_seg.values()))], dev)[0]
     clk = clocks.stop()
 
     status = csa2.get_device_status()
@@ -488,14 +537,20 @@ def run_gpu(args, w0):
     value = job_tokens_per_s(world, args.steps, w0.B, w0.T, w0.L, total_ms)
     e2e_value = job_tokens_per_s(world, args.steps, w0.B, w0.T, w0.L, e2e_ms)
 
-    ab = algorithmic_bytes(w0)
+    ab = algorithmic_bytes(w0, args.keys)
     peak, peak_kind = measured_peaks()
-    scan_n, scan_ms = per_kernel.get("index_scan", (0, 0.0))
-    scan_launch_bytes = w0.B * ab["keys"]
-    scan_avg_ms = scan_ms / max(scan_n, 1)
-    achieved = scan_launch_bytes / (scan_avg_ms * 1e-3) / 1e9 if scan_n else None
     step_bytes = w0.B * w0.L * ab["total"]
-    step_gbs = step_bytes / (total_ms / args.steps * 1e-3) / 1e9
+    ms_step = total_ms / args.steps
+    step_gbs = step_bytes / (ms_step * 1e-3) / 1e9
+    # The dominant kernel: one launch per layer does the whole layer (scan,
+    # top-k, gather, attention), so its algorithmic bytes per launch are the
+    # layer's: B x (keys + gathered entries + window).
+    dom = "decode_fused" if "decode_fused" in per_kernel else "index_scan"
+    dom_n, dom_ms = per_kernel.get(dom, (0, 0.0))
+    dom_avg_ms = dom_ms / max(dom_n, 1)
+    dom_bytes = w0.B * (ab["total"] if dom == "decode_fused" else ab["keys"])
+    achieved = dom_bytes / (dom_avg_ms * 1e-3) / 1e9 if dom_n else None
+    kernel_ms_per_step = sum(v[1] for v in per_kernel.values()) / args.steps
 
     line = None
     if rank == 0:
@@ -514,22 +569,32 @@ def run_gpu(args, w0):
             "config": {"workload": w0.name, "B": w0.B, "N": w0.N, "context_tokens": w0.N * 4,
                        "layers": "Full+Reindex" if w0.L == 2 else w0.L, "topk": w0.topk,
                        "H": w0.H, "D": w0.D, "H_I": w0.H_I, "d_I": w0.d_I, "W": w0.W,
+                       "index_keys": args.keys, "entry_append_per_step": bool(args.append),
                        "parallelism": f"replicas x{world}",
                        "l2": "flushed before every layer (256 MiB write, then 256 MiB read), flush not timed",
                        "step_algorithmic_bytes": step_bytes,
                        "step_hbm_gbs": step_gbs, "step_hbm_frac": step_gbs / peak,
                        "wall_s_timed_region": wall_s},
-            "roofline": {"bound": "hbm", "kernel": "index_scan", "timing": trace_kind,
+            "roofline": {"bound": "hbm", "kernel": dom, "timing": trace_kind,
                          "achieved": achieved,
                          "peak": peak, "peak_kind": f"{peak_kind} (copy bandwidth)",
                          "unit": "GB/s", "frac": (achieved / peak) if achieved else None,
-                         "traffic": ncu_traffic(),
-                         "bytes_per_launch": scan_launch_bytes,
-                         "avg_launch_ms": scan_avg_ms},
-            "kernels": {k: {"launches": c, "avg_us": s / c * 1e3, "share": s / sum(
-                v[1] for v in per_kernel.values())} for k, (c, s) in sorted(per_kernel.items())},
+                         "frac_of_8tbs_nominal": (achieved / 8000.0) if achieved else None,
+                         "traffic": ncu_traffic(dom),
+                         "bytes_per_launch": dom_bytes,
+                         "avg_launch_ms": dom_avg_ms,
+                         "step": {"achieved": step_gbs, "frac": step_gbs / peak,
+                                  "frac_of_8tbs_nominal": step_gbs / 8000.0,
+                                  "note": "algorithmic bytes of a whole step over ms_per_step "
+                                          "(launch gaps and workspace clears included)"}},
+            "kernels": {k: {"launches": c, "avg_us": s / c * 1e3,
+                            "ms_per_step": s / args.steps,
+                            "share_of_step": s / args.steps / ms_step}
+                        for k, (c, s) in sorted(per_kernel.items())},
+            "kernel_ms_per_step": kernel_ms_per_step,
             "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": h2d,
-                    "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms / args.steps},
+                    "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms / args.steps,
+                    "segments_ms_per_step": {k: v / args.steps for k, v in e2e_seg.items()}},
             "gpu_launches": int(round(launches_per_step * args.steps)),
             "clocks": clk,
             "cpu_baseline": cpu,

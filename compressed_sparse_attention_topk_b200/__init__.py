@@ -32,7 +32,9 @@ EXPORTED = (
     "csa2_group_cache_bytes", "csa2_layer_group_workspace_size", "csa2_layer_group_run",
     "csa2_get_device_status", "csa2_trace_enable", "csa2_trace_count", "csa2_trace_get",
     "csa2_layer_run", "csa2_index_topk_noalloc", "csa2_index_pool_workspace_size",
-    "csa2_index_pool", "csa2_pool_topk_workspace_size", "csa2_pool_topk",
+    "csa2_index_pool", "csa2_pool_topk_workspace_size", "csa2_pool_topk", "csa2_append_entry",
+    "csa2_pack_index_keys_fp4", "csa2_index_topk_fp4k_workspace_size", "csa2_index_topk_fp4k",
+    "csa2_wait_timeout_selftest",
 )
 
 
@@ -56,7 +58,8 @@ class Dims(ctypes.Structure):
 
 class LayerIO(ctypes.Structure):
     _fields_ = [(n, ctypes.c_void_p) for n in (
-        "q", "q_idx", "w", "win_k", "win_v", "codes", "scales", "k_idx", "idx", "out", "lse")]
+        "q", "q_idx", "w", "win_k", "win_v", "codes", "scales", "k_idx", "idx", "out", "lse",
+        "k_exps", "app_src", "app_key", "app_pos")]
 
 
 _lib = None
@@ -78,6 +81,10 @@ def lib() -> ctypes.CDLL:
         "csa2_version": ([], i32),
         "csa2_pack_fp4": ([P, i64, i32, P, P, P], i32),
         "csa2_unpack_fp4": ([P, P, i64, i32, P, P], i32),
+        "csa2_append_entry": ([P, P, P, i32, i32, i32, i64, P, P, P, P], i32),
+        "csa2_pack_index_keys_fp4": ([P, i64, i32, P, P, P], i32),
+        "csa2_index_topk_fp4k_workspace_size": ([i32, i32, i32, i64, i32], sz),
+        "csa2_index_topk_fp4k": ([P, P, P, P, i32, i32, i32, i64, i32, P, P, sz, P], i32),
         "csa2_index_topk_workspace_size": ([i32, i32, i32, i32, i64, i32], sz),
         "csa2_index_topk": ([P, P, P, i32, i32, i32, i32, i64, i64, i32, i32, P, P, P, sz, P], i32),
         "csa2_sparse_attn_workspace_size": ([i32, i32, i32, i32, i32, i32], sz),
@@ -97,6 +104,7 @@ def lib() -> ctypes.CDLL:
         "csa2_pool_topk_workspace_size": ([i32, i32, i32], sz),
         "csa2_pool_topk": ([P, P, P, i32, i32, i32, i64, P, i32, i32, P, P, sz, P], i32),
         "csa2_get_device_status": ([P, P], i32),
+        "csa2_wait_timeout_selftest": ([i64, P], i32),
         "csa2_trace_enable": ([i32], i32),
         "csa2_trace_count": ([], i32),
         "csa2_trace_get": ([i32, ctypes.POINTER(ctypes.c_char_p), ctypes.POINTER(f32)], i32),
@@ -174,6 +182,25 @@ def pack_fp4(src, codes=None, scales=None) -> Tuple[object, object]:
     return codes, scales
 
 
+def append_entry(src, key, pos, codes, scales, k_idx):
+    """One decode step's entry append, in place: for each sequence b with
+    pos[b] >= 0, src[b] (fp32 [B, D]) packed to FP4 into row pos[b] of
+    codes [B, N, D/2] / scales [B, N, D/16] and key[b] (int8 [B, d_I]) into
+    row pos[b] of k_idx [B, N, d_I]; pos is int64 [B] on the device."""
+    torch = _torch()
+    src = _dev(src, "src", torch.float32)
+    key = _dev(key, "key", torch.int8)
+    pos = _dev(pos, "pos", torch.int64)
+    codes = _dev(codes, "codes", torch.uint8)
+    scales = _dev(scales, "scales", torch.float32)
+    k_idx = _dev(k_idx, "k_idx", torch.int8)
+    B, D = src.shape
+    d_I = key.shape[1]
+    N = codes.shape[1]
+    _check(lib().csa2_append_entry(_ptr(src), _ptr(key), _ptr(pos), B, D, d_I, N, _ptr(codes),
+                                   _ptr(scales), _ptr(k_idx), _stream()), "csa2_append_entry")
+
+
 def unpack_fp4(codes, scales, D: int, out=None):
     torch = _torch()
     codes = _dev(codes, "codes", torch.uint8)
@@ -213,6 +240,47 @@ def index_topk(q_idx, w, k_idx, topk: int, n_prior: int = -1, ratio: int = 4, id
                                  ratio, topk, _ptr(idx_out), _ptr(scores), _ptr(ws), ws.numel(),
                                  _stream()), "csa2_index_topk")
     return (idx_out, scores) if want_scores else idx_out
+
+
+# --- FP4 index keys -----------------------------------------------------------
+
+def pack_index_keys_fp4(src, codes=None, exps=None):
+    """fp32 [..., d_I] -> (uint8 [..., d_I/2] E2M1 codes, uint8 [..., d_I/32]
+    biased block exponents): FP4 index keys with one power-of-two scale per
+    32 elements."""
+    torch = _torch()
+    src = _dev(src, "src", torch.float32)
+    d_I = src.shape[-1]
+    rows = src.numel() // d_I if d_I else 0
+    if codes is None:
+        codes = torch.empty(src.shape[:-1] + (d_I // 2,), dtype=torch.uint8, device=src.device)
+    if exps is None:
+        exps = torch.empty(src.shape[:-1] + (d_I // 32,), dtype=torch.uint8, device=src.device)
+    _check(lib().csa2_pack_index_keys_fp4(_ptr(src), rows, d_I, _ptr(codes), _ptr(exps),
+                                          _stream()), "csa2_pack_index_keys_fp4")
+    return codes, exps
+
+
+def index_topk_fp4k(q_idx, w, codes, exps, topk: int, idx_out=None, ws=None):
+    """Decode rows over FP4 index keys: q_idx int8 [B,H_I,d_I] (or
+    [B,1,H_I,d_I]), w fp32 [B,H_I], codes uint8 [B,N,d_I/2], exps uint8
+    [B,N,d_I/32] -> idx int32 [B, topk]."""
+    torch = _torch()
+    q_idx = _dev(q_idx, "q_idx", torch.int8)
+    w = _dev(w, "w", torch.float32)
+    codes = _dev(codes, "codes", torch.uint8)
+    exps = _dev(exps, "exps", torch.uint8)
+    B = q_idx.shape[0]
+    H_I, d_I = q_idx.shape[-2:]
+    N = codes.shape[1]
+    if idx_out is None:
+        idx_out = torch.empty((B, topk), dtype=torch.int32, device=q_idx.device)
+    if ws is None:
+        ws = workspace(int(lib().csa2_index_topk_fp4k_workspace_size(B, H_I, d_I, N, topk)))
+    _check(lib().csa2_index_topk_fp4k(_ptr(q_idx), _ptr(w), _ptr(codes), _ptr(exps), B, H_I, d_I,
+                                      N, topk, _ptr(idx_out), _ptr(ws), ws.numel(), _stream()),
+           "csa2_index_topk_fp4k")
+    return idx_out
 
 
 # --- hierarchical indexer -----------------------------------------------------

@@ -146,11 +146,12 @@ __device__ __forceinline__ void st_async_v2(void *dst, uint32_t a, uint32_t b, u
 // polling without suspension; on timeout record it in the status word and
 // return false.  The clock is read only once the phase is found incomplete:
 // a clock read costs as much as ~150 cycles on the waiting thread's path.
-__device__ __forceinline__ bool mbar_wait_bounded(uint64_t *bar, uint32_t parity) {
+__device__ __forceinline__ bool mbar_wait_bounded(uint64_t *bar, uint32_t parity,
+                                                  long long limit = (1ll << 32)) {
   if (mbar_test_wait(bar, parity)) return true;
   const long long start = clock64();
   while (!mbar_test_wait(bar, parity)) {
-    if (clock64() - start > (1ll << 32)) {
+    if (clock64() - start > limit) {
       raise_status(kStatusWaitTimeout);
       return false;
     }

@@ -6,10 +6,12 @@
 #include <algorithm>
 #include <atomic>
 #include <cstdint>
+#include <cstdlib>
 #include <cstring>
 
 #include "attn_rows.cuh"
 #include "common.cuh"
+#include "decode_fused.cuh"
 #include "index_scan.cuh"
 #include "pack.cuh"
 #include "pool.cuh"
@@ -646,13 +648,249 @@ csa2_status run_attn(const uint16_t *q, const uint8_t *codes, const float *scale
                      int32_t T, int32_t H, int32_t D, int64_t N, int32_t topk, int32_t W,
                      float sm_scale, float *out, float *lse, cudaStream_t st);
 
+// ---------------------------------------------------------------------------
+// The fused decode layer kernel (decode_fused.cuh): decode rows (one query
+// per sequence, every entry visible), no score output.
+// ---------------------------------------------------------------------------
+constexpr int kFusedMaxP = 16;                        // attention CTAs per row
+constexpr int64_t kFusedMaxRows = fd::kMaxG / 4;      // rows per launch (at least 4 CTAs each)
+constexpr int kFusedMaxPartD = 128;
+
+// Which decode kernel serves decode rows: the fused kernel unless the
+// environment sets CSA2_DECODE_KERNEL=cluster (the scan + per-row cluster
+// kernels), read once per process.
+bool fused_enabled() {
+  static int v = -1;
+  if (v < 0) {
+    const char *e = std::getenv("CSA2_DECODE_KERNEL");
+    v = (e && std::strcmp(e, "cluster") == 0) ? 0 : 1;
+  }
+  return v == 1;
+}
+
+struct FusedWs {
+  uint32_t *hist1, *arrive, *cnt;
+  uint2 *cand;
+  float *part;
+  size_t sync_bytes, bytes;
+};
+
+// Workspace of one launch of R rows: histograms and counters (cleared
+// before the launch, contiguous), slice counts, candidate lists, partials.
+FusedWs fused_ws_layout(void *base, int64_t R, int64_t N) {
+  FusedWs w{};
+  size_t off = 0;
+  auto take = [&](size_t bytes) {
+    size_t o = off;
+    off += align_up(bytes, 256);
+    return o;
+  };
+  const size_t o_hist = take(size_t(R) * fd::kHistStride * 4);
+  const size_t o_arr = off;  // right after the histograms: one clear covers both
+  off = o_arr + align_up(size_t(R) * fd::kArrive * 4, 256);
+  w.sync_bytes = off;
+  const size_t o_cnt = take(size_t(R) * fd::kMaxG * 4);
+  const size_t o_cand = take(size_t(R) * N * 8);
+  const size_t o_part = take(size_t(R) * kFusedMaxP * fd::kHeads * (kFusedMaxPartD + 4) * 4);
+  char *p = static_cast<char *>(base);
+  w.hist1 = reinterpret_cast<uint32_t *>(p + o_hist);
+  w.arrive = reinterpret_cast<uint32_t *>(p + o_arr);
+  w.cnt = reinterpret_cast<uint32_t *>(p + o_cnt);
+  w.cand = reinterpret_cast<uint2 *>(p + o_cand);
+  w.part = reinterpret_cast<float *>(p + o_part);
+  w.bytes = off;
+  return w;
+}
+
+size_t fused_ws_bytes(int64_t rows, int64_t N) {
+  return fused_ws_layout(nullptr, std::min<int64_t>(rows, kFusedMaxRows), N).bytes;
+}
+
+bool fused_shape_ok(int32_t T, int32_t H_I, int32_t d_I, int64_t N, int64_t n_prior,
+                    int32_t topk, bool fp4_keys = false) {
+  if (T != 1 || n_prior >= 0 || N < 1 || topk > fd::kSelCap) return false;
+  if (fp4_keys)  // bulk copies of the block exponents start on 16-byte boundaries
+    return (d_I == 32 || d_I == 64) && H_I == 4 && N % 16 == 0;
+  return (d_I == 32 || d_I == 64) && (H_I == 4 || H_I == 8);
+}
+
+struct FusedPlan {
+  bool ok;
+  int G, P, stages;
+  int64_t R, per_cta;
+  uint32_t off_sc, off_hist, off_qs, cap;
+  size_t dyn;
+};
+
+// Launch shape for `rows` rows: rows per launch, CTAs, slice length and the
+// shared-memory layout (key ring, the slice's scores, histogram, index
+// query; the candidate list and attention buffers reuse the same bytes).
+FusedPlan plan_fused(int64_t rows, int64_t N, int32_t d_I, int32_t H_I, int32_t D, int32_t topk,
+                     size_t static_smem, int sms, int blocks_per_sm, size_t tile) {
+  FusedPlan pl{};
+  const size_t maxdyn = size_t(232448) - static_smem - 1024;
+  const size_t aw = size_t(fd::kAttnWarps) * (D == 128 ? sizeof(ar::WarpArea<128>)
+                                                        : sizeof(ar::WarpArea<64>));
+  const int gmax = std::min(sms * std::max(blocks_per_sm, 0), fd::kMaxG);
+  for (int64_t R = std::min<int64_t>(rows, std::max(1, gmax / 4)); R >= 1; R = R / 2) {
+    const int64_t tot = R * N;
+    int G = (int)std::min<int64_t>(gmax, std::max<int64_t>(16 * R, ceil_div(tot, 4096)));
+    if (G < R) continue;
+    const int64_t per = align_up(size_t(ceil_div(tot, G)), 16);
+    G = (int)ceil_div(tot, per);  // no empty slices
+    const int P = std::min<int>(kFusedMaxP, G / (int)R);
+    if (P < 1 || ceil_div(topk, P) > fd::kSelCap) continue;
+    const size_t sc = align_up(size_t(per) * 4, 128);
+    const size_t fixed = sc + size_t(kBins1) * 4 + align_up(size_t(H_I) * d_I, 128);
+    if (fixed + 2 * tile > maxdyn) continue;
+    const int stages = (int)std::min<size_t>(4, (maxdyn - fixed) / tile);
+    const size_t dyn_a = stages * tile + fixed;
+    size_t dyn = std::max(dyn_a, aw);
+    dyn = std::max(dyn, size_t(4096) * 8 + size_t(kBins2) * 4);
+    if (dyn > maxdyn) continue;
+    pl.ok = true;
+    pl.G = G;
+    pl.P = P;
+    pl.stages = stages;
+    pl.R = R;
+    pl.per_cta = per;
+    pl.off_sc = (uint32_t)(stages * tile);
+    pl.off_hist = (uint32_t)(pl.off_sc + sc);
+    pl.off_qs = (uint32_t)(pl.off_hist + size_t(kBins1) * 4);
+    pl.cap = (uint32_t)((dyn - size_t(kBins2) * 4) / 8);
+    pl.dyn = dyn;
+    return pl;
+  }
+  return pl;
+}
+
+template <int DI, int HI, int D, int KF>
+csa2_status run_fused_t(const fd::Params &base, int64_t rows, cudaStream_t st, void *ws,
+                        size_t ws_bytes) {
+  auto kern = fd::decode_fused_kernel<DI, HI, D, KF>;
+  const size_t tile = fd::Shape<DI, HI, KF>::TILE_BYTES;
+  static size_t static_smem[256] = {0};
+  static int bps[256] = {0};
+  int dev = 0;
+  cudaGetDevice(&dev);
+  if (dev < 0 || dev >= 256) return CSA2_ERR_CUDA;
+  if (!bps[dev]) {
+    cudaFuncAttributes fa{};
+    if (cudaFuncGetAttributes(&fa, kern) != cudaSuccess) return CSA2_ERR_CUDA;
+    const size_t mx = size_t(232448) - fa.sharedSizeBytes - 1024;
+    if (set_smem_attr(kern, mx, false) != CSA2_OK) return CSA2_ERR_CUDA;
+    int nb = 0;
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&nb, kern, fd::kThreads, mx) !=
+        cudaSuccess)
+      return CSA2_ERR_CUDA;
+    static_smem[dev] = fa.sharedSizeBytes;
+    bps[dev] = nb > 0 ? nb : -1;
+  }
+  if (bps[dev] < 1) return CSA2_ERR_UNSUPPORTED;
+  const FusedPlan pl = plan_fused(rows, base.N, DI, HI, D, base.topk, static_smem[dev],
+                                  device_sms(), bps[dev], tile);
+  if (!pl.ok) return CSA2_ERR_UNSUPPORTED;
+  const FusedWs L = fused_ws_layout(ws, pl.R, base.N);
+  if (!ws || ws_bytes < L.bytes) return CSA2_ERR_WORKSPACE;
+  for (int64_t row0 = 0; row0 < rows;) {
+    // a launch of q.R rows; the last ones may take fewer rows, with a plan
+    // of their own that never holds more rows than the workspace layout
+    const int64_t nr = std::min<int64_t>(pl.R, rows - row0);
+    const FusedPlan q = nr == pl.R ? pl
+                                   : plan_fused(nr, base.N, DI, HI, D, base.topk,
+                                                static_smem[dev], device_sms(), bps[dev], tile);
+    if (!q.ok || q.R > nr) return CSA2_ERR_UNSUPPORTED;
+    if (cudaMemsetAsync(L.hist1, 0, L.sync_bytes, st) != cudaSuccess) return CSA2_ERR_CUDA;
+    fd::Params p = base;
+    p.R = (int32_t)q.R;
+    p.row0 = row0;
+    row0 += q.R;
+    p.per_cta = q.per_cta;
+    p.hist1 = L.hist1;
+    p.arrive = L.arrive;
+    p.cnt = L.cnt;
+    p.cand = L.cand;
+    p.part = L.part;
+    p.off_sc = q.off_sc;
+    p.off_hist = q.off_hist;
+    p.off_qs = q.off_qs;
+    p.cap = q.cap;
+    p.stages = q.stages;
+    p.p_att = q.P;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)q.G, 1, 1);
+    cfg.blockDim = dim3(fd::kThreads, 1, 1);
+    cfg.dynamicSmemBytes = q.dyn;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeCooperative;
+    attr[0].val.cooperative = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    TraceScope ts(p.do_attn ? "decode_fused" : "decode_fused_topk", st);
+    if (cudaLaunchKernelEx(&cfg, kern, p) != cudaSuccess) return CSA2_ERR_CUDA;
+  }
+  return CSA2_OK;
+}
+
+using FusedRun = csa2_status (*)(const fd::Params &, int64_t, cudaStream_t, void *, size_t);
+
+FusedRun pick_fused(int32_t d_I, int32_t H_I, int32_t D, bool fp4_keys) {
+#define CSA2_FD_CASE(DI, HI, KF)                                                  \
+  if (d_I == DI && H_I == HI)                                                     \
+    return D == 128 ? &run_fused_t<DI, HI, 128, KF> : &run_fused_t<DI, HI, 64, KF>;
+  if (fp4_keys) {
+    CSA2_FD_CASE(32, 4, fd::kKeysFp4) CSA2_FD_CASE(64, 4, fd::kKeysFp4)
+    return nullptr;
+  }
+  CSA2_FD_CASE(32, 4, fd::kKeysInt8) CSA2_FD_CASE(32, 8, fd::kKeysInt8)
+  CSA2_FD_CASE(64, 4, fd::kKeysInt8) CSA2_FD_CASE(64, 8, fd::kKeysInt8)
+#undef CSA2_FD_CASE
+  return nullptr;
+}
+
 // Index + top-k (and, when `att` is given, the layer's attention fused into
 // the same per-row cluster kernel), in passes of R rows.
-csa2_status run_index_topk(const int8_t *q_idx, const float *w, const int8_t *k_idx, int32_t B,
-                           int32_t T, int32_t H_I, int32_t d_I, int64_t N, int64_t n_prior,
-                           int32_t ratio, int32_t topk, int32_t *idx_out, float *score_out,
-                           const AttnArgs *att, void *ws, size_t ws_bytes, cudaStream_t st) {
+// k_exps: NULL for int8 index keys; else the keys are FP4 (k_idx holds the
+// codes) and only the fused decode kernel serves the call.
+csa2_status run_index_topk(const int8_t *q_idx, const float *w, const int8_t *k_idx,
+                           const uint8_t *k_exps, int32_t B, int32_t T, int32_t H_I, int32_t d_I,
+                           int64_t N, int64_t n_prior, int32_t ratio, int32_t topk,
+                           int32_t *idx_out, float *score_out, const AttnArgs *att, void *ws,
+                           size_t ws_bytes, cudaStream_t st) {
   const int64_t rows = int64_t(B) * T;
+  const bool fp4 = k_exps != nullptr;
+  if ((fused_enabled() || fp4) && score_out == nullptr &&
+      fused_shape_ok(T, H_I, d_I, N, n_prior, topk, fp4) &&
+      (!att || (att->H <= fd::kHeads && (att->D == 64 || att->D == 128)))) {
+    const FusedRun run = pick_fused(d_I, H_I, att ? att->D : 64, fp4);
+    if (run) {
+      fd::Params p{};
+      p.q_idx = q_idx;
+      p.w = w;
+      p.k_idx = k_idx;
+      p.k_exps = k_exps;
+      p.N = N;
+      p.topk = topk;
+      p.idx = idx_out;
+      if (att) {
+        p.do_attn = 1;
+        p.q = att->q;
+        p.codes = att->codes;
+        p.scales = att->scales;
+        p.win_k = att->win_k;
+        p.win_v = att->win_v;
+        p.H = att->H;
+        p.W = att->W;
+        p.q_scale = att->sm_scale * 1.4426950408889634f;
+        p.out = att->out;
+        p.lse = att->lse;
+      }
+      const csa2_status rc = run(p, rows, st, ws, ws_bytes);
+      if (rc != CSA2_ERR_UNSUPPORTED || fp4) return rc;  // else the general path below
+    }
+  }
+  if (fp4) return CSA2_ERR_UNSUPPORTED;
   if (pf_eligible(T, H_I, d_I, N, topk, score_out)) {
     const int64_t Rp = pf_rows_per_pass(T, N, d_I);
     const PfWs Lp0 = pf_ws_layout(nullptr, Rp, N, d_I);
@@ -1070,6 +1308,24 @@ csa2_status csa2_pack_fp4(const float *src, int64_t rows, int32_t D, uint8_t *co
   return after_launch();
 }
 
+csa2_status csa2_append_entry(const float *src, const int8_t *key, const int64_t *pos, int32_t B,
+                              int32_t D, int32_t d_I, int64_t N, uint8_t *codes, float *scales,
+                              int8_t *k_idx, void *stream) {
+  if (B < 0 || D <= 0 || D % 16 != 0 || d_I <= 0 || d_I % 16 != 0 || N < 0)
+    return CSA2_ERR_INVALID_ARG;
+  if (B == 0) return CSA2_OK;
+  if (!src || !key || !pos || (N > 0 && (!codes || !scales || !k_idx)) || !aligned(src, 16) ||
+      !aligned(key, 16) || !aligned(pos, 8) || (codes && !aligned(codes, 8)) ||
+      (scales && !aligned(scales, 4)) || (k_idx && !aligned(k_idx, 16)))
+    return CSA2_ERR_INVALID_ARG;
+  const int64_t units = int64_t(B) * (D / 16 + d_I / 16);
+  const int64_t blocks = std::min<int64_t>(ceil_div(units, 128), int64_t(device_sms()) * 8);
+  TraceScope ts("append_entry", as_stream(stream));
+  append_entry_kernel<<<(unsigned)blocks, 128, 0, as_stream(stream)>>>(src, key, pos, B, D, d_I,
+                                                                      N, codes, scales, k_idx);
+  return after_launch();
+}
+
 csa2_status csa2_unpack_fp4(const uint8_t *codes, const float *scales, int64_t rows, int32_t D,
                             float *out, void *stream) {
   if (rows < 0 || D <= 0 || D % 16 != 0) return CSA2_ERR_INVALID_ARG;
@@ -1088,6 +1344,8 @@ size_t csa2_index_topk_workspace_size(int32_t B, int32_t T, int32_t H_I, int32_t
   if (B < 0 || T < 0 || N < 0 || topk < 1 || !scan_shape_supported(H_I, d_I)) return 0;
   size_t bytes = topk_ws_bytes(B, T, N);
   if (pf_shape_ok(T, H_I, d_I, N, topk)) bytes = std::max(bytes, pf_ws_bytes(T, N, d_I));
+  if (fused_shape_ok(T, H_I, d_I, N, -1, topk))
+    bytes = std::max(bytes, fused_ws_bytes(int64_t(B) * T, N));
   return bytes;
 }
 
@@ -1098,8 +1356,43 @@ csa2_status csa2_index_topk(const int8_t *q_idx, const float *w, const int8_t *k
   csa2_status rc = check_topk_args(q_idx, w, k_idx, B, T, H_I, d_I, N, n_prior, ratio, topk,
                                    idx_out, score_out);
   if (rc != CSA2_OK || int64_t(B) * T == 0) return rc;
-  return run_index_topk(q_idx, w, k_idx, B, T, H_I, d_I, N, n_prior, ratio, topk, idx_out,
-                        score_out, nullptr, ws, ws_bytes, as_stream(stream));
+  return run_index_topk(q_idx, w, k_idx, nullptr, B, T, H_I, d_I, N, n_prior, ratio, topk,
+                        idx_out, score_out, nullptr, ws, ws_bytes, as_stream(stream));
+}
+
+csa2_status csa2_pack_index_keys_fp4(const float *src, int64_t rows, int32_t d_I,
+                                     uint8_t *codes, uint8_t *exps, void *stream) {
+  if (rows < 0 || d_I <= 0 || d_I % 32 != 0) return CSA2_ERR_INVALID_ARG;
+  if (rows == 0) return CSA2_OK;
+  if (!src || !codes || !exps || !aligned(src, 16) || !aligned(codes, 16))
+    return CSA2_ERR_INVALID_ARG;
+  const int64_t blocks = rows * (d_I / 32);
+  const int64_t grid = std::min<int64_t>(ceil_div(blocks, 256), int64_t(device_sms()) * 16);
+  TraceScope ts("pack_keys_fp4", as_stream(stream));
+  pack_keys_fp4_kernel<<<(unsigned)grid, 256, 0, as_stream(stream)>>>(src, blocks, codes, exps);
+  return after_launch();
+}
+
+size_t csa2_index_topk_fp4k_workspace_size(int32_t B, int32_t H_I, int32_t d_I, int64_t N,
+                                           int32_t topk) {
+  if (B < 0 || topk < 1 || !fused_shape_ok(1, H_I, d_I, N, -1, topk, true)) return 0;
+  return fused_ws_bytes(B, N);
+}
+
+csa2_status csa2_index_topk_fp4k(const int8_t *q_idx, const float *w, const uint8_t *k_codes,
+                                 const uint8_t *k_exps, int32_t B, int32_t H_I, int32_t d_I,
+                                 int64_t N, int32_t topk, int32_t *idx_out, void *ws,
+                                 size_t ws_bytes, void *stream) {
+  if (B < 0 || N < 0 || topk < 1 || H_I < 1 || d_I < 1 || d_I % 32 != 0)
+    return CSA2_ERR_INVALID_ARG;
+  if (!fused_shape_ok(1, H_I, d_I, N, -1, topk, true)) return CSA2_ERR_UNSUPPORTED;
+  if (B == 0) return CSA2_OK;
+  if (!q_idx || !w || !k_codes || !k_exps || !idx_out || !aligned(q_idx, 16) ||
+      !aligned(k_codes, 16) || !aligned(k_exps, 16) || !aligned(w, 4) || !aligned(idx_out, 4))
+    return CSA2_ERR_INVALID_ARG;
+  return run_index_topk(q_idx, w, reinterpret_cast<const int8_t *>(k_codes), k_exps, B, 1, H_I,
+                        d_I, N, -1, 4, topk, idx_out, nullptr, nullptr, ws, ws_bytes,
+                        as_stream(stream));
 }
 
 size_t csa2_index_pool_workspace_size(int32_t B, int32_t H_I, int32_t d_I, int64_t N,
@@ -1227,6 +1520,15 @@ csa2_status check_layers(const csa2_layer_mode *modes, const csa2_layer_io *io, 
       rc = check_topk_args(x.q_idx, x.w, kv.k_idx, d->B, d->T, d->H_I, d->d_I, d->N, d->n_prior,
                            d->ratio, d->topk, x.idx, nullptr);
       if (rc != CSA2_OK) return rc;
+      if (kv.k_exps && (!aligned(kv.k_exps, 16) ||
+                        !fused_shape_ok(d->T, d->H_I, d->d_I, d->N, d->n_prior, d->topk, true) ||
+                        d->H > fd::kHeads))
+        return kv.k_exps && !aligned(kv.k_exps, 16) ? CSA2_ERR_INVALID_ARG : CSA2_ERR_UNSUPPORTED;
+    }
+    if (modes[l].mode == CSA2_FULL && x.app_pos) {
+      if (!x.app_src || !x.app_key || x.k_exps || !aligned(x.app_src, 16) ||
+          !aligned(x.app_key, 16) || !aligned(x.app_pos, 8) || d->d_I % 16 != 0)
+        return CSA2_ERR_INVALID_ARG;
     }
     rc = check_attn_args(x.q, kv.codes, kv.scales, ix.idx, x.win_k, x.win_v, d->B, d->T, d->H,
                          d->D, d->N, d->topk, d->W, x.out, x.lse);
@@ -1243,10 +1545,19 @@ csa2_status run_layer(const csa2_layer_mode *modes, const csa2_layer_io *io, int
   if (modes[l].mode != CSA2_REUSE) {
     // Full / Reindex: scan this layer's index query over the kv store's keys,
     // then select and attend in one per-row cluster kernel.
+    if (modes[l].mode == CSA2_FULL && x.app_pos) {  // this step's entry append first
+      const int64_t units = int64_t(d->B) * (d->D / 16 + d->d_I / 16);
+      TraceScope ts("append_entry", st);
+      append_entry_kernel<<<(unsigned)std::min<int64_t>(ceil_div(units, 128), 1024), 128, 0, st>>>(
+          x.app_src, x.app_key, x.app_pos, d->B, d->D, d->d_I, d->N,
+          const_cast<uint8_t *>(x.codes), const_cast<float *>(x.scales),
+          const_cast<int8_t *>(x.k_idx));
+      if (after_launch() != CSA2_OK) return CSA2_ERR_CUDA;
+    }
     AttnArgs att{x.q, kv.codes, kv.scales, x.win_k, x.win_v, d->H, d->D, d->W, d->sm_scale,
                  x.out, x.lse};
-    return run_index_topk(x.q_idx, x.w, kv.k_idx, d->B, d->T, d->H_I, d->d_I, d->N, d->n_prior,
-                          d->ratio, d->topk, x.idx, nullptr, &att, ws, ws_bytes, st);
+    return run_index_topk(x.q_idx, x.w, kv.k_idx, kv.k_exps, d->B, d->T, d->H_I, d->d_I, d->N,
+                          d->n_prior, d->ratio, d->topk, x.idx, nullptr, &att, ws, ws_bytes, st);
   }
   // Reuse: attend with the source layer's selection.
   return run_attn(x.q, kv.codes, kv.scales, ix.idx, x.win_k, x.win_v, d->B, d->T, d->H, d->D,
@@ -1354,8 +1665,14 @@ csa2_status csa2_index_topk_noalloc(const int8_t *q_idx, const float *w, const i
     return CSA2_ERR_UNSUPPORTED;
   void *ws = noalloc_scratch(&rc);
   if (!ws) return rc;
-  return run_index_topk(q_idx, w, k_idx, B, T, H_I, d_I, N, n_prior, ratio, topk, idx_out,
-                        score_out, nullptr, ws, kNoAllocScratchBytes, as_stream(stream));
+  return run_index_topk(q_idx, w, k_idx, nullptr, B, T, H_I, d_I, N, n_prior, ratio, topk,
+                        idx_out, score_out, nullptr, ws, kNoAllocScratchBytes, as_stream(stream));
+}
+
+csa2_status csa2_wait_timeout_selftest(int64_t limit_cycles, void *stream) {
+  if (limit_cycles < 1 || limit_cycles > (int64_t(1) << 32)) return CSA2_ERR_INVALID_ARG;
+  fd::wait_timeout_selftest_kernel<<<1, 32, 0, as_stream(stream)>>>((long long)limit_cycles);
+  return after_launch();
 }
 
 csa2_status csa2_get_device_status(void *stream, int32_t *code_out) {

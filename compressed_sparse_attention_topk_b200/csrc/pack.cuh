@@ -20,6 +20,32 @@ __device__ __forceinline__ uint32_t e2m1_mag_code(float y) {
          (uint32_t)(y > 5.0f);
 }
 
+// The FP4 codes (two words) and scale of one group of 16 fp32 values.
+__device__ __forceinline__ void pack_group16(const float (&x)[16], uint2 &code, float &scale) {
+  float amax = 0.0f;
+#pragma unroll
+  for (int i = 0; i < 16; ++i) {
+    const float a = fabsf(x[i]);
+    if (a > amax) amax = a;
+  }
+  const float s = __fdiv_rn(amax, 6.0f);
+  uint32_t lo = 0, hi = 0;
+  if (s > 0.0f) {
+#pragma unroll
+    for (int i = 0; i < 16; ++i) {
+      const float y = __fdiv_rn(x[i], s);
+      uint32_t c = e2m1_mag_code(fabsf(y));
+      if (c != 0u && x[i] < 0.0f) c |= 8u;
+      if (i < 8)
+        lo |= c << (4 * i);
+      else
+        hi |= c << (4 * (i - 8));
+    }
+  }
+  code = make_uint2(lo, hi);
+  scale = s;
+}
+
 // One thread per group of 16 elements.
 __global__ void __launch_bounds__(256) pack_fp4_kernel(const float *__restrict__ src,
                                                        int64_t groups,
@@ -37,29 +63,147 @@ __global__ void __launch_bounds__(256) pack_fp4_kernel(const float *__restrict__
       x[4 * i + 2] = v.z;
       x[4 * i + 3] = v.w;
     }
-    float amax = 0.0f;
-#pragma unroll
-    for (int i = 0; i < 16; ++i) {
-      float a = fabsf(x[i]);
-      if (a > amax) amax = a;
-    }
-    const float s = __fdiv_rn(amax, 6.0f);
-    uint32_t lo = 0, hi = 0;
-    if (s > 0.0f) {
-#pragma unroll
-      for (int i = 0; i < 16; ++i) {
-        const float y = __fdiv_rn(x[i], s);
-        uint32_t c = e2m1_mag_code(fabsf(y));
-        if (c != 0u && x[i] < 0.0f) c |= 8u;
-        if (i < 8)
-          lo |= c << (4 * i);
-        else
-          hi |= c << (4 * (i - 8));
-      }
-    }
-    reinterpret_cast<uint2 *>(codes)[g] = make_uint2(lo, hi);
+    uint2 code;
+    float s;
+    pack_group16(x, code, s);
+    reinterpret_cast<uint2 *>(codes)[g] = code;
     scales[g] = s;
   }
+}
+
+// Entry append ("DeepSeek-V4.1-Flash", section "Fast memory, persistent
+// storage and recomputation": the main cache entries are stored in FP4;
+// "Inference-Efficient LLMs", section 6: per-group scaling): one decode
+// step writes each sequence's completed entry into row pos[b] of its store
+// -- the FP4 codes and scales of src[b] (the rule of pack_fp4_kernel) and
+// the int8 index key key[b] -- and nothing for a sequence with pos[b] < 0.
+// A position >= N is recorded as a bad index and skipped.  One thread per
+// 16-element group of an entry or 16-byte piece of a key.
+__global__ void __launch_bounds__(128) append_entry_kernel(
+    const float *__restrict__ src, const int8_t *__restrict__ key, const int64_t *__restrict__ pos,
+    int32_t B, int32_t D, int32_t d_I, int64_t N, uint8_t *__restrict__ codes,
+    float *__restrict__ scales, int8_t *__restrict__ k_idx) {
+  const int G = D / 16, KP = d_I / 16;  // groups and key pieces per sequence
+  const int64_t total = (int64_t)B * (G + KP);
+  for (int64_t u = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; u < total;
+       u += (int64_t)gridDim.x * blockDim.x) {
+    const int64_t b = u / (G + KP);
+    const int q = (int)(u % (G + KP));
+    const int64_t n = pos[b];
+    if (n < 0) continue;
+    if (n >= N) {
+      if (q == 0) raise_status(kStatusBadIndex);
+      continue;
+    }
+    const int64_t row = b * N + n;
+    if (q < G) {
+      const float4 *p = reinterpret_cast<const float4 *>(src + b * D + 16 * q);
+      float x[16];
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        const float4 v = p[i];
+        x[4 * i + 0] = v.x;
+        x[4 * i + 1] = v.y;
+        x[4 * i + 2] = v.z;
+        x[4 * i + 3] = v.w;
+      }
+      uint2 code;
+      float s;
+      pack_group16(x, code, s);
+      reinterpret_cast<uint2 *>(codes + row * (D / 2))[q] = code;
+      scales[row * G + q] = s;
+    } else {
+      const int k = q - G;
+      reinterpret_cast<int4 *>(k_idx + row * d_I)[k] =
+          reinterpret_cast<const int4 *>(key + b * d_I)[k];
+    }
+  }
+}
+
+// ---------------------------------------------------------------------------
+// FP4 index keys ("Inference-Efficient LLMs", section 6: FP4 in parts of the
+// attention indexing machinery).  This library's reading: E2M1 elements with
+// one power-of-two scale per block of 32 elements, kept as an 8-bit biased
+// exponent (the OCP Microscaling MXFP4 block format).  Per block: shared
+// exponent s = floor(log2(amax)) - 2 (2 = the largest E2M1 exponent),
+// clamped to [-127, 127], stored as s + 127; each element's code is the
+// E2M1 value nearest to x / 2^s (IEEE divide; ties to the even code,
+// saturating at 6; a zero magnitude is code 0); an all-zero block stores
+// exponent byte 0 and zero codes.  Element 2i is the low nibble of byte i.
+// ---------------------------------------------------------------------------
+
+// floor(log2(a)) of a finite a > 0, from its bits.
+__device__ __forceinline__ int floor_log2_pos(float a) {
+  const uint32_t u = __float_as_uint(a);
+  const int e = (int)((u >> 23) & 0xffu);
+  if (e != 0) return e - 127;
+  return (31 - __clz((int)(u & 0x7fffffu))) - 149;  // subnormal: mantissa * 2^-149
+}
+
+// 2^e as fp32 for -149 <= e <= 127 (exact).
+__device__ __forceinline__ float pow2_f32(int e) {
+  return e >= -126 ? __uint_as_float((uint32_t)(e + 127) << 23)
+                   : __uint_as_float(1u << (e + 149));
+}
+
+// One thread per block of 32 elements: codes [blocks, 16] bytes, exps [blocks].
+__global__ void __launch_bounds__(256) pack_keys_fp4_kernel(const float *__restrict__ src,
+                                                            int64_t blocks,
+                                                            uint8_t *__restrict__ codes,
+                                                            uint8_t *__restrict__ exps) {
+  for (int64_t g = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; g < blocks;
+       g += (int64_t)gridDim.x * blockDim.x) {
+    const float4 *p = reinterpret_cast<const float4 *>(src + g * 32);
+    float x[32];
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      const float4 v = p[i];
+      x[4 * i + 0] = v.x;
+      x[4 * i + 1] = v.y;
+      x[4 * i + 2] = v.z;
+      x[4 * i + 3] = v.w;
+    }
+    float amax = 0.0f;
+#pragma unroll
+    for (int i = 0; i < 32; ++i) amax = fmaxf(amax, fabsf(x[i]));
+    uint32_t w[4] = {0u, 0u, 0u, 0u};
+    uint8_t eb = 0;
+    if (amax > 0.0f) {
+      int s = floor_log2_pos(amax) - 2;
+      s = s < -127 ? -127 : (s > 127 ? 127 : s);
+      eb = (uint8_t)(s + 127);
+      const float X = pow2_f32(s);
+#pragma unroll
+      for (int i = 0; i < 32; ++i) {
+        const float y = __fdiv_rn(x[i], X);
+        uint32_t c = e2m1_mag_code(fabsf(y));
+        if (c != 0u && x[i] < 0.0f) c |= 8u;
+        w[i >> 3] |= c << (4 * (i & 7));
+      }
+    }
+    reinterpret_cast<uint4 *>(codes)[g] = make_uint4(w[0], w[1], w[2], w[3]);
+    exps[g] = eb;
+  }
+}
+
+// Eight E2M1 codes (one word, element order) -> two words of four int8
+// values, each twice the E2M1 value (an integer in {0, +-1, +-2, +-3, +-4,
+// +-6, +-8, +-12}), element order: byte permutes from a magnitude table and
+// its negation, chosen per byte by the code's sign bit (replicated into a
+// byte mask by the permute's sign mode).
+__device__ __forceinline__ uint32_t prmt(uint32_t a, uint32_t b, uint32_t sel) {
+  uint32_t d;
+  asm("prmt.b32 %0, %1, %2, %3;" : "=r"(d) : "r"(a), "r"(b), "r"(sel));
+  return d;
+}
+__device__ __forceinline__ void e2m1x8_to_i8x8(uint32_t w, uint32_t &lo, uint32_t &hi) {
+  constexpr uint32_t kPos0 = 0x03020100u, kPos1 = 0x0C080604u;  // 0 1 2 3 | 4 6 8 12
+  constexpr uint32_t kNeg0 = 0xFDFEFF00u, kNeg1 = 0xF4F8FAFCu;  // their negations
+  const uint32_t a = w << 4;  // even elements' sign bits to their byte's top bit
+  const uint32_t sl = w & 0x7777u, sh = (w >> 16) & 0x7777u;
+  const uint32_t ml = prmt(a, w, 0xD9C8u), mh = prmt(a, w, 0xFBEAu);  // 0xFF where negative
+  lo = (prmt(kPos0, kPos1, sl) & ~ml) | (prmt(kNeg0, kNeg1, sl) & ml);
+  hi = (prmt(kPos0, kPos1, sh) & ~mh) | (prmt(kNeg0, kNeg1, sh) & mh);
 }
 
 // Four E2M1 codes pairs (one 32-bit word = 8 codes) -> 8 fp32 values times a

@@ -89,7 +89,7 @@ MTP5 = Workload("mtp5_decode_1m_b4_n262144", B=4, T=5, H=16, D=128, N=262144, H_
 ALL = {w.name: w for w in (TINY, DECODE, GROUP, LONG, PREFILL, MTP5)}
 
 _TENSOR_IDS = {"entries": 1, "k_idx": 2, "q_idx": 3, "w": 4, "q": 5, "win_k": 6, "win_v": 7,
-               "outliers": 8}
+               "outliers": 8, "key_src": 9, "app_src": 10, "app_key": 11}
 
 
 def rng_for(seed: int, tensor: str, layer: int = 0) -> np.random.Generator:
@@ -156,3 +156,21 @@ def all_layer_inputs(wl: Workload, B: Optional[int] = None) -> List[dict]:
 def with_sizes(wl: Workload, **kw) -> Workload:
     """A copy of a workload with some sizes changed (smaller parity cases)."""
     return dataclasses.replace(wl, **kw)
+
+
+def index_key_sources(wl: Workload, layer: int = 0, B: Optional[int] = None) -> np.ndarray:
+    """fp32 [B, N, d_I] N(0,1) sources of a store's index keys, for stores that
+    keep them in FP4 (each side packs them on its own)."""
+    B = wl.B if B is None else B
+    return rng_for(wl.seed, "key_src", layer).standard_normal((B, wl.N, wl.d_I),
+                                                              dtype=np.float32)
+
+
+def append_inputs(wl: Workload, step: int = 0, B: Optional[int] = None) -> dict:
+    """One decode step's completed entries: fp32 [B, D] N(0,1) entry values
+    and int8 [B, d_I] uniform index keys (the compressor's and the indexer
+    key projection's outputs, which this library does not model)."""
+    B = wl.B if B is None else B
+    return {"src": rng_for(wl.seed, "app_src", step).standard_normal((B, wl.D),
+                                                                     dtype=np.float32),
+            "key": int8_uniform(rng_for(wl.seed, "app_key", step), (B, wl.d_I))}

@@ -102,6 +102,29 @@ int32_t csa2_version(void);
 csa2_status csa2_pack_fp4(const float *src, int64_t rows, int32_t D, uint8_t *codes,
                           float *scales, void *stream);
 
+/* Entry append: the per-token write side of the cache.  When a decode
+ * token completes a compressed entry, the entry is stored in FP4 ("DeepSeek-
+ * V4.1-Flash" visual explainer, section "Fast memory, persistent storage and
+ * recomputation"; "Inference-Efficient LLMs", section 6: FP4 with per-group
+ * scaling) in the next row of its sequence's store, with its int8 index key
+ * beside it.  For each sequence b with pos[b] >= 0: src[b] is packed with
+ * the rule of csa2_pack_fp4 into row pos[b] of codes/scales, and key[b] is
+ * copied into row pos[b] of k_idx; a sequence with pos[b] < 0 appends
+ * nothing.  A position >= N is skipped and recorded in the device status
+ * word (bit 0).  The entry values and the key come from the model (the
+ * compressor and the indexer's key projection), which this library does
+ * not hold.
+ *   src    device, fp32 [B, D]      (16-byte aligned)
+ *   key    device, int8 [B, d_I]    (16-byte aligned)
+ *   pos    device, int64 [B]
+ *   codes  device, uint8 [B, N, D/2]   (updated)
+ *   scales device, fp32 [B, N, D/16]   (updated)
+ *   k_idx  device, int8 [B, N, d_I]    (updated)
+ *   D % 16 == 0, d_I % 16 == 0. */
+csa2_status csa2_append_entry(const float *src, const int8_t *key, const int64_t *pos, int32_t B,
+                              int32_t D, int32_t d_I, int64_t N, uint8_t *codes, float *scales,
+                              int8_t *k_idx, void *stream);
+
 /* Dequantise: out[r, i] = E2M1(code[r, i]) * scale[r, i / 16] (one fp32
  * multiply).  codes device uint8 [rows, D/2]; scales device fp32 [rows,
  * D/16]; out device fp32 [rows, D]. */
@@ -168,6 +191,48 @@ csa2_status csa2_index_topk_noalloc(const int8_t *q_idx, const float *w, const i
                                     int32_t B, int32_t T, int32_t H_I, int32_t d_I, int64_t N,
                                     int64_t n_prior, int32_t ratio, int32_t topk,
                                     int32_t *idx_out, float *score_out, void *stream);
+
+/* ---------------------------------------------------------------------- */
+/* FP4 index keys                                                          */
+/* ---------------------------------------------------------------------- */
+
+/* "Inference-Efficient LLMs", section 6: V4 already used FP4 for parts of
+ * its attention indexing machinery.  This library's reading for the index
+ * keys: E2M1 elements with one power-of-two scale per block of 32 elements,
+ * stored as an 8-bit biased exponent (the OCP Microscaling MXFP4 block
+ * format), so a key of d_I elements takes d_I/2 + d_I/32 bytes (34 for
+ * d_I = 64, against 64 as int8).  Per block: s = floor(log2(amax)) - 2,
+ * clamped to [-127, 127], exponent byte s + 127; each element's code is the
+ * E2M1 value nearest to x / 2^s (IEEE divide, ties to the even code,
+ * saturating at 6; zero magnitude is code 0); an all-zero block stores
+ * exponent byte 0 and zero codes; element 2i is the low nibble of byte i.
+ *   src   device, fp32 [rows, d_I]
+ *   codes device, uint8 [rows, d_I/2]   (output, 16-byte aligned)
+ *   exps  device, uint8 [rows, d_I/32]  (output)
+ *   d_I % 32 == 0. */
+csa2_status csa2_pack_index_keys_fp4(const float *src, int64_t rows, int32_t d_I,
+                                     uint8_t *codes, uint8_t *exps, void *stream);
+
+/* Workspace bytes for csa2_index_topk_fp4k (0 on unsupported sizes). */
+size_t csa2_index_topk_fp4k_workspace_size(int32_t B, int32_t H_I, int32_t d_I, int64_t N,
+                                           int32_t topk);
+
+/* Index score + Top-K over FP4 keys, decode rows (one query per sequence,
+ * every entry visible).  Score of entry n (this library's reading): per
+ * head h and key block g the exact integer idot = sum over the block of
+ * q_idx[b,h,i] * (2 * E2M1(code_i)); the head's dot is the fp32 sum over the
+ * blocks in ascending order of idot * 2^(exp_g - 128) (each multiply and add
+ * rounded on its own); the heads are combined with their weights exactly as
+ * in csa2_index_topk.  Selection as in csa2_index_topk.
+ *   q_idx   device, int8 [B, H_I, d_I];  w device, fp32 [B, H_I]
+ *   k_codes device, uint8 [B, N, d_I/2]; k_exps device, uint8 [B, N, d_I/32]
+ *   idx_out device, int32 [B, topk]   (output)
+ *   ws      device workspace of ws_bytes >= csa2_index_topk_fp4k_workspace_size
+ * Supported: d_I in {32, 64}, H_I == 4, N % 16 == 0, N >= 1, topk <= 4096. */
+csa2_status csa2_index_topk_fp4k(const int8_t *q_idx, const float *w, const uint8_t *k_codes,
+                                 const uint8_t *k_exps, int32_t B, int32_t H_I, int32_t d_I,
+                                 int64_t N, int32_t topk, int32_t *idx_out, void *ws,
+                                 size_t ws_bytes, void *stream);
 
 /* ---------------------------------------------------------------------- */
 /* Hierarchical indexer: a Full layer's candidate pool, a Reindex layer's  */
@@ -302,6 +367,21 @@ typedef struct csa2_layer_io {
     int32_t *idx;
     float *out;
     float *lse;
+    /* Optional, read for a Full layer's store: index keys in FP4 (see
+     * csa2_pack_index_keys_fp4) instead of int8 -- k_idx then points at the
+     * FP4 codes [B, N, d_I/2] and k_exps at the block exponents [B, N,
+     * d_I/32].  NULL: int8 keys.  Layers over FP4 keys need the decode shape
+     * of csa2_index_topk_fp4k and H <= 16. */
+    const uint8_t *k_exps;
+    /* Optional, Full layers with int8 keys: this step's entry append
+     * (csa2_append_entry) into the layer's own store before its index scan,
+     * so a completed entry is visible to the same step's query.  app_src fp32
+     * [B, D], app_key int8 [B, d_I], app_pos int64 [B] (device); NULL app_pos
+     * = no append.  With app_pos set, the layer's codes, scales and k_idx
+     * are written. */
+    const float *app_src;
+    const int8_t *app_key;
+    const int64_t *app_pos;
 } csa2_layer_io;
 
 /* CSA2_OK when the table follows the rules of csa2_layer_mode. */
@@ -356,6 +436,16 @@ csa2_status csa2_trace_get(int32_t i, const char **name, float *ms);
 /* ---------------------------------------------------------------------- */
 /* Device status                                                           */
 /* ---------------------------------------------------------------------- */
+
+/* Self-test of the library's bounded waits (every wait on a pipeline
+ * barrier, on another CTA's delivery or on another CTA's counter gives up
+ * after a limit, records bit 1 in the device status word and lets the
+ * kernel finish).  Launches one thread that waits, with a limit of
+ * limit_cycles SM cycles (1 .. 2^32), on a barrier phase that never
+ * completes and on a counter that nothing raises: afterwards
+ * csa2_get_device_status reports bit 1 and the device keeps working.  The
+ * pages describe no such call; it exists for tests. */
+csa2_status csa2_wait_timeout_selftest(int64_t limit_cycles, void *stream);
 
 /* Synchronise `stream`, then read and clear the current device's status
  * word.  *code_out (may be NULL) receives the raw word: 0 = clean, bit 0 =

@@ -89,6 +89,13 @@ def _check_index(q, w, k, topk, n_prior=-1, ratio=4, rows=None, check_scores=Tru
         if rows is not None:
             g_sc = g_sc[rows]
         assert_bits_equal(g_sc, o_sc, "scores")
+        # the same call without a score output: with one query per sequence
+        # this takes the fused decode kernel (scores stay on chip)
+        g2 = host(csa2.index_topk(dev(q), dev(w), dev(k), topk, n_prior, ratio))
+        g2 = g2.reshape(B * T, topk)
+        if rows is not None:
+            g2 = g2[rows]
+        assert_bits_equal(g2, o_idx, "indices without score output")
     assert_bits_equal(g_idx, o_idx, "indices")
     return g_idx
 
@@ -135,6 +142,27 @@ def test_topk_candidate_lists_many_slices(N):
     # one row: the scan splits it into up to ~2 slices per SM, each emitting a list
     q, w, k = _index_case(1, 1, 4, 64, N, seed=N)
     _check_index(q, w, k, 2048)
+
+
+def test_topk_all_equal_scores_beyond_on_chip_list():
+    # every entry is a candidate: the list of a row exceeds what a CTA keeps
+    # in shared memory, so the exact selection reads it from L2
+    q, w, k = _index_case(2, 1, 4, 64, 60000, seed=4, q_zero=True)
+    idx = _check_index(q, w, k, 300)
+    assert np.array_equal(idx, np.tile(np.arange(300, dtype=np.int32), (2, 1)))
+
+
+def test_topk_heavy_ties_fused_shapes():
+    q, w, k = _index_case(4, 1, 4, 32, 20000, seed=8, key_levels=1)
+    w[:] = 1.0
+    _check_index(q, w, k, 1000)
+
+
+def test_topk_more_rows_than_one_launch():
+    # 40 sequences: more rows than one fused launch takes (about a quarter of
+    # the SMs), so the rows go in several launches
+    q, w, k = _index_case(40, 1, 4, 64, 3000, seed=40)
+    _check_index(q, w, k, 256)
 
 
 def test_topk_empty_store():
@@ -416,6 +444,53 @@ def _run_group_and_compare(w0, rows=None):
         assert_close(lse, ref[l]["lse"], f"layer {l} lse")
     assert csa2.get_device_status() == 0
     return tens
+
+
+@pytest.mark.parametrize("B,N,topk,W,H,D,H_I,d_I", [
+    (2, 5000, 2048, 128, 16, 128, 4, 64),
+    (3, 1000, 2048, 128, 16, 128, 4, 64),     # fewer entries than k: padding
+    (1, 3000, 100, 0, 16, 128, 4, 64),        # no window
+    (2, 7777, 512, 1, 5, 64, 8, 32),          # one window row, 5 heads
+    (5, 20000, 4096, 70, 16, 128, 8, 64),
+    (2, 100, 7, 128, 16, 128, 4, 32),
+])
+def test_decode_layer_shapes(B, N, topk, W, H, D, H_I, d_I):
+    """Full + Reindex decode layers through the layer call (fused decode
+    kernel): selection bit-exact, attention within tolerance."""
+    w0 = wl.with_sizes(wl.LONG, name=f"decode_{B}_{N}_{topk}", B=B, N=N, topk=topk, W=W, H=H,
+                       D=D, H_I=H_I, d_I=d_I, seed=B * 1000 + N)
+    _run_group_and_compare(w0)
+
+
+def test_decode_layer_cuda_graph_replay():
+    """The layer call captured into a CUDA graph (as the benchmark runs it)
+    and replayed gives the eager results, bit for bit, on every replay."""
+    w0 = wl.with_sizes(wl.LONG, name="graph_replay", B=4, N=20000, seed=77)
+    layers = wl.all_layer_inputs(w0)
+    tens = _group_tensors(w0, layers)
+    dims = csa2.make_dims(w0.B, w0.T, w0.H, w0.D, w0.N, w0.H_I, w0.d_I, w0.topk, w0.W)
+    group = csa2.LayerGroup(list(w0.modes), tens, dims)
+    group.run()
+    torch.cuda.synchronize()
+    eager = [(t["idx"].clone(), t["out"].clone(), t["lse"].clone()) for t in tens]
+    for t in tens:
+        t["idx"].fill_(-5)
+        t["out"].fill_(7.0)
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        group.run()
+    for _ in range(2):
+        for t in tens:
+            t["idx"].fill_(-5)
+            t["out"].fill_(7.0)
+        g.replay()
+        torch.cuda.synchronize()
+        for (i0, o0, l0), t in zip(eager, tens):
+            assert torch.equal(t["idx"], i0)
+            assert torch.equal(t["out"], o0)
+            assert torch.equal(t["lse"], l0)
+    del g
+    assert csa2.get_device_status() == 0
 
 
 def test_group_workload_16_layers():
