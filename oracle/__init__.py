@@ -26,6 +26,10 @@ _LIB_PATH = os.path.join(_HERE, "liboracle.so")
 
 OK, EINVAL, ENOMEM, ERANGE = 0, 1, 2, 3
 FULL, REINDEX, REUSE = 0, 1, 2
+# A Reindex layer that searches only its Full source's candidate pool
+# ("Inference-Efficient LLMs", section 5: later Reindex layers search within
+# the pool an earlier Full layer kept).  Same table rules as REINDEX.
+REINDEX_POOL = 3
 
 
 def build(force: bool = False) -> str:
@@ -315,7 +319,8 @@ def group_cache_bytes(modes, entries, numbers_per_entry, bits_per_number) -> int
     return int(out[0])
 
 
-def layer_group(modes, layers, topk, n_prior=-1, ratio=4, sm_scale=None, rows=None):
+def layer_group(modes, layers, topk, n_prior=-1, ratio=4, sm_scale=None, rows=None,
+                pool=None):
     """Walk a mode table in layer order.
 
     ``layers[l]`` is a dict with the layer's own ``q``, ``q_idx``, ``w``,
@@ -323,18 +328,35 @@ def layer_group(modes, layers, topk, n_prior=-1, ratio=4, sm_scale=None, rows=No
     ``codes``, ``scales``, ``k_idx``.  Per layer the entry store is that of
     layer kv_src and the selection is computed (Full, Reindex: own index
     query over the store's index keys) or taken from layer idx_src (Reuse).
+    A REINDEX_POOL layer (decode rows only; ``pool`` = (block, n_blocks))
+    scores only the candidate pool of its kv_src Full layer -- the n_blocks
+    best blocks of `block` positions by the Full layer's own index scores
+    (``block_pool``) -- with its own index query and keeps their top-k
+    (``pool_topk``).
     Returns a list of dicts with ``idx``, ``out``, ``lse`` and ``store`` (the
     layer id whose entries were read).
     """
     m = _c(modes, np.int32).reshape(-1, 3)
-    if not validate_modes(m):
+    checked = m.copy()
+    checked[checked[:, 0] == REINDEX_POOL, 0] = REINDEX  # the same table rules
+    if not validate_modes(checked):
         raise OracleError("invalid mode table")
     results = []
     for l, (mode, kv_src, idx_src) in enumerate(m.tolist()):
         lay = layers[l]
         store = layers[kv_src]
         B, T = lay["q"].shape[:2]
-        if mode in (FULL, REINDEX):
+        if mode == REINDEX_POOL:
+            if pool is None or n_prior >= 0 or T != 1 or rows is not None:
+                raise OracleError("a pool layer needs pool=(block, n_blocks) and decode rows")
+            block, n_blocks = pool
+            idx = np.empty((B, 1, topk), np.int32)
+            for b in range(B):
+                full = index_score_row(store["q_idx"][b, 0], store["w"][b, 0], store["k_idx"][b])
+                cand = block_pool(full, block, n_blocks)
+                idx[b, 0] = pool_topk(lay["q_idx"][b, 0], lay["w"][b, 0], store["k_idx"][b],
+                                      cand, topk)
+        elif mode in (FULL, REINDEX):
             sel = index_topk(lay["q_idx"], lay["w"], store["k_idx"], topk, n_prior, ratio,
                              rows=rows)
             if rows is None:

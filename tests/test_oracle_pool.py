@@ -113,3 +113,50 @@ def test_pool_topk_rejects_positions_outside_the_store():
     keys = np.ones((10, 16), np.int8)
     with pytest.raises(Exception):
         oracle.pool_topk(q, w, keys, np.array([3, 10], np.int32), 2)
+
+
+# ---------------------------------------------------------------------------
+# The mode-table walk with a Reindex layer that searches its Full source's
+# pool (oracle.REINDEX_POOL).
+# ---------------------------------------------------------------------------
+
+def _pool_group(B=2, N=3000, topk=64, seed=3):
+    from compressed_sparse_attention_topk_b200 import workloads as wl
+    w0 = wl.with_sizes(wl.LONG, name="pool_walk", B=B, N=N, topk=topk, seed=seed)
+    layers = wl.all_layer_inputs(w0)
+    c, s_ = oracle.pack_fp4(layers[0]["entries"].reshape(B * N, -1))
+    layers[0]["codes"], layers[0]["scales"] = c.reshape(B, N, -1), s_.reshape(B, N, -1)
+    return w0, layers
+
+
+def test_pool_layer_with_a_pool_covering_the_store_equals_reindex():
+    w0, layers = _pool_group()
+    plain = oracle.layer_group([(0, 0, 0), (1, 0, 1)], layers, w0.topk)
+    pooled = oracle.layer_group([(0, 0, 0), (oracle.REINDEX_POOL, 0, 1)], layers, w0.topk,
+                                pool=(8, (w0.N + 7) // 8))
+    assert np.array_equal(pooled[1]["idx"], plain[1]["idx"])
+    assert np.array_equal(pooled[1]["out"], plain[1]["out"])
+    assert np.array_equal(pooled[0]["idx"], plain[0]["idx"])
+
+
+def test_pool_layer_selects_within_the_full_layers_best_blocks():
+    w0, layers = _pool_group(N=5000, topk=100, seed=4)
+    block, n_blocks = 8, 40
+    res = oracle.layer_group([(0, 0, 0), (oracle.REINDEX_POOL, 0, 1), (2, 0, 1)], layers + [
+        dict(layers[1])], w0.topk, pool=(block, n_blocks))
+    for b in range(w0.B):
+        full = oracle.index_score_row(layers[0]["q_idx"][b, 0], layers[0]["w"][b, 0],
+                                      layers[0]["k_idx"][b])
+        # the kept blocks: the n_blocks largest block maxima (no ties here)
+        bmax = full.reshape(-1, block).max(axis=1)
+        kept = set(np.argsort(-bmax, kind="stable")[:n_blocks].tolist())
+        sel = res[1]["idx"][b, 0]
+        assert all(int(n) // block in kept for n in sel if n >= 0)
+        # within the pool the selection is the exact top-k of the layer's own scores
+        mine = oracle.index_score_row(layers[1]["q_idx"][b, 0], layers[1]["w"][b, 0],
+                                      layers[0]["k_idx"][b])
+        pool = [n for n in range(w0.N) if n // block in kept]
+        best = sorted(pool, key=lambda n: (-float(mine[n]), n))[:w0.topk]
+        assert sel.tolist() == sorted(best)
+    # a Reuse layer after it copies its selection
+    assert np.array_equal(res[2]["idx"], res[1]["idx"])
