@@ -54,6 +54,10 @@ def parse_args():
     ap.add_argument("--keys", default="int8", choices=["int8", "fp4"],
                     help="index key format of the entry stores (fp4: E2M1 with a power-of-two "
                          "scale per 32 elements; a supplementary line)")
+    ap.add_argument("--pool", action="store_true",
+                    help="hierarchical indexer: the Full layer keeps a pool of 2,048 blocks of 8 "
+                         "positions from its scan and the second layer selects within that pool "
+                         "(a supplementary line)")
     ap.add_argument("--append", action="store_true",
                     help="every step first appends one completed entry per sequence (FP4 "
                          "entry + int8 key, at the store's last row) in the Full layer")
@@ -286,6 +290,19 @@ def run_reference(args, w0):
 
 # --------------------------------------------------------------------------- GPU arm
 
+POOL_BLOCK, POOL_BLOCKS = 8, 2048   # the pages' example: 2,048 blocks x 8 = 16,384 candidates
+
+
+def layer_bytes(w0, args, l) -> int:
+    """Algorithmic bytes of layer l for one sequence and token: keys scanned
+    (the whole store, or the Full layer's pool for a pool layer) + gathered
+    entries + window."""
+    ab = algorithmic_bytes(w0, args.keys)
+    if args.pool and w0.modes[l][0] == 3:
+        return POOL_BLOCK * POOL_BLOCKS * w0.d_I + ab["gather"] + ab["window"]
+    return ab["total"]
+
+
 def run_gpu(args, w0):
     import torch
     import compressed_sparse_attention_topk_b200 as csa2
@@ -352,8 +369,12 @@ def run_gpu(args, w0):
     out_keys = ("out", "lse", "idx")
     dev_in, _ = pack_into_one_buffer(tens, in_keys, dev)
     dev_out, _ = pack_into_one_buffer(tens, out_keys, dev)
+    pool_kw = {"pool_block": POOL_BLOCK, "pool_blocks": POOL_BLOCKS} if args.pool else {}
+    if args.pool:
+        tens[0]["pool"] = torch.empty((w0.B, POOL_BLOCK * POOL_BLOCKS), dtype=torch.int32,
+                                      device=dev)
     dims = csa2.make_dims(w0.B, w0.T, w0.H, w0.D, w0.N, w0.H_I, w0.d_I, w0.topk, w0.W,
-                          w0.n_prior, w0.ratio, w0.sm_scale)
+                          w0.n_prior, w0.ratio, w0.sm_scale, **pool_kw)
     group = csa2.LayerGroup(list(w0.modes), tens, dims)
     flush_buf = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
     flush_src = torch.ones(256 << 20, dtype=torch.uint8, device=dev)
@@ -539,7 +560,7 @@ def run_gpu(args, w0):
 
     ab = algorithmic_bytes(w0, args.keys)
     peak, peak_kind = measured_peaks()
-    step_bytes = w0.B * w0.L * ab["total"]
+    step_bytes = w0.B * sum(layer_bytes(w0, args, l) for l in range(w0.L))
     ms_step = total_ms / args.steps
     step_gbs = step_bytes / (ms_step * 1e-3) / 1e9
     # The dominant kernel: one launch per layer does the whole layer (scan,
@@ -570,6 +591,9 @@ def run_gpu(args, w0):
                        "layers": "Full+Reindex" if w0.L == 2 else w0.L, "topk": w0.topk,
                        "H": w0.H, "D": w0.D, "H_I": w0.H_I, "d_I": w0.d_I, "W": w0.W,
                        "index_keys": args.keys, "entry_append_per_step": bool(args.append),
+                       "pool": ({"block": POOL_BLOCK, "blocks": POOL_BLOCKS,
+                                 "second_layer": "Reindex within the Full layer's pool"}
+                                if args.pool else None),
                        "parallelism": f"replicas x{world}",
                        "l2": "flushed before every layer (256 MiB write, then 256 MiB read), flush not timed",
                        "step_algorithmic_bytes": step_bytes,
@@ -668,6 +692,10 @@ def run_prefill(args, w0):
 def main():
     args = parse_args()
     w0 = wl.ALL[args.workload]
+    if args.pool:
+        if w0.modes != ((0, 0, 0), (1, 0, 1)):
+            raise SystemExit("--pool runs the Full + Reindex decode workloads")
+        w0 = wl.with_sizes(w0, modes=((0, 0, 0), (3, 0, 1)))
     if args.impl == "reference":
         if w0.T != 1:
             raise SystemExit("the reference leg times decode workloads")

@@ -23,7 +23,7 @@ LIB_PATH = os.path.join(_PKG, "libcsa2.so")
 
 CSA2_OK, CSA2_ERR_INVALID_ARG, CSA2_ERR_UNSUPPORTED, CSA2_ERR_CUDA = 0, 1, 2, 3
 CSA2_ERR_WORKSPACE, CSA2_ERR_DEVICE_STATUS = 4, 5
-FULL, REINDEX, REUSE = 0, 1, 2
+FULL, REINDEX, REUSE, REINDEX_POOL = 0, 1, 2, 3
 
 EXPORTED = (
     "csa2_status_string", "csa2_version", "csa2_pack_fp4", "csa2_unpack_fp4",
@@ -53,13 +53,14 @@ class Dims(ctypes.Structure):
                 ("D", ctypes.c_int32), ("N", ctypes.c_int64), ("H_I", ctypes.c_int32),
                 ("d_I", ctypes.c_int32), ("topk", ctypes.c_int32), ("W", ctypes.c_int32),
                 ("n_prior", ctypes.c_int64), ("ratio", ctypes.c_int32),
-                ("sm_scale", ctypes.c_float)]
+                ("sm_scale", ctypes.c_float), ("pool_block", ctypes.c_int32),
+                ("pool_blocks", ctypes.c_int32)]
 
 
 class LayerIO(ctypes.Structure):
     _fields_ = [(n, ctypes.c_void_p) for n in (
         "q", "q_idx", "w", "win_k", "win_v", "codes", "scales", "k_idx", "idx", "out", "lse",
-        "k_exps", "app_src", "app_key", "app_pos")]
+        "k_exps", "app_src", "app_key", "app_pos", "pool")]
 
 
 _lib = None
@@ -423,9 +424,10 @@ def group_cache_bytes(modes, entries: int, numbers_per_entry: int, bits_per_numb
     return int(out.value)
 
 
-def make_dims(B, T, H, D, N, H_I, d_I, topk, W, n_prior=-1, ratio=4, sm_scale=None) -> Dims:
+def make_dims(B, T, H, D, N, H_I, d_I, topk, W, n_prior=-1, ratio=4, sm_scale=None,
+              pool_block=0, pool_blocks=0) -> Dims:
     return Dims(B, T, H, D, N, H_I, d_I, topk, W, n_prior, ratio,
-                1.0 / math.sqrt(D) if sm_scale is None else sm_scale)
+                1.0 / math.sqrt(D) if sm_scale is None else sm_scale, pool_block, pool_blocks)
 
 
 def layer_group_workspace_size(dims: Dims) -> int:

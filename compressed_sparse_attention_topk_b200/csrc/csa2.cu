@@ -652,7 +652,7 @@ csa2_status run_attn(const uint16_t *q, const uint8_t *codes, const float *scale
 // The fused decode layer kernel (decode_fused.cuh): decode rows (one query
 // per sequence, every entry visible), no score output.
 // ---------------------------------------------------------------------------
-constexpr int kFusedMaxP = 16;                        // attention CTAs per row
+constexpr int kFusedMaxP = fd::kMaxP;                 // attention CTAs per row
 constexpr int64_t kFusedMaxRows = fd::kMaxG / 4;      // rows per launch (at least 4 CTAs each)
 constexpr int kFusedMaxPartD = 128;
 
@@ -853,14 +853,18 @@ FusedRun pick_fused(int32_t d_I, int32_t H_I, int32_t D, bool fp4_keys) {
 // the same per-row cluster kernel), in passes of R rows.
 // k_exps: NULL for int8 index keys; else the keys are FP4 (k_idx holds the
 // codes) and only the fused decode kernel serves the call.
+// bkey (optional, fused decode kernel only): block maxima of the rows'
+// scores as keys, [B, ceil(N / pool_block)], cleared by the caller.
 csa2_status run_index_topk(const int8_t *q_idx, const float *w, const int8_t *k_idx,
                            const uint8_t *k_exps, int32_t B, int32_t T, int32_t H_I, int32_t d_I,
                            int64_t N, int64_t n_prior, int32_t ratio, int32_t topk,
                            int32_t *idx_out, float *score_out, const AttnArgs *att, void *ws,
-                           size_t ws_bytes, cudaStream_t st) {
+                           size_t ws_bytes, cudaStream_t st, uint32_t *bkey = nullptr,
+                           int32_t pool_block = 0) {
   const int64_t rows = int64_t(B) * T;
   const bool fp4 = k_exps != nullptr;
-  if ((fused_enabled() || fp4) && score_out == nullptr &&
+  const bool need_fused = fp4 || bkey != nullptr;
+  if ((fused_enabled() || need_fused) && score_out == nullptr &&
       fused_shape_ok(T, H_I, d_I, N, n_prior, topk, fp4) &&
       (!att || (att->H <= fd::kHeads && (att->D == 64 || att->D == 128)))) {
     const FusedRun run = pick_fused(d_I, H_I, att ? att->D : 64, fp4);
@@ -870,6 +874,9 @@ csa2_status run_index_topk(const int8_t *q_idx, const float *w, const int8_t *k_
       p.w = w;
       p.k_idx = k_idx;
       p.k_exps = k_exps;
+      p.bkey = bkey;
+      p.pool_block = pool_block;
+      p.n_pool_blocks = bkey ? ceil_div(N, pool_block) : 0;
       p.N = N;
       p.topk = topk;
       p.idx = idx_out;
@@ -887,10 +894,10 @@ csa2_status run_index_topk(const int8_t *q_idx, const float *w, const int8_t *k_
         p.lse = att->lse;
       }
       const csa2_status rc = run(p, rows, st, ws, ws_bytes);
-      if (rc != CSA2_ERR_UNSUPPORTED || fp4) return rc;  // else the general path below
+      if (rc != CSA2_ERR_UNSUPPORTED || need_fused) return rc;  // else the general path below
     }
   }
-  if (fp4) return CSA2_ERR_UNSUPPORTED;
+  if (need_fused) return CSA2_ERR_UNSUPPORTED;
   if (pf_eligible(T, H_I, d_I, N, topk, score_out)) {
     const int64_t Rp = pf_rows_per_pass(T, N, d_I);
     const PfWs Lp0 = pf_ws_layout(nullptr, Rp, N, d_I);
@@ -1250,6 +1257,89 @@ csa2_status run_attn(const uint16_t *q, const uint8_t *codes, const float *scale
 }
 
 // ---------------------------------------------------------------------------
+// Candidate pools kept by Full layers for CSA2_REINDEX_POOL layers: the
+// fused decode kernel leaves each row's block maxima (as score keys); the
+// best pool_blocks blocks are selected by the row kernel's exact top-k and
+// expanded to positions.  Workspace after the fused kernel's.
+// ---------------------------------------------------------------------------
+struct PoolExt {
+  uint32_t *bkey;   // [B, nb] block maxima as keys (cleared before the scan)
+  float *bscores;   // [B, round4(nb)]
+  uint32_t *bhist;  // [B, kHistStride]
+  uint2 *bcand;     // [B, nb] candidate overflow of the block top-k
+  int32_t *bidx;    // [B, pool_blocks]
+  size_t bytes;
+};
+
+bool pool_dims_ok(const csa2_dims *d) {
+  return d->pool_block >= 1 && d->pool_block <= kPoolMaxBlock && d->pool_blocks >= 1 &&
+         int64_t(d->pool_block) * d->pool_blocks <= kPoolMaxLen && d->T == 1 && d->n_prior < 0;
+}
+
+PoolExt pool_ext_layout(void *base, const csa2_dims *d) {
+  PoolExt w{};
+  const int64_t B = d->B, nb = ceil_div(d->N, d->pool_block);
+  size_t off = 0;
+  auto take = [&](size_t bytes) {
+    size_t o = off;
+    off += align_up(bytes, 256);
+    return o;
+  };
+  const size_t o_k = take(size_t(B) * nb * 4);
+  const size_t o_s = take(size_t(B) * ((nb + 3) & ~int64_t(3)) * 4);
+  const size_t o_h = take(size_t(B) * kHistStride * 4);
+  const size_t o_c = take(size_t(B) * nb * 8);
+  const size_t o_i = take(size_t(B) * d->pool_blocks * 4);
+  char *p = static_cast<char *>(base);
+  w.bkey = reinterpret_cast<uint32_t *>(p + o_k);
+  w.bscores = reinterpret_cast<float *>(p + o_s);
+  w.bhist = reinterpret_cast<uint32_t *>(p + o_h);
+  w.bcand = reinterpret_cast<uint2 *>(p + o_c);
+  w.bidx = reinterpret_cast<int32_t *>(p + o_i);
+  w.bytes = off;
+  return w;
+}
+
+// The pool regions start after the largest fused-kernel workspace.
+size_t pool_ext_offset(const csa2_dims *d) {
+  return align_up(fused_ws_bytes(int64_t(d->B) * d->T, d->N), 256);
+}
+
+// After the Full layer's fused launch(es): the best blocks and the pool.
+csa2_status pool_from_block_keys(const PoolExt &X, const csa2_dims *d, int32_t *pool,
+                                 cudaStream_t st) {
+  const int64_t B = d->B, nb = ceil_div(d->N, d->pool_block);
+  const int64_t bstride = (nb + 3) & ~int64_t(3);
+  if (cudaMemsetAsync(X.bhist, 0, size_t(B) * kHistStride * 4, st) != cudaSuccess)
+    return CSA2_ERR_CUDA;
+  {
+    TraceScope ts("pool_block_keys", st);
+    block_keys_to_scores_kernel<<<dim3((unsigned)ceil_div(nb, kPoolThreads), (unsigned)B),
+                                  kPoolThreads, 0, st>>>(X.bkey, nb, X.bscores, bstride, X.bhist);
+    if (after_launch() != CSA2_OK) return CSA2_ERR_CUDA;
+  }
+  RowParams p{};
+  p.scores = X.bscores;
+  p.score_stride = bstride;
+  p.hist1 = X.bhist;
+  p.cand = X.bcand;
+  p.N = nb;
+  p.T = 1;
+  p.n_prior = -1;
+  p.ratio = 1;
+  p.row0 = 0;
+  p.topk = d->pool_blocks;
+  p.idx = X.bidx;
+  p.do_topk = 1;
+  if (launch_row(p, 64, B, st) != CSA2_OK) return CSA2_ERR_CUDA;
+  const int64_t P = int64_t(d->pool_block) * d->pool_blocks;
+  TraceScope ts("pool_expand", st);
+  expand_pool_kernel<<<dim3((unsigned)ceil_div(P, kPoolThreads), (unsigned)B), kPoolThreads, 0,
+                       st>>>(X.bidx, d->pool_blocks, d->pool_block, d->N, pool);
+  return after_launch();
+}
+
+// ---------------------------------------------------------------------------
 // Mode tables.
 // ---------------------------------------------------------------------------
 csa2_status check_modes(const csa2_layer_mode *m, int32_t L) {
@@ -1261,6 +1351,7 @@ csa2_status check_modes(const csa2_layer_mode *m, int32_t L) {
         if (kv != l || ix != l) return CSA2_ERR_INVALID_ARG;
         break;
       case CSA2_REINDEX:
+      case CSA2_REINDEX_POOL:
         if (kv < 0 || kv >= l || m[kv].mode != CSA2_FULL || ix != l) return CSA2_ERR_INVALID_ARG;
         break;
       case CSA2_REUSE:
@@ -1499,7 +1590,15 @@ csa2_status csa2_group_cache_bytes(const csa2_layer_mode *modes, int32_t L, int6
 size_t csa2_layer_group_workspace_size(const csa2_dims *d) {
   if (!d) return 0;
   if (d->B < 0 || d->T < 0 || d->H < 1 || (d->D != 64 && d->D != 128) || d->W < 0) return 0;
-  return csa2_index_topk_workspace_size(d->B, d->T, d->H_I, d->d_I, d->N, d->topk);
+  size_t bytes = csa2_index_topk_workspace_size(d->B, d->T, d->H_I, d->d_I, d->N, d->topk);
+  if (bytes && (d->pool_block || d->pool_blocks)) {
+    if (!pool_dims_ok(d)) return 0;
+    bytes = std::max(bytes, pool_ext_offset(d) + pool_ext_layout(nullptr, d).bytes);
+    const int64_t P = int64_t(d->pool_block) * d->pool_blocks;
+    bytes = std::max(bytes, pool_topk_ws_layout(nullptr, topk_rows_per_pass(d->B, P), d->B, P,
+                                                d->topk).bytes);
+  }
+  return bytes;
 }
 
 }  // extern "C"
@@ -1530,6 +1629,14 @@ csa2_status check_layers(const csa2_layer_mode *modes, const csa2_layer_io *io, 
           !aligned(x.app_key, 16) || !aligned(x.app_pos, 8) || d->d_I % 16 != 0)
         return CSA2_ERR_INVALID_ARG;
     }
+    // a pool layer reads its Full source's pool; that Full layer writes it
+    const bool keeps_pool = modes[l].mode == CSA2_FULL && x.pool;
+    if (modes[l].mode == CSA2_REINDEX_POOL || keeps_pool) {
+      if (!pool_dims_ok(d) || kv.k_exps ||
+          !fused_shape_ok(d->T, d->H_I, d->d_I, d->N, d->n_prior, d->topk))
+        return CSA2_ERR_UNSUPPORTED;
+      if (!kv.pool || !aligned(kv.pool, 4)) return CSA2_ERR_INVALID_ARG;
+    }
     rc = check_attn_args(x.q, kv.codes, kv.scales, ix.idx, x.win_k, x.win_v, d->B, d->T, d->H,
                          d->D, d->N, d->topk, d->W, x.out, x.lse);
     if (rc != CSA2_OK) return rc;
@@ -1542,6 +1649,15 @@ csa2_status run_layer(const csa2_layer_mode *modes, const csa2_layer_io *io, int
   const csa2_layer_io &x = io[l];
   const csa2_layer_io &kv = io[modes[l].kv_src];
   const csa2_layer_io &ix = io[modes[l].idx_src];
+  if (modes[l].mode == CSA2_REINDEX_POOL) {
+    // the top-k within the Full source's pool, then attention with it
+    const int64_t P = int64_t(d->pool_block) * d->pool_blocks;
+    csa2_status rc = run_pool_topk(x.q_idx, x.w, kv.k_idx, d->B, d->H_I, d->d_I, d->N, kv.pool,
+                                   (int32_t)P, d->topk, x.idx, ws, ws_bytes, st);
+    if (rc != CSA2_OK) return rc;
+    return run_attn(x.q, kv.codes, kv.scales, x.idx, x.win_k, x.win_v, d->B, d->T, d->H, d->D,
+                    d->N, d->topk, d->W, d->sm_scale, x.out, x.lse, st);
+  }
   if (modes[l].mode != CSA2_REUSE) {
     // Full / Reindex: scan this layer's index query over the kv store's keys,
     // then select and attend in one per-row cluster kernel.
@@ -1556,6 +1672,19 @@ csa2_status run_layer(const csa2_layer_mode *modes, const csa2_layer_io *io, int
     }
     AttnArgs att{x.q, kv.codes, kv.scales, x.win_k, x.win_v, d->H, d->D, d->W, d->sm_scale,
                  x.out, x.lse};
+    if (modes[l].mode == CSA2_FULL && x.pool) {  // the layer also keeps its candidate pool
+      const size_t off = pool_ext_offset(d);
+      if (ws_bytes < off + pool_ext_layout(nullptr, d).bytes) return CSA2_ERR_WORKSPACE;
+      const PoolExt X = pool_ext_layout(static_cast<char *>(ws) + off, d);
+      if (cudaMemsetAsync(X.bkey, 0, size_t(d->B) * ceil_div(d->N, d->pool_block) * 4, st) !=
+          cudaSuccess)
+        return CSA2_ERR_CUDA;
+      csa2_status rc = run_index_topk(x.q_idx, x.w, kv.k_idx, kv.k_exps, d->B, d->T, d->H_I,
+                                      d->d_I, d->N, d->n_prior, d->ratio, d->topk, x.idx, nullptr,
+                                      &att, ws, off, st, X.bkey, d->pool_block);
+      if (rc != CSA2_OK) return rc;
+      return pool_from_block_keys(X, d, x.pool, st);
+    }
     return run_index_topk(x.q_idx, x.w, kv.k_idx, kv.k_exps, d->B, d->T, d->H_I, d->d_I, d->N,
                           d->n_prior, d->ratio, d->topk, x.idx, nullptr, &att, ws, ws_bytes, st);
   }

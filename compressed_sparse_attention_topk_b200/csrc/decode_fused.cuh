@@ -54,6 +54,7 @@ constexpr int kHeads = 16;         // heads of a query row (the MMAs' M)
 constexpr int kMaxStages = 8;
 constexpr int kMaxG = 512;         // CTAs of a launch (one per SM)
 constexpr int kSelCap = 4096;      // output positions one CTA handles
+constexpr int kMaxP = 16;          // attention CTAs per row at most
 constexpr int kHistStride = kBins1 + 4;
 constexpr int kArrive = 4;         // counters per row: scanned, listed, attended
 
@@ -76,6 +77,12 @@ struct Params {
   uint32_t *cnt;         // [R, G] candidates per slice
   uint2 *cand;           // [R, N] (key, entry) lists, slice c's at its first entry
   float *part;           // [R, p_att, kHeads, D + 4] partial states (m, l, -, -, acc)
+  // optional: block maxima of the rows' scores for a candidate pool
+  // (hierarchical indexer): bkey[rg, j] = the largest score key of positions
+  // [j*pool_block, (j+1)*pool_block) of global row rg (zero at launch)
+  uint32_t *bkey;        // [rows_global, n_pool_blocks] or null
+  int32_t pool_block;
+  int64_t n_pool_blocks;
   // shared-memory layout (bytes)
   uint32_t off_sc, off_hist, off_qs, cap;  // ring at 0; phase-3 buffers alias it
   int32_t stages;
@@ -157,6 +164,17 @@ __device__ __forceinline__ uint32_t key_class(uint32_t k, uint32_t t1, uint32_t 
 // Key formats: int8 index keys, or FP4 index keys (E2M1 codes with one
 // power-of-two scale per 32 elements, pack.cuh).
 constexpr int kKeysInt8 = 0, kKeysFp4 = 1;
+
+// A row's global histogram into shared memory: every thread issues its
+// loads before storing any (one L2 round trip, not one per bin).
+__device__ __forceinline__ void load_hist(uint32_t *dst, const uint32_t *src) {
+  constexpr int PER = kBins1 / kThreads;
+  uint32_t v[PER];
+#pragma unroll
+  for (int u = 0; u < PER; ++u) v[u] = __ldcg(src + threadIdx.x + u * kThreads);
+#pragma unroll
+  for (int u = 0; u < PER; ++u) dst[threadIdx.x + u * kThreads] = v[u];
+}
 
 template <int DI, int HI, int KF>
 struct Shape {
@@ -435,8 +453,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_fused_kernel(const Params 
     row_ctas(r, N, p.per_cta, cf, cl);
     if (tid == 0) wait_count(p.arrive + (int64_t)r * kArrive + 0, (uint32_t)(cl - cf + 1));
     __syncthreads();
-    const uint32_t *g = p.hist1 + (int64_t)r * kHistStride;
-    for (int i = tid; i < kBins1; i += kThreads) hist[i] = __ldcg(g + i);
+    load_hist(hist, p.hist1 + (int64_t)r * kHistStride);
     __syncthreads();
     radix_threshold<kThreads, kBins1>(hist, (uint32_t)K, ss.scratch, ss.thr);
     const uint32_t t1 = ss.thr[0];
@@ -470,6 +487,17 @@ __global__ void __launch_bounds__(kThreads, 1) decode_fused_kernel(const Params 
       count += total;
     }
     if (tid == 0) p.cnt[(int64_t)r * G + c] = count;
+    if (p.bkey) {  // block maxima of this segment (a block may span two slices)
+      const int64_t blk = p.pool_block;
+      uint32_t *brow = p.bkey + (p.row0 + r) * p.n_pool_blocks;
+      for (int64_t jb = s0 / blk + tid; jb * blk < s1; jb += kThreads) {
+        const int64_t a = jb * blk > s0 ? jb * blk : s0;
+        const int64_t e = (jb + 1) * blk < s1 ? (jb + 1) * blk : s1;
+        float m = srow[a - s0];
+        for (int64_t n = a + 1; n < e; ++n) m = fmaxf(m, srow[n - s0]);
+        atomicMax(brow + jb, score_key(m));
+      }
+    }
     arrive_all(p.arrive + (int64_t)r * kArrive + 1);
   }
 
@@ -488,10 +516,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_fused_kernel(const Params 
   if (tid == 0) wait_count(p.arrive + (int64_t)ra * kArrive + 1, (uint32_t)nseg);
   __syncthreads();
   // digit-1 threshold of the row again (from the complete histogram)
-  {
-    const uint32_t *g = p.hist1 + (int64_t)ra * kHistStride;
-    for (int i = tid; i < kBins1; i += kThreads) h2[i] = __ldcg(g + i);
-  }
+  load_hist(h2, p.hist1 + (int64_t)ra * kHistStride);
   // slice counts -> list offsets (one slice per thread; nseg <= kMaxG)
   const uint32_t my_cnt = tid < nseg ? __ldcg(p.cnt + (int64_t)ra * G + cf + tid) : 0u;
   uint32_t Ctot;
@@ -527,16 +552,16 @@ __global__ void __launch_bounds__(kThreads, 1) decode_fused_kernel(const Params 
     const int64_t a = (cs > ra * N ? cs : ra * N) - ra * N;
     return __ldcg(p.cand + (int64_t)ra * N + a + (i - ss.pref[s]));
   };
-  if (in_smem) {
-    for (uint32_t i0 = tid; i0 < Ctot; i0 += 4 * kThreads) {
-      uint2 v[4];
+  if (in_smem) {  // 8 loads in flight per thread and round
+    for (uint32_t i0 = tid; i0 < Ctot; i0 += 8 * kThreads) {
+      uint2 v[8];
 #pragma unroll
-      for (int u = 0; u < 4; ++u) {
-        const uint32_t i = i0 + u * kThreads;
-        if (i < Ctot) v[u] = from_global(i);
+      for (int u = 0; u < 8; ++u) {
+        const uint32_t i = min(i0 + u * kThreads, Ctot - 1);
+        v[u] = from_global(i);
       }
 #pragma unroll
-      for (int u = 0; u < 4; ++u) {
+      for (int u = 0; u < 8; ++u) {
         const uint32_t i = i0 + u * kThreads;
         if (i < Ctot) clist[i] = v[u];
       }
@@ -726,7 +751,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_fused_kernel(const Params 
     const float M = warp_max(l > 0.0f ? m : -INFINITY);
     const float f = (M != -INFINITY && l > 0.0f) ? exp2f(m - M) : 0.0f;
     const float L = warp_sum(l * f);
-    if (lane < P) ss.fac[lane][h] = f;
+    if (lane < kMaxP) ss.fac[lane][h] = lane < P ? f : 0.0f;
     if (lane == 0) {
       ss.mrg_m[h] = M;
       ss.mrg_l[h] = L;
@@ -735,19 +760,29 @@ __global__ void __launch_bounds__(kThreads, 1) decode_fused_kernel(const Params 
     }
   }
   __syncthreads();
-  for (int i = tid; i < nh * D; i += kThreads) {
-    const int h = i / D, e = i % D;
-    float *op = p.out + (rg * p.H + h) * (int64_t)D;
-    if (ss.mrg_m[h] == -INFINITY) {
-      op[e] = 0.0f;
-      continue;
-    }
-    float a = 0.0f;
-    for (int q = 0; q < P; ++q) {
+  // thread -> 4 consecutive dims of one head; the kMaxP partial loads are
+  // issued together (slots past P read partial P-1 with factor 0)
+  for (int i = tid; i < nh * (D / 4); i += kThreads) {
+    const int h = i / (D / 4), e = 4 * (i % (D / 4));
+    float4 v[kMaxP];
+#pragma unroll
+    for (int q = 0; q < kMaxP; ++q)
+      v[q] = __ldcg(reinterpret_cast<const float4 *>(
+          rpart + ((int64_t)min(q, P - 1) * kHeads + h) * (D + 4) + 4 + e));
+    float4 a = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
+#pragma unroll
+    for (int q = 0; q < kMaxP; ++q) {
+      if (q >= P) break;
       const float fq = ss.fac[q][h];
-      if (fq != 0.0f) a = fmaf(__ldcg(rpart + ((int64_t)q * kHeads + h) * (D + 4) + 4 + e), fq, a);
+      a.x = fmaf(v[q].x, fq, a.x);
+      a.y = fmaf(v[q].y, fq, a.y);
+      a.z = fmaf(v[q].z, fq, a.z);
+      a.w = fmaf(v[q].w, fq, a.w);
     }
-    op[e] = a * (1.0f / ss.mrg_l[h]);
+    const bool none = ss.mrg_m[h] == -INFINITY;
+    const float il = none ? 0.0f : 1.0f / ss.mrg_l[h];
+    *reinterpret_cast<float4 *>(p.out + (rg * p.H + h) * (int64_t)D + e) =
+        make_float4(a.x * il, a.y * il, a.z * il, a.w * il);
   }
 }
 

@@ -138,4 +138,26 @@ __global__ void __launch_bounds__(kPoolThreads) map_pool_kernel(
   idx_out[r * topk + j] = pos;
 }
 
+// grid = (ceil(nb / 256), rows).  Block maxima kept as score keys (by the
+// fused decode kernel) -> block scores and their digit-1 histogram, the
+// input of the row kernel's top-k.  bkey [rows, nb]; bscores [rows,
+// bstride]; bhist [rows, kHistStride], zeroed.
+__global__ void __launch_bounds__(kPoolThreads) block_keys_to_scores_kernel(
+    const uint32_t *__restrict__ bkey, int64_t nb, float *__restrict__ bscores, int64_t bstride,
+    uint32_t *__restrict__ bhist) {
+  __shared__ uint32_t sh[kBins1];
+  for (int i = threadIdx.x; i < kBins1; i += kPoolThreads) sh[i] = 0u;
+  __syncthreads();
+  const int64_t r = blockIdx.y;
+  const int64_t j = (int64_t)blockIdx.x * kPoolThreads + threadIdx.x;
+  if (j < nb) {
+    const uint32_t k = bkey[r * nb + j];
+    const float m = __uint_as_float((k & 0x80000000u) ? (k & 0x7fffffffu) : ~k);
+    bscores[r * bstride + j] = m;
+    atomicAdd(&sh[key_d1(k)], 1u);
+  }
+  __syncthreads();
+  flush_hist(sh, bhist + r * kHistStride);
+}
+
 }  // namespace csa2

@@ -63,7 +63,18 @@ typedef enum csa2_status {
  * layers"): Full computes its own entries and its own selection; Reindex
  * shares another layer's entries and makes a fresh selection; Reuse shares
  * both.  Every layer keeps its own queries and its own local window. */
-typedef enum csa2_mode { CSA2_FULL = 0, CSA2_REINDEX = 1, CSA2_REUSE = 2 } csa2_mode;
+typedef enum csa2_mode {
+    CSA2_FULL = 0,
+    CSA2_REINDEX = 1,
+    CSA2_REUSE = 2,
+    /* A Reindex layer that searches only the candidate pool its kv_src Full
+     * layer kept ("Inference-Efficient LLMs", section 5: later Reindex layers
+     * search within the pool an earlier Full layer narrowed the context to;
+     * the pool rule is that of csa2_index_pool, the selection that of
+     * csa2_pool_topk).  Table rules as for CSA2_REINDEX; decode rows only;
+     * the pool shape comes from csa2_dims.pool_block / pool_blocks. */
+    CSA2_REINDEX_POOL = 3
+} csa2_mode;
 
 /* One row of the per-layer mode table.  kv_src: the layer whose entry store
  * (FP4 codes, scales, int8 index keys) this layer reads; idx_src: the layer
@@ -348,6 +359,8 @@ typedef struct csa2_dims {
     int64_t n_prior;         /* -1: decode; >= 0: prefill chunk after n_prior entries */
     int32_t ratio;           /* tokens per entry (prefill visibility) */
     float sm_scale;          /* softmax scale (1/sqrt(D) by convention) */
+    int32_t pool_block;      /* pool layers: positions per block (1..64), else 0 */
+    int32_t pool_blocks;     /* pool layers: blocks kept (pool_block*pool_blocks <= 65536) */
 } csa2_dims;
 
 /* Per-layer device pointers (shapes as in the calls above).  q, q_idx, w,
@@ -382,6 +395,11 @@ typedef struct csa2_layer_io {
     const float *app_src;
     const int8_t *app_key;
     const int64_t *app_pos;
+    /* A Full layer that is the kv_src of a CSA2_REINDEX_POOL layer writes its
+     * candidate pool here: int32 [B, pool_blocks * pool_block], positions
+     * ascending then -1 (csa2_index_pool's layout), from the same scan as its
+     * own selection; the pool layer reads it from its kv_src's entry. */
+    int32_t *pool;
 } csa2_layer_io;
 
 /* CSA2_OK when the table follows the rules of csa2_layer_mode. */

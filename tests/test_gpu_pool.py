@@ -4,6 +4,7 @@ top-k of a Reindex layer within a pool (csa2_pool_topk), bit-exact against
 the oracle's block_pool / pool_topk on the same seeded inputs."""
 import numpy as np
 import pytest
+import torch
 
 import oracle
 import compressed_sparse_attention_topk_b200 as csa2
@@ -131,3 +132,60 @@ def test_pool_topk_entry_beyond_the_store_is_recorded_and_skipped():
     got = host(csa2.pool_topk(dev(q), dev(w), dev(k), dev(pool), 400))
     assert csa2.get_device_status() & 1   # reading clears it
     assert_bits_equal(got, _oracle_pool_topk(q, w, k, pool, 400), "indices")
+
+
+# ---------------------------------------------------------------------------
+# Pool layers in the layer call: a Full layer keeps its candidate pool from
+# the same scan as its own selection, a CSA2_REINDEX_POOL layer selects
+# within it, a Reuse layer takes that selection.
+# ---------------------------------------------------------------------------
+
+def _pool_layers(w0, layers, block, n_blocks):
+    from tests._parity import gpu_store
+    tens = []
+    P = block * n_blocks
+    for lay in layers:
+        d = {k: dev(v) for k, v in lay.items() if k != "entries"}
+        d["q"] = d["q"][:, 0].contiguous()
+        if "entries" in lay:
+            d["codes"], d["scales"] = gpu_store(lay["entries"])
+            d["pool"] = torch.full((w0.B, P), -9, dtype=torch.int32, device="cuda")
+        d["idx"] = torch.empty((w0.B, 1, w0.topk), dtype=torch.int32, device="cuda")
+        d["out"] = torch.empty((w0.B, w0.H, w0.D), dtype=torch.float32, device="cuda")
+        d["lse"] = torch.empty((w0.B, w0.H), dtype=torch.float32, device="cuda")
+        tens.append(d)
+    return tens
+
+
+@pytest.mark.parametrize("B,N,block,n_blocks,topk", [(4, 262144, 8, 2048, 2048),
+                                                     (3, 20001, 8, 300, 512),
+                                                     (2, 5000, 16, 40, 100),
+                                                     (2, 3000, 8, 400, 64)])
+def test_pool_layers_in_the_layer_call(B, N, block, n_blocks, topk):
+    from tests._parity import assert_close, oracle_store
+    w0 = wl.with_sizes(wl.LONG, name=f"pool_layers_{N}", B=B, N=N, topk=topk, seed=N + B,
+                       modes=((0, 0, 0), (csa2.REINDEX_POOL, 0, 1), (2, 0, 1)))
+    layers = wl.all_layer_inputs(w0)
+    tens = _pool_layers(w0, layers, block, n_blocks)
+    dims = csa2.make_dims(B, 1, w0.H, w0.D, N, w0.H_I, w0.d_I, topk, w0.W, pool_block=block,
+                          pool_blocks=n_blocks)
+    csa2.layer_group_run(list(w0.modes), tens, dims)
+    layers[0]["codes"], layers[0]["scales"] = oracle_store(layers[0]["entries"])
+    ref = oracle.layer_group(list(w0.modes), layers, topk, pool=(block, n_blocks))
+    # the Full layer's pool, from the same scan as its own selection
+    for b in range(B):
+        full = oracle.index_score_row(layers[0]["q_idx"][b, 0], layers[0]["w"][b, 0],
+                                      layers[0]["k_idx"][b])
+        want = oracle.block_pool(full, block, n_blocks)
+        got = host(tens[0]["pool"])[b]
+        assert_bits_equal(got[: len(want)], want, "pool")
+        assert np.all(got[len(want):] == -1)
+    for l in range(3):
+        src = w0.modes[l][2]
+        assert_bits_equal(host(tens[src]["idx"]).reshape(B, -1), ref[l]["idx"].reshape(B, -1),
+                          f"layer {l} idx")
+        assert_close(host(tens[l]["out"]).reshape(ref[l]["out"].shape), ref[l]["out"],
+                     f"layer {l} out")
+        assert_close(host(tens[l]["lse"]).reshape(ref[l]["lse"].shape), ref[l]["lse"],
+                     f"layer {l} lse")
+    assert csa2.get_device_status() == 0
