@@ -54,6 +54,9 @@ def parse_args():
     ap.add_argument("--keys", default="int8", choices=["int8", "fp4"],
                     help="index key format of the entry stores (fp4: E2M1 with a power-of-two "
                          "scale per 32 elements; a supplementary line)")
+    ap.add_argument("--decode-kernel", default="scan_cluster", choices=["scan_cluster", "fused"],
+                    help="which kernels serve the decode rows: the index scan + per-row cluster "
+                         "kernel (default) or the fused single-launch kernel")
     ap.add_argument("--pool", action="store_true",
                     help="hierarchical indexer: the Full layer keeps a pool of 2,048 blocks of 8 "
                          "positions from its scan and the second layer selects within that pool "
@@ -319,6 +322,8 @@ def run_gpu(args, w0):
         torch.cuda.set_device(0)
     dev = torch.device("cuda", torch.cuda.current_device())
     csa2.lib()
+    csa2.set_decode_kernel(csa2.DECODE_FUSED if args.decode_kernel == "fused"
+                           else csa2.DECODE_SCAN_CLUSTER)
     stream = torch.cuda.current_stream()
 
     def to_dev(a):
@@ -590,6 +595,7 @@ def run_gpu(args, w0):
             "config": {"workload": w0.name, "B": w0.B, "N": w0.N, "context_tokens": w0.N * 4,
                        "layers": "Full+Reindex" if w0.L == 2 else w0.L, "topk": w0.topk,
                        "H": w0.H, "D": w0.D, "H_I": w0.H_I, "d_I": w0.d_I, "W": w0.W,
+                       "decode_kernel": args.decode_kernel,
                        "index_keys": args.keys, "entry_append_per_step": bool(args.append),
                        "pool": ({"block": POOL_BLOCK, "blocks": POOL_BLOCKS,
                                  "second_layer": "Reindex within the Full layer's pool"}

@@ -34,8 +34,9 @@ EXPORTED = (
     "csa2_layer_run", "csa2_index_topk_noalloc", "csa2_index_pool_workspace_size",
     "csa2_index_pool", "csa2_pool_topk_workspace_size", "csa2_pool_topk", "csa2_append_entry",
     "csa2_pack_index_keys_fp4", "csa2_index_topk_fp4k_workspace_size", "csa2_index_topk_fp4k",
-    "csa2_wait_timeout_selftest",
+    "csa2_wait_timeout_selftest", "csa2_set_decode_kernel", "csa2_get_decode_kernel",
 )
+DECODE_SCAN_CLUSTER, DECODE_FUSED = 0, 1
 
 
 class CSA2Error(RuntimeError):
@@ -106,6 +107,8 @@ def lib() -> ctypes.CDLL:
         "csa2_pool_topk": ([P, P, P, i32, i32, i32, i64, P, i32, i32, P, P, sz, P], i32),
         "csa2_get_device_status": ([P, P], i32),
         "csa2_wait_timeout_selftest": ([i64, P], i32),
+        "csa2_set_decode_kernel": ([i32], i32),
+        "csa2_get_decode_kernel": ([], i32),
         "csa2_trace_enable": ([i32], i32),
         "csa2_trace_count": ([], i32),
         "csa2_trace_get": ([i32, ctypes.POINTER(ctypes.c_char_p), ctypes.POINTER(f32)], i32),
@@ -481,6 +484,16 @@ class LayerGroup:
         _check(lib().csa2_layer_group_run(self.modes, self.io, self.L, ctypes.byref(self.dims),
                                           _ptr(self.ws), self.ws.numel(), _stream()),
                "csa2_layer_group_run")
+
+
+def set_decode_kernel(kernel: int):
+    """DECODE_SCAN_CLUSTER (default) or DECODE_FUSED: which kernels serve
+    decode rows (process-wide)."""
+    _check(lib().csa2_set_decode_kernel(kernel), "csa2_set_decode_kernel")
+
+
+def get_decode_kernel() -> int:
+    return int(lib().csa2_get_decode_kernel())
 
 
 def get_device_status() -> int:

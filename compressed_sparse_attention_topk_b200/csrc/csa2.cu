@@ -159,26 +159,45 @@ csa2_status set_smem_attr(K kernel, size_t bytes, bool big_cluster) {
   return CSA2_OK;
 }
 
+// Index-key format of a scan: int8 keys, or FP4 keys (k_exps != nullptr).
+template <int DI, int HI, int KF>
+void launch_scan_kf(dim3 grid, cudaStream_t st, const int8_t *q_idx, const float *w,
+                    const int8_t *k_idx, const uint8_t *k_exps, int32_t T, int64_t N,
+                    int64_t n_prior, int32_t ratio, int64_t row0, float *scores, int64_t stride,
+                    uint32_t *hist1, int write_masked) {
+  using S = ScanShape<DI, HI, KF>;
+  static bool done[256] = {false};
+  int dev = 0;
+  cudaGetDevice(&dev);
+  if (dev < 0 || dev >= 256 || !done[dev]) {
+    set_smem_attr(index_scan_kernel<DI, HI, KF>, S::SMEM, false);
+    if (dev >= 0 && dev < 256) done[dev] = true;
+  }
+  index_scan_kernel<DI, HI, KF><<<grid, kScanThreads, S::SMEM, st>>>(
+      q_idx, w, k_idx, k_exps, T, N, n_prior, ratio, row0, scores, stride, hist1, write_masked);
+}
+
 template <int DI, int HI>
 void launch_scan(dim3 grid, cudaStream_t st, const int8_t *q_idx, const float *w,
                  const int8_t *k_idx, int32_t T, int64_t N, int64_t n_prior, int32_t ratio,
                  int64_t row0, float *scores, int64_t stride, uint32_t *hist1,
                  int write_masked) {
-  using S = ScanShape<DI, HI>;
-  static bool done[256] = {false};
-  int dev = 0;
-  cudaGetDevice(&dev);
-  if (dev < 0 || dev >= 256 || !done[dev]) {
-    set_smem_attr(index_scan_kernel<DI, HI>, S::SMEM, false);
-    if (dev >= 0 && dev < 256) done[dev] = true;
-  }
-  index_scan_kernel<DI, HI><<<grid, kScanThreads, S::SMEM, st>>>(
-      q_idx, w, k_idx, T, N, n_prior, ratio, row0, scores, stride, hist1, write_masked);
+  launch_scan_kf<DI, HI, kScanKeysInt8>(grid, st, q_idx, w, k_idx, nullptr, T, N, n_prior, ratio,
+                                        row0, scores, stride, hist1, write_masked);
 }
 
 using ScanLaunch = void (*)(dim3, cudaStream_t, const int8_t *, const float *, const int8_t *,
                             int32_t, int64_t, int64_t, int32_t, int64_t, float *, int64_t,
                             uint32_t *, int);
+using ScanLaunchFp4 = void (*)(dim3, cudaStream_t, const int8_t *, const float *, const int8_t *,
+                               const uint8_t *, int32_t, int64_t, int64_t, int32_t, int64_t,
+                               float *, int64_t, uint32_t *, int);
+
+ScanLaunchFp4 pick_scan_fp4(int32_t d_I, int32_t H_I) {
+  if (d_I == 32 && H_I == 4) return &launch_scan_kf<32, 4, kScanKeysFp4>;
+  if (d_I == 64 && H_I == 4) return &launch_scan_kf<64, 4, kScanKeysFp4>;
+  return nullptr;
+}
 
 ScanLaunch pick_scan(int32_t d_I, int32_t H_I) {
 #define CSA2_SCAN_CASE(DI, HI) \
@@ -656,16 +675,19 @@ constexpr int kFusedMaxP = fd::kMaxP;                 // attention CTAs per row
 constexpr int64_t kFusedMaxRows = fd::kMaxG / 4;      // rows per launch (at least 4 CTAs each)
 constexpr int kFusedMaxPartD = 128;
 
-// Which decode kernel serves decode rows: the fused kernel unless the
-// environment sets CSA2_DECODE_KERNEL=cluster (the scan + per-row cluster
-// kernels), read once per process.
+// Which kernels serve decode rows (csa2_set_decode_kernel): the index scan
+// + per-row cluster kernel (default), or the fused single-launch kernel.
+// The environment variable CSA2_DECODE_KERNEL=fused sets the initial choice.
+std::atomic<int> g_decode_kernel{-1};
+
 bool fused_enabled() {
-  static int v = -1;
+  int v = g_decode_kernel.load(std::memory_order_relaxed);
   if (v < 0) {
     const char *e = std::getenv("CSA2_DECODE_KERNEL");
-    v = (e && std::strcmp(e, "cluster") == 0) ? 0 : 1;
+    v = (e && std::strcmp(e, "fused") == 0) ? CSA2_DECODE_FUSED : CSA2_DECODE_SCAN_CLUSTER;
+    g_decode_kernel.store(v, std::memory_order_relaxed);
   }
-  return v == 1;
+  return v == CSA2_DECODE_FUSED;
 }
 
 struct FusedWs {
@@ -706,6 +728,12 @@ size_t fused_ws_bytes(int64_t rows, int64_t N) {
   return fused_ws_layout(nullptr, std::min<int64_t>(rows, kFusedMaxRows), N).bytes;
 }
 
+// FP4 index keys: decode rows, d_I in {32, 64}, H_I == 4, N % 16 == 0 (the
+// bulk copies of the block exponents start on 16-byte boundaries).
+bool fp4_shape_ok(int32_t T, int32_t H_I, int32_t d_I, int64_t N, int64_t n_prior) {
+  return T == 1 && n_prior < 0 && (d_I == 32 || d_I == 64) && H_I == 4 && N >= 1 && N % 16 == 0;
+}
+
 bool fused_shape_ok(int32_t T, int32_t H_I, int32_t d_I, int64_t N, int64_t n_prior,
                     int32_t topk, bool fp4_keys = false) {
   if (T != 1 || n_prior >= 0 || N < 1 || topk > fd::kSelCap) return false;
@@ -716,7 +744,7 @@ bool fused_shape_ok(int32_t T, int32_t H_I, int32_t d_I, int64_t N, int64_t n_pr
 
 struct FusedPlan {
   bool ok;
-  int G, P, stages;
+  int G, P, stages, g_row;
   int64_t R, per_cta;
   uint32_t off_sc, off_hist, off_qs, cap;
   size_t dyn;
@@ -733,13 +761,17 @@ FusedPlan plan_fused(int64_t rows, int64_t N, int32_t d_I, int32_t H_I, int32_t 
                                                         : sizeof(ar::WarpArea<64>));
   const int gmax = std::min(sms * std::max(blocks_per_sm, 0), fd::kMaxG);
   for (int64_t R = std::min<int64_t>(rows, std::max(1, gmax / 4)); R >= 1; R = R / 2) {
+    // g_row CTAs per row, each scanning one slice of the row (slices never
+    // cross rows); at least 16 per row so the attention spreads, at most
+    // what fills the SMs
     const int64_t tot = R * N;
-    int G = (int)std::min<int64_t>(gmax, std::max<int64_t>(16 * R, ceil_div(tot, 4096)));
-    if (G < R) continue;
-    const int64_t per = align_up(size_t(ceil_div(tot, G)), 16);
-    G = (int)ceil_div(tot, per);  // no empty slices
-    const int P = std::min<int>(kFusedMaxP, G / (int)R);
-    if (P < 1 || ceil_div(topk, P) > fd::kSelCap) continue;
+    const int64_t G0 = std::min<int64_t>(gmax, std::max<int64_t>(16 * R, ceil_div(tot, 4096)));
+    const int g_row = (int)(G0 / R);
+    if (g_row < 1) continue;
+    const int64_t per = align_up(size_t(ceil_div(N, g_row)), 16);
+    const int G = g_row * (int)R;
+    const int P = std::min<int>(kFusedMaxP, g_row);
+    if (ceil_div(topk, P) > fd::kSelCap) continue;
     const size_t sc = align_up(size_t(per) * 4, 128);
     const size_t fixed = sc + size_t(kBins1) * 4 + align_up(size_t(H_I) * d_I, 128);
     if (fixed + 2 * tile > maxdyn) continue;
@@ -750,6 +782,7 @@ FusedPlan plan_fused(int64_t rows, int64_t N, int32_t d_I, int32_t H_I, int32_t 
     if (dyn > maxdyn) continue;
     pl.ok = true;
     pl.G = G;
+    pl.g_row = g_row;
     pl.P = P;
     pl.stages = stages;
     pl.R = R;
@@ -806,6 +839,7 @@ csa2_status run_fused_t(const fd::Params &base, int64_t rows, cudaStream_t st, v
     p.row0 = row0;
     row0 += q.R;
     p.per_cta = q.per_cta;
+    p.g_row = q.g_row;
     p.hist1 = L.hist1;
     p.arrive = L.arrive;
     p.cnt = L.cnt;
@@ -853,18 +887,39 @@ FusedRun pick_fused(int32_t d_I, int32_t H_I, int32_t D, bool fp4_keys) {
 // the same per-row cluster kernel), in passes of R rows.
 // k_exps: NULL for int8 index keys; else the keys are FP4 (k_idx holds the
 // codes) and only the fused decode kernel serves the call.
-// bkey (optional, fused decode kernel only): block maxima of the rows'
-// scores as keys, [B, ceil(N / pool_block)], cleared by the caller.
+// A Full layer's candidate pool, kept from the same scan as its selection
+// (decode rows): the best n_blocks blocks of `block` positions by their
+// largest score, expanded to positions.  Scratch regions after the scan's.
+struct PoolExt {
+  uint32_t *bkey;   // [B, nb] block maxima as score keys (fused kernel)
+  float *bscores;   // [B, round4(nb)] block maxima
+  uint32_t *bhist;  // [B, kHistStride] their digit-1 histograms
+  uint2 *bcand;     // [B, nb] candidate overflow of the block top-k
+  int32_t *bidx;    // [B, n_blocks] kept blocks
+  size_t bytes;
+};
+struct PoolReq {
+  int32_t block, n_blocks;
+  int32_t *pool;  // [B, n_blocks * block] output
+  PoolExt X;
+};
+csa2_status pool_select_expand(const PoolExt &X, int64_t B, int64_t N, int32_t block,
+                               int32_t n_blocks, int32_t *pool, cudaStream_t st);
+csa2_status pool_from_block_keys(const PoolExt &X, int64_t B, int64_t N, int32_t block,
+                                 int32_t n_blocks, int32_t *pool, cudaStream_t st);
+
+// k_exps != nullptr: FP4 index keys (k_idx holds the codes); decode rows
+// only.  pr != nullptr: also keep the rows' candidate pool (decode rows).
 csa2_status run_index_topk(const int8_t *q_idx, const float *w, const int8_t *k_idx,
                            const uint8_t *k_exps, int32_t B, int32_t T, int32_t H_I, int32_t d_I,
                            int64_t N, int64_t n_prior, int32_t ratio, int32_t topk,
                            int32_t *idx_out, float *score_out, const AttnArgs *att, void *ws,
-                           size_t ws_bytes, cudaStream_t st, uint32_t *bkey = nullptr,
-                           int32_t pool_block = 0) {
+                           size_t ws_bytes, cudaStream_t st, const PoolReq *pr = nullptr) {
   const int64_t rows = int64_t(B) * T;
   const bool fp4 = k_exps != nullptr;
-  const bool need_fused = fp4 || bkey != nullptr;
-  if ((fused_enabled() || need_fused) && score_out == nullptr &&
+  const bool decode = T == 1 && n_prior < 0;
+  if ((fp4 || pr) && !decode) return CSA2_ERR_UNSUPPORTED;
+  if (fused_enabled() && score_out == nullptr &&
       fused_shape_ok(T, H_I, d_I, N, n_prior, topk, fp4) &&
       (!att || (att->H <= fd::kHeads && (att->D == 64 || att->D == 128)))) {
     const FusedRun run = pick_fused(d_I, H_I, att ? att->D : 64, fp4);
@@ -874,9 +929,14 @@ csa2_status run_index_topk(const int8_t *q_idx, const float *w, const int8_t *k_
       p.w = w;
       p.k_idx = k_idx;
       p.k_exps = k_exps;
-      p.bkey = bkey;
-      p.pool_block = pool_block;
-      p.n_pool_blocks = bkey ? ceil_div(N, pool_block) : 0;
+      if (pr) {
+        const int64_t nb = ceil_div(N, pr->block);
+        if (cudaMemsetAsync(pr->X.bkey, 0, size_t(B) * nb * 4, st) != cudaSuccess)
+          return CSA2_ERR_CUDA;
+        p.bkey = pr->X.bkey;
+        p.pool_block = pr->block;
+        p.n_pool_blocks = nb;
+      }
       p.N = N;
       p.topk = topk;
       p.idx = idx_out;
@@ -893,12 +953,13 @@ csa2_status run_index_topk(const int8_t *q_idx, const float *w, const int8_t *k_
         p.out = att->out;
         p.lse = att->lse;
       }
-      const csa2_status rc = run(p, rows, st, ws, ws_bytes);
-      if (rc != CSA2_ERR_UNSUPPORTED || need_fused) return rc;  // else the general path below
+      csa2_status rc = run(p, rows, st, ws, ws_bytes);
+      if (rc == CSA2_OK && pr)
+        rc = pool_from_block_keys(pr->X, B, N, pr->block, pr->n_blocks, pr->pool, st);
+      if (rc != CSA2_ERR_UNSUPPORTED) return rc;  // else the general path below
     }
   }
-  if (need_fused) return CSA2_ERR_UNSUPPORTED;
-  if (pf_eligible(T, H_I, d_I, N, topk, score_out)) {
+  if (!fp4 && !pr && pf_eligible(T, H_I, d_I, N, topk, score_out)) {
     const int64_t Rp = pf_rows_per_pass(T, N, d_I);
     const PfWs Lp0 = pf_ws_layout(nullptr, Rp, N, d_I);
     if (!ws || ws_bytes < Lp0.bytes || !aligned(ws, 16)) return CSA2_ERR_WORKSPACE;
@@ -915,12 +976,18 @@ csa2_status run_index_topk(const int8_t *q_idx, const float *w, const int8_t *k_
   const TopkWs L0 = topk_ws_layout(nullptr, R0, N);
   if (!ws || ws_bytes < L0.bytes || !aligned(ws, 16)) return CSA2_ERR_WORKSPACE;
   const TopkWs L = topk_ws_layout(ws, R0, N);
-  const ScanLaunch scan = pick_scan(d_I, H_I);
-  if (!scan) return CSA2_ERR_UNSUPPORTED;
+  const ScanLaunch scan = fp4 ? nullptr : pick_scan(d_I, H_I);
+  const ScanLaunchFp4 scan4 = fp4 ? pick_scan_fp4(d_I, H_I) : nullptr;
+  if (!scan && !scan4) return CSA2_ERR_UNSUPPORTED;
+  if (fp4 && N % 16 != 0) return CSA2_ERR_UNSUPPORTED;
   // several rows per sequence: whole sequences per pass, one shared scan each
-  const ScanLaunch scan_group = pick_scan_group(d_I, H_I, T);
+  const ScanLaunch scan_group = fp4 ? nullptr : pick_scan_group(d_I, H_I, T);
   const int64_t R = (scan_group && R0 >= T) ? R0 / T * T : R0;
   const int sms = device_sms();
+  const int64_t nbk = pr ? ceil_div(N, pr->block) : 0;
+  const int64_t bstride = (nbk + 3) & ~int64_t(3);
+  if (pr && cudaMemsetAsync(pr->X.bhist, 0, size_t(B) * kHistStride * 4, st) != cudaSuccess)
+    return CSA2_ERR_CUDA;
 
   for (int64_t row0 = 0; row0 < rows; row0 += R) {
     const int64_t nr = std::min<int64_t>(R, rows - row0);
@@ -937,8 +1004,13 @@ csa2_status run_index_topk(const int8_t *q_idx, const float *w, const int8_t *k_
     const int G = (int)std::min(g_want, g_max);
     {
       TraceScope ts("index_scan", st);
-      (grouped ? scan_group : scan)(dim3(G, (unsigned)units), st, q_idx, w, k_idx, T, N, n_prior,
-                                    ratio, row0, scores, stride, L.hist1, score_out != nullptr);
+      if (scan4)
+        scan4(dim3(G, (unsigned)units), st, q_idx, w, k_idx, k_exps, T, N, n_prior, ratio, row0,
+              scores, stride, L.hist1, score_out != nullptr);
+      else
+        (grouped ? scan_group : scan)(dim3(G, (unsigned)units), st, q_idx, w, k_idx, T, N,
+                                      n_prior, ratio, row0, scores, stride, L.hist1,
+                                      score_out != nullptr);
     }
     if (after_launch() != CSA2_OK) return CSA2_ERR_CUDA;
     RowParams p{};
@@ -970,7 +1042,15 @@ csa2_status run_index_topk(const int8_t *q_idx, const float *w, const int8_t *k_
       D = att->D;
     }
     if (launch_row(p, D, nr, st) != CSA2_OK) return CSA2_ERR_CUDA;
+    if (pr) {  // block maxima of these rows' scores, before the next pass reuses them
+      TraceScope ts("pool_block_max", st);
+      block_max_kernel<<<dim3((unsigned)ceil_div(nbk, kPoolThreads), (unsigned)nr), kPoolThreads,
+                         0, st>>>(scores, stride, N, pr->block, pr->X.bscores + row0 * bstride,
+                                  bstride, pr->X.bhist + row0 * kHistStride);
+      if (after_launch() != CSA2_OK) return CSA2_ERR_CUDA;
+    }
   }
+  if (pr) return pool_select_expand(pr->X, B, N, pr->block, pr->n_blocks, pr->pool, st);
   return CSA2_OK;
 }
 
@@ -1257,28 +1337,19 @@ csa2_status run_attn(const uint16_t *q, const uint8_t *codes, const float *scale
 }
 
 // ---------------------------------------------------------------------------
-// Candidate pools kept by Full layers for CSA2_REINDEX_POOL layers: the
-// fused decode kernel leaves each row's block maxima (as score keys); the
-// best pool_blocks blocks are selected by the row kernel's exact top-k and
-// expanded to positions.  Workspace after the fused kernel's.
+// Candidate pools kept by Full layers for CSA2_REINDEX_POOL layers: block
+// maxima of the Full rows' scores (from the scan's score rows, or left as
+// score keys by the fused kernel), the best pool_blocks blocks by the row
+// kernel's exact top-k, expanded to positions.  Scratch after the scan's.
 // ---------------------------------------------------------------------------
-struct PoolExt {
-  uint32_t *bkey;   // [B, nb] block maxima as keys (cleared before the scan)
-  float *bscores;   // [B, round4(nb)]
-  uint32_t *bhist;  // [B, kHistStride]
-  uint2 *bcand;     // [B, nb] candidate overflow of the block top-k
-  int32_t *bidx;    // [B, pool_blocks]
-  size_t bytes;
-};
-
 bool pool_dims_ok(const csa2_dims *d) {
   return d->pool_block >= 1 && d->pool_block <= kPoolMaxBlock && d->pool_blocks >= 1 &&
          int64_t(d->pool_block) * d->pool_blocks <= kPoolMaxLen && d->T == 1 && d->n_prior < 0;
 }
 
-PoolExt pool_ext_layout(void *base, const csa2_dims *d) {
+PoolExt pool_ext_layout(void *base, int64_t B, int64_t N, int32_t block, int32_t n_blocks) {
   PoolExt w{};
-  const int64_t B = d->B, nb = ceil_div(d->N, d->pool_block);
+  const int64_t nb = ceil_div(N, block);
   size_t off = 0;
   auto take = [&](size_t bytes) {
     size_t o = off;
@@ -1289,7 +1360,7 @@ PoolExt pool_ext_layout(void *base, const csa2_dims *d) {
   const size_t o_s = take(size_t(B) * ((nb + 3) & ~int64_t(3)) * 4);
   const size_t o_h = take(size_t(B) * kHistStride * 4);
   const size_t o_c = take(size_t(B) * nb * 8);
-  const size_t o_i = take(size_t(B) * d->pool_blocks * 4);
+  const size_t o_i = take(size_t(B) * n_blocks * 4);
   char *p = static_cast<char *>(base);
   w.bkey = reinterpret_cast<uint32_t *>(p + o_k);
   w.bscores = reinterpret_cast<float *>(p + o_s);
@@ -1300,27 +1371,21 @@ PoolExt pool_ext_layout(void *base, const csa2_dims *d) {
   return w;
 }
 
-// The pool regions start after the largest fused-kernel workspace.
+// The pool regions start after the largest scan / fused-kernel workspace.
 size_t pool_ext_offset(const csa2_dims *d) {
-  return align_up(fused_ws_bytes(int64_t(d->B) * d->T, d->N), 256);
+  return align_up(std::max(fused_ws_bytes(int64_t(d->B) * d->T, d->N),
+                           topk_ws_bytes(d->B, d->T, d->N)),
+                  256);
 }
 
-// After the Full layer's fused launch(es): the best blocks and the pool.
-csa2_status pool_from_block_keys(const PoolExt &X, const csa2_dims *d, int32_t *pool,
-                                 cudaStream_t st) {
-  const int64_t B = d->B, nb = ceil_div(d->N, d->pool_block);
-  const int64_t bstride = (nb + 3) & ~int64_t(3);
-  if (cudaMemsetAsync(X.bhist, 0, size_t(B) * kHistStride * 4, st) != cudaSuccess)
-    return CSA2_ERR_CUDA;
-  {
-    TraceScope ts("pool_block_keys", st);
-    block_keys_to_scores_kernel<<<dim3((unsigned)ceil_div(nb, kPoolThreads), (unsigned)B),
-                                  kPoolThreads, 0, st>>>(X.bkey, nb, X.bscores, bstride, X.bhist);
-    if (after_launch() != CSA2_OK) return CSA2_ERR_CUDA;
-  }
+// The best n_blocks blocks of each row (block scores and their digit-1
+// histograms in X) -> the pool's positions.
+csa2_status pool_select_expand(const PoolExt &X, int64_t B, int64_t N, int32_t block,
+                               int32_t n_blocks, int32_t *pool, cudaStream_t st) {
+  const int64_t nb = ceil_div(N, block);
   RowParams p{};
   p.scores = X.bscores;
-  p.score_stride = bstride;
+  p.score_stride = (nb + 3) & ~int64_t(3);
   p.hist1 = X.bhist;
   p.cand = X.bcand;
   p.N = nb;
@@ -1328,15 +1393,31 @@ csa2_status pool_from_block_keys(const PoolExt &X, const csa2_dims *d, int32_t *
   p.n_prior = -1;
   p.ratio = 1;
   p.row0 = 0;
-  p.topk = d->pool_blocks;
+  p.topk = n_blocks;
   p.idx = X.bidx;
   p.do_topk = 1;
   if (launch_row(p, 64, B, st) != CSA2_OK) return CSA2_ERR_CUDA;
-  const int64_t P = int64_t(d->pool_block) * d->pool_blocks;
+  const int64_t P = int64_t(block) * n_blocks;
   TraceScope ts("pool_expand", st);
   expand_pool_kernel<<<dim3((unsigned)ceil_div(P, kPoolThreads), (unsigned)B), kPoolThreads, 0,
-                       st>>>(X.bidx, d->pool_blocks, d->pool_block, d->N, pool);
+                       st>>>(X.bidx, n_blocks, block, N, pool);
   return after_launch();
+}
+
+// After the fused kernel: block maxima kept as keys -> block scores -> pool.
+csa2_status pool_from_block_keys(const PoolExt &X, int64_t B, int64_t N, int32_t block,
+                                 int32_t n_blocks, int32_t *pool, cudaStream_t st) {
+  const int64_t nb = ceil_div(N, block);
+  if (cudaMemsetAsync(X.bhist, 0, size_t(B) * kHistStride * 4, st) != cudaSuccess)
+    return CSA2_ERR_CUDA;
+  {
+    TraceScope ts("pool_block_keys", st);
+    block_keys_to_scores_kernel<<<dim3((unsigned)ceil_div(nb, kPoolThreads), (unsigned)B),
+                                  kPoolThreads, 0, st>>>(X.bkey, nb, X.bscores,
+                                                         (nb + 3) & ~int64_t(3), X.bhist);
+    if (after_launch() != CSA2_OK) return CSA2_ERR_CUDA;
+  }
+  return pool_select_expand(X, B, N, block, n_blocks, pool, st);
 }
 
 // ---------------------------------------------------------------------------
@@ -1466,8 +1547,8 @@ csa2_status csa2_pack_index_keys_fp4(const float *src, int64_t rows, int32_t d_I
 
 size_t csa2_index_topk_fp4k_workspace_size(int32_t B, int32_t H_I, int32_t d_I, int64_t N,
                                            int32_t topk) {
-  if (B < 0 || topk < 1 || !fused_shape_ok(1, H_I, d_I, N, -1, topk, true)) return 0;
-  return fused_ws_bytes(B, N);
+  if (B < 0 || topk < 1 || topk > 65536 || !fp4_shape_ok(1, H_I, d_I, N, -1)) return 0;
+  return std::max(fused_ws_bytes(B, N), topk_ws_bytes(B, 1, N));
 }
 
 csa2_status csa2_index_topk_fp4k(const int8_t *q_idx, const float *w, const uint8_t *k_codes,
@@ -1476,7 +1557,7 @@ csa2_status csa2_index_topk_fp4k(const int8_t *q_idx, const float *w, const uint
                                  size_t ws_bytes, void *stream) {
   if (B < 0 || N < 0 || topk < 1 || H_I < 1 || d_I < 1 || d_I % 32 != 0)
     return CSA2_ERR_INVALID_ARG;
-  if (!fused_shape_ok(1, H_I, d_I, N, -1, topk, true)) return CSA2_ERR_UNSUPPORTED;
+  if (topk > 65536 || !fp4_shape_ok(1, H_I, d_I, N, -1)) return CSA2_ERR_UNSUPPORTED;
   if (B == 0) return CSA2_OK;
   if (!q_idx || !w || !k_codes || !k_exps || !idx_out || !aligned(q_idx, 16) ||
       !aligned(k_codes, 16) || !aligned(k_exps, 16) || !aligned(w, 4) || !aligned(idx_out, 4))
@@ -1593,7 +1674,9 @@ size_t csa2_layer_group_workspace_size(const csa2_dims *d) {
   size_t bytes = csa2_index_topk_workspace_size(d->B, d->T, d->H_I, d->d_I, d->N, d->topk);
   if (bytes && (d->pool_block || d->pool_blocks)) {
     if (!pool_dims_ok(d)) return 0;
-    bytes = std::max(bytes, pool_ext_offset(d) + pool_ext_layout(nullptr, d).bytes);
+    bytes = std::max(bytes, pool_ext_offset(d) + pool_ext_layout(nullptr, d->B, d->N,
+                                                                  d->pool_block,
+                                                                  d->pool_blocks).bytes);
     const int64_t P = int64_t(d->pool_block) * d->pool_blocks;
     bytes = std::max(bytes, pool_topk_ws_layout(nullptr, topk_rows_per_pass(d->B, P), d->B, P,
                                                 d->topk).bytes);
@@ -1619,10 +1702,9 @@ csa2_status check_layers(const csa2_layer_mode *modes, const csa2_layer_io *io, 
       rc = check_topk_args(x.q_idx, x.w, kv.k_idx, d->B, d->T, d->H_I, d->d_I, d->N, d->n_prior,
                            d->ratio, d->topk, x.idx, nullptr);
       if (rc != CSA2_OK) return rc;
-      if (kv.k_exps && (!aligned(kv.k_exps, 16) ||
-                        !fused_shape_ok(d->T, d->H_I, d->d_I, d->N, d->n_prior, d->topk, true) ||
-                        d->H > fd::kHeads))
-        return kv.k_exps && !aligned(kv.k_exps, 16) ? CSA2_ERR_INVALID_ARG : CSA2_ERR_UNSUPPORTED;
+      if (kv.k_exps && !aligned(kv.k_exps, 16)) return CSA2_ERR_INVALID_ARG;
+      if (kv.k_exps && !fp4_shape_ok(d->T, d->H_I, d->d_I, d->N, d->n_prior))
+        return CSA2_ERR_UNSUPPORTED;
     }
     if (modes[l].mode == CSA2_FULL && x.app_pos) {
       if (!x.app_src || !x.app_key || x.k_exps || !aligned(x.app_src, 16) ||
@@ -1632,8 +1714,7 @@ csa2_status check_layers(const csa2_layer_mode *modes, const csa2_layer_io *io, 
     // a pool layer reads its Full source's pool; that Full layer writes it
     const bool keeps_pool = modes[l].mode == CSA2_FULL && x.pool;
     if (modes[l].mode == CSA2_REINDEX_POOL || keeps_pool) {
-      if (!pool_dims_ok(d) || kv.k_exps ||
-          !fused_shape_ok(d->T, d->H_I, d->d_I, d->N, d->n_prior, d->topk))
+      if (!pool_dims_ok(d) || kv.k_exps || !scan_shape_supported(d->H_I, d->d_I))
         return CSA2_ERR_UNSUPPORTED;
       if (!kv.pool || !aligned(kv.pool, 4)) return CSA2_ERR_INVALID_ARG;
     }
@@ -1674,16 +1755,14 @@ csa2_status run_layer(const csa2_layer_mode *modes, const csa2_layer_io *io, int
                  x.out, x.lse};
     if (modes[l].mode == CSA2_FULL && x.pool) {  // the layer also keeps its candidate pool
       const size_t off = pool_ext_offset(d);
-      if (ws_bytes < off + pool_ext_layout(nullptr, d).bytes) return CSA2_ERR_WORKSPACE;
-      const PoolExt X = pool_ext_layout(static_cast<char *>(ws) + off, d);
-      if (cudaMemsetAsync(X.bkey, 0, size_t(d->B) * ceil_div(d->N, d->pool_block) * 4, st) !=
-          cudaSuccess)
-        return CSA2_ERR_CUDA;
-      csa2_status rc = run_index_topk(x.q_idx, x.w, kv.k_idx, kv.k_exps, d->B, d->T, d->H_I,
-                                      d->d_I, d->N, d->n_prior, d->ratio, d->topk, x.idx, nullptr,
-                                      &att, ws, off, st, X.bkey, d->pool_block);
-      if (rc != CSA2_OK) return rc;
-      return pool_from_block_keys(X, d, x.pool, st);
+      const PoolExt X0 = pool_ext_layout(nullptr, d->B, d->N, d->pool_block, d->pool_blocks);
+      if (ws_bytes < off + X0.bytes) return CSA2_ERR_WORKSPACE;
+      PoolReq pr{d->pool_block, d->pool_blocks, x.pool,
+                 pool_ext_layout(static_cast<char *>(ws) + off, d->B, d->N, d->pool_block,
+                                 d->pool_blocks)};
+      return run_index_topk(x.q_idx, x.w, kv.k_idx, kv.k_exps, d->B, d->T, d->H_I, d->d_I, d->N,
+                            d->n_prior, d->ratio, d->topk, x.idx, nullptr, &att, ws, off, st,
+                            &pr);
     }
     return run_index_topk(x.q_idx, x.w, kv.k_idx, kv.k_exps, d->B, d->T, d->H_I, d->d_I, d->N,
                           d->n_prior, d->ratio, d->topk, x.idx, nullptr, &att, ws, ws_bytes, st);
@@ -1797,6 +1876,16 @@ csa2_status csa2_index_topk_noalloc(const int8_t *q_idx, const float *w, const i
   return run_index_topk(q_idx, w, k_idx, nullptr, B, T, H_I, d_I, N, n_prior, ratio, topk,
                         idx_out, score_out, nullptr, ws, kNoAllocScratchBytes, as_stream(stream));
 }
+
+csa2_status csa2_set_decode_kernel(int32_t kernel) {
+  if (kernel != CSA2_DECODE_SCAN_CLUSTER && kernel != CSA2_DECODE_FUSED)
+    return CSA2_ERR_INVALID_ARG;
+  g_decode_kernel.store(kernel, std::memory_order_relaxed);
+  return CSA2_OK;
+}
+
+int32_t csa2_get_decode_kernel(void) { return fused_enabled() ? CSA2_DECODE_FUSED
+                                                              : CSA2_DECODE_SCAN_CLUSTER; }
 
 csa2_status csa2_wait_timeout_selftest(int64_t limit_cycles, void *stream) {
   if (limit_cycles < 1 || limit_cycles > (int64_t(1) << 32)) return CSA2_ERR_INVALID_ARG;

@@ -71,6 +71,7 @@ struct Params {
   int32_t topk;
   int32_t *idx;          // [rows_global, topk]
   int64_t per_cta;       // keys per CTA slice (a multiple of 16)
+  int32_t g_row;         // CTAs per row: CTA c scans slice c % g_row of row c / g_row
   // workspace
   uint32_t *hist1;       // [R, kHistStride]  (zero at launch)
   uint32_t *arrive;      // [R, kArrive]      (zero at launch)
@@ -134,20 +135,20 @@ __device__ __forceinline__ uint32_t arrive_all(uint32_t *ctr) {
   return old;
 }
 
-__host__ __device__ __forceinline__ int64_t slice_begin(int64_t c, int64_t per, int64_t total) {
-  const int64_t f = c * per;
-  return f < total ? f : total;
+// Slice s of a row: entries [min(s*per, N), min((s+1)*per, N)).
+__host__ __device__ __forceinline__ int64_t slice_begin(int64_t s, int64_t per, int64_t N) {
+  const int64_t f = s * per;
+  return f < N ? f : N;
 }
 
-// CTAs whose slice holds part of row r: [first, last].
-__device__ __forceinline__ void row_ctas(int64_t r, int64_t N, int64_t per, int &first,
+// CTAs whose slice holds part of row r: [first, last] (the row's first
+// ceil(N / per) CTAs; the rest of its g_row CTAs have empty slices).
+__device__ __forceinline__ void row_ctas(int64_t r, int64_t N, int64_t per, int g_row, int &first,
                                          int &last) {
-  first = (int)((r * N) / per);
-  last = (int)(((r + 1) * N - 1) / per);
+  const int64_t ns = (N + per - 1) / per;
+  first = (int)(r * g_row);
+  last = first + (int)(ns < g_row ? ns : g_row) - 1;
 }
-
-// First CTA of the block of CTAs that serve row r in round 2.
-__device__ __forceinline__ int row_base(int r, int R, int G) { return (int)(((int64_t)r * G) / R); }
 
 // Candidate class against the threshold key (t1, t2, t3): 2 above, 1 equal, 0 below.
 __device__ __forceinline__ uint32_t key_class(uint32_t k, uint32_t t1, uint32_t t2, uint32_t t3,
@@ -225,10 +226,14 @@ __global__ void __launch_bounds__(kThreads, 1) decode_fused_kernel(const Params 
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int c = blockIdx.x, G = gridDim.x;
   const int64_t N = p.N;
-  const int64_t Ktot = (int64_t)p.R * N;
-  const int64_t f0 = slice_begin(c, p.per_cta, Ktot), f1 = slice_begin(c + 1, p.per_cta, Ktot);
-  const int r_lo = f0 < f1 ? (int)(f0 / N) : 0;
-  const int r_hi = f0 < f1 ? (int)((f1 - 1) / N) : -1;  // rows [r_lo, r_hi] hold this slice
+  // this CTA's slice: entries [n0, n1) of row c / g_row, as flattened
+  // positions f = row * N + n (a slice never crosses a row)
+  const int my_row = c / p.g_row;
+  const int64_t my_n0 = slice_begin(c % p.g_row, p.per_cta, N);
+  const int64_t my_n1 = slice_begin(c % p.g_row + 1, p.per_cta, N);
+  const int64_t f0 = (int64_t)my_row * N + my_n0, f1 = (int64_t)my_row * N + my_n1;
+  const int r_lo = f0 < f1 ? my_row : 0;
+  const int r_hi = f0 < f1 ? my_row : -1;  // rows [r_lo, r_hi] hold this slice
   const int64_t K = N < p.topk ? N : p.topk;            // entries selected per row
 
   float *sc = reinterpret_cast<float *>(dsm + p.off_sc);       // this slice's scores
@@ -345,63 +350,13 @@ __global__ void __launch_bounds__(kThreads, 1) decode_fused_kernel(const Params 
     const unsigned char *tile = dsm + (size_t)s * S::TILE_BYTES;
     const int64_t lbase = (int64_t)row * N + n0 - f0;  // local index of the tile's first key
     if constexpr (KF == kKeysFp4) {
-     if (tid < nk) {
-      // per block b (chunk c = b ^ x): exact integer dot of the int8 query
-      // with twice the E2M1 values, times 2^(exponent - 128); blocks summed
-      // in ascending order
-      const unsigned char *kc = tile + tid * S::CB;
-      const unsigned char *ke = tile + TK * S::CB + tid * S::EB;
-      uint32_t ew = 0;
-#pragma unroll
-      for (int b = 0; b < NCH; ++b) ew |= (uint32_t)ke[b] << (8 * b);
-      float term[HI][NCH];
-#pragma unroll
-      for (int cc = 0; cc < NCH; ++cc) {
-        const int blk = cc ^ x;
-        const int4 kv = *reinterpret_cast<const int4 *>(kc + (blk << 4));
-        uint32_t kw[8];
-        e2m1x8_to_i8x8((uint32_t)kv.x, kw[0], kw[1]);
-        e2m1x8_to_i8x8((uint32_t)kv.y, kw[2], kw[3]);
-        e2m1x8_to_i8x8((uint32_t)kv.z, kw[4], kw[5]);
-        e2m1x8_to_i8x8((uint32_t)kv.w, kw[6], kw[7]);
-        const float scale = pow2_f32((int)((ew >> (8 * blk)) & 0xffu) - 128);
-#pragma unroll
-        for (int h = 0; h < HI; ++h) {
-          int4 q0, q1;
-          if constexpr (S::QREG) {
-            q0 = qreg[(h * NCH + cc) * QW + 0];
-            q1 = qreg[(h * NCH + cc) * QW + 1];
-          } else {
-            q0 = reinterpret_cast<const int4 *>(qs)[(h * NCH + blk) * QW + 0];
-            q1 = reinterpret_cast<const int4 *>(qs)[(h * NCH + blk) * QW + 1];
-          }
-          int idot = 0;
-          idot = __dp4a((int)kw[0], q0.x, idot);
-          idot = __dp4a((int)kw[1], q0.y, idot);
-          idot = __dp4a((int)kw[2], q0.z, idot);
-          idot = __dp4a((int)kw[3], q0.w, idot);
-          idot = __dp4a((int)kw[4], q1.x, idot);
-          idot = __dp4a((int)kw[5], q1.y, idot);
-          idot = __dp4a((int)kw[6], q1.z, idot);
-          idot = __dp4a((int)kw[7], q1.w, idot);
-          const float t = __fmul_rn(__int2float_rn(idot), scale);
-#pragma unroll
-          for (int b = 0; b < NCH; ++b)
-            if (b == blk) term[h][b] = t;
-        }
+      if (tid < nk) {
+        const float score = fp4_key_score<NCH, HI, S::QREG>(
+            tile + tid * S::CB, tile + TK * S::CB + tid * S::EB, qreg,
+            reinterpret_cast<const int4 *>(qs), wh, x);
+        sc[lbase + tid] = score;
+        atomicAdd(&hist[key_d1(score_key(score))], 1u);
       }
-      float acc = 0.0f;
-#pragma unroll
-      for (int h = 0; h < HI; ++h) {
-        float dot = 0.0f;
-#pragma unroll
-        for (int b = 0; b < NCH; ++b) dot = __fadd_rn(dot, term[h][b]);
-        acc = __fadd_rn(acc, __fmul_rn(wh[h], dot));
-      }
-      const float score = __fadd_rn(acc, 0.0f);
-      sc[lbase + tid] = score;
-      atomicAdd(&hist[key_d1(score_key(score))], 1u);
-     }
     } else if (tid < nk) {
       const unsigned char *krow = tile + tid * DI;
       int dot[HI];
@@ -450,7 +405,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_fused_kernel(const Params 
   // Per row segment: the digit-1 threshold, then this slice's candidates.
   for (int r = r_lo; r <= r_hi; ++r) {
     int cf, cl;
-    row_ctas(r, N, p.per_cta, cf, cl);
+    row_ctas(r, N, p.per_cta, p.g_row, cf, cl);
     if (tid == 0) wait_count(p.arrive + (int64_t)r * kArrive + 0, (uint32_t)(cl - cf + 1));
     __syncthreads();
     load_hist(hist, p.hist1 + (int64_t)r * kHistStride);
@@ -502,14 +457,13 @@ __global__ void __launch_bounds__(kThreads, 1) decode_fused_kernel(const Params 
   }
 
   // ----------------------------------------------------------- round 2 --
-  int ra = 0;
-  while (ra + 1 < p.R && row_base(ra + 1, p.R, G) <= c) ++ra;
-  const int j = c - row_base(ra, p.R, G);
+  const int ra = my_row;
+  const int j = c % p.g_row;  // attention CTA j of row ra when j < P
   const int P = p.p_att;
   if (j >= P || ra >= p.R) return;
   const int64_t rg = p.row0 + ra;
   int cf, cl;
-  row_ctas(ra, N, p.per_cta, cf, cl);
+  row_ctas(ra, N, p.per_cta, p.g_row, cf, cl);
   const int nseg = cl - cf + 1;
   uint2 *clist = reinterpret_cast<uint2 *>(dsm);                    // candidate list
   uint32_t *h2 = reinterpret_cast<uint32_t *>(dsm + (size_t)p.cap * 8);  // digit-2/3 histogram
@@ -524,8 +478,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_fused_kernel(const Params 
     // clamp: a slice never lists more entries than it holds
     uint32_t v = my_cnt;
     if (tid < nseg) {
-      const int64_t cs = slice_begin(cf + tid, p.per_cta, Ktot), ce = slice_begin(cf + tid + 1, p.per_cta, Ktot);
-      const int64_t a = cs > ra * N ? cs : ra * N, b = ce < (ra + 1) * N ? ce : (ra + 1) * N;
+      const int64_t a = slice_begin(tid, p.per_cta, N), b = slice_begin(tid + 1, p.per_cta, N);
       if ((int64_t)v > b - a) v = (uint32_t)(b - a);
     }
     const uint32_t e = block_excl_scan<kThreads>(v, ss.scratch, Ctot);
@@ -548,8 +501,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_fused_kernel(const Params 
   };
   auto from_global = [&](uint32_t i) -> uint2 {
     const int s = seg_of(i);
-    const int64_t cs = slice_begin(cf + s, p.per_cta, Ktot);
-    const int64_t a = (cs > ra * N ? cs : ra * N) - ra * N;
+    const int64_t a = slice_begin(s, p.per_cta, N);
     return __ldcg(p.cand + (int64_t)ra * N + a + (i - ss.pref[s]));
   };
   if (in_smem) {  // 8 loads in flight per thread and round

@@ -21,6 +21,7 @@
 // global histogram at the end for the top-k selection.
 #pragma once
 #include "common.cuh"
+#include "pack.cuh"
 
 namespace csa2 {
 
@@ -29,16 +30,26 @@ constexpr int kScanThreads = 256;
 // the scan), padded to keep rows 16-byte aligned.
 constexpr int kHistStride = kBins1 + 4;
 
-template <int DI, int HI>
+// Index key formats: int8, or FP4 (E2M1 codes with one power-of-two scale
+// per 32 elements: d_I/2 code bytes + d_I/32 exponent bytes per key, see
+// pack.cuh).
+constexpr int kScanKeysInt8 = 0, kScanKeysFp4 = 1;
+
+template <int DI, int HI, int KF = kScanKeysInt8>
 struct ScanShape {
-  static constexpr int NCH = DI / 16;                     // 16-byte chunks per key
-  static constexpr int KPT = (DI >= 64) ? 1 : 64 / DI;    // keys per thread per tile
+  static constexpr bool FP4 = KF == kScanKeysFp4;
+  static constexpr int NCH = FP4 ? DI / 32 : DI / 16;     // 16-byte chunks (FP4: blocks) per key
+  static constexpr int CB = FP4 ? DI / 2 : DI;            // key bytes in the tile
+  static constexpr int EB = FP4 ? DI / 32 : 0;            // exponent bytes per key
+  static constexpr int KPT = FP4 ? 512 / DI : ((DI >= 64) ? 1 : 64 / DI);  // keys per thread per tile
   static constexpr int TILE_KEYS = kScanThreads * KPT;
-  static constexpr int TILE_BYTES = TILE_KEYS * DI;       // 16 KiB (32 KiB for d_I = 128)
-  static constexpr int STAGES = (TILE_BYTES > 16384) ? 3 : 4;
-  static constexpr bool QREG = HI * NCH <= 16;            // index query fits in registers
+  static constexpr int TILE_BYTES = TILE_KEYS * (CB + EB); // 16 KiB int8 (32 KiB for d_I = 128); 17-18 KiB FP4
+  static constexpr int STAGES = (TILE_BYTES > 20000) ? 3 : 4;
+  static constexpr int QW = FP4 ? 2 : 1;                  // query int4 per chunk
+  static constexpr bool QREG = HI * NCH * QW <= 16;       // index query fits in registers
   static constexpr size_t SMEM = size_t(STAGES) * TILE_BYTES;
   static_assert(DI % 16 == 0 && NCH >= 1 && NCH <= 8, "d_I in {16,32,64,128}");
+  static_assert(!FP4 || (DI % 32 == 0 && QREG), "FP4 keys: d_I % 32 == 0, query in registers");
 };
 
 // Rotation of the chunk order of thread t (see the header comment).
@@ -47,19 +58,22 @@ __device__ __forceinline__ int chunk_xor(int t) {
   return (NCH == 1) ? 0 : (t / (8 / NCH)) % NCH;
 }
 
-// grid = (G slices, rows).  hist1: [rows][kHistStride], zeroed.
-template <int DI, int HI>
+// grid = (G slices, rows).  hist1: [rows][kHistStride], zeroed.  With FP4
+// keys, k_idx holds the codes [B, N, d_I/2] and k_exps the exponents [B, N,
+// d_I/32] (N % 16 == 0, so every copy starts on a 16-byte boundary).
+template <int DI, int HI, int KF = kScanKeysInt8>
 __global__ void __launch_bounds__(kScanThreads, 2)
     index_scan_kernel(const int8_t *__restrict__ q_idx, const float *__restrict__ w,
-                      const int8_t *__restrict__ k_idx, int32_t T, int64_t N, int64_t n_prior,
-                      int32_t ratio, int64_t row0, float *__restrict__ scores,
-                      int64_t score_stride, uint32_t *__restrict__ hist1, int write_masked) {
-  using S = ScanShape<DI, HI>;
-  constexpr int NCH = S::NCH, STAGES = S::STAGES, TK = S::TILE_KEYS;
+                      const int8_t *__restrict__ k_idx, const uint8_t *__restrict__ k_exps,
+                      int32_t T, int64_t N, int64_t n_prior, int32_t ratio, int64_t row0,
+                      float *__restrict__ scores, int64_t score_stride,
+                      uint32_t *__restrict__ hist1, int write_masked) {
+  using S = ScanShape<DI, HI, KF>;
+  constexpr int NCH = S::NCH, STAGES = S::STAGES, TK = S::TILE_KEYS, QW = S::QW;
   extern __shared__ __align__(128) unsigned char smem_tiles[];
   __shared__ uint64_t full_bar[STAGES];
   __shared__ uint32_t sh_hist[kBins1];
-  __shared__ __align__(16) int4 sh_q[S::QREG ? 1 : HI * NCH];
+  __shared__ __align__(16) int4 sh_q[S::QREG ? 1 : HI * NCH * QW];
 
   const int tid = threadIdx.x;
   const int64_t r_local = blockIdx.y, r = row0 + r_local;
@@ -75,7 +89,16 @@ __global__ void __launch_bounds__(kScanThreads, 2)
   const int64_t n0 = ((V * g) / G) & ~int64_t(15);
   const int64_t n1 = (g == G - 1) ? V : (((V * (g + 1)) / G) & ~int64_t(15));
   const int ntiles = (int)((n1 - n0 + TK - 1) / TK);
-  const int8_t *src = k_idx + (b * N + n0) * DI;
+  // tile t: keys [n0 + t*TK, ...) -> its stage (codes, then FP4 exponents)
+  auto issue = [&](int t, int stage) {
+    const int64_t keys = min64(TK, n1 - n0 - (int64_t)t * TK);
+    const int64_t key0 = b * N + n0 + (int64_t)t * TK;
+    unsigned char *dst = smem_tiles + stage * S::TILE_BYTES;
+    const uint32_t cb = (uint32_t)(keys * S::CB), eb = (uint32_t)(keys * S::EB);
+    mbar_arrive_expect_tx(&full_bar[stage], cb + eb);
+    bulk_g2s(dst, k_idx + key0 * S::CB, cb, &full_bar[stage]);
+    if constexpr (S::FP4) bulk_g2s(dst + TK * S::CB, k_exps + key0 * S::EB, eb, &full_bar[stage]);
+  };
 
   // The per-row selection kernel that follows may be scheduled now; it waits
   // for this grid's results before reading them.
@@ -86,26 +109,22 @@ __global__ void __launch_bounds__(kScanThreads, 2)
     fence_barrier_init();
   }
   __syncthreads();
-  if (tid == 0) {
-    for (int s = 0; s < STAGES && s < ntiles; ++s) {
-      const int64_t keys = min64(TK, n1 - n0 - (int64_t)s * TK);
-      const uint32_t bytes = (uint32_t)(keys * DI);
-      mbar_arrive_expect_tx(&full_bar[s], bytes);
-      bulk_g2s(smem_tiles + s * S::TILE_BYTES, src + (int64_t)s * TK * DI, bytes, &full_bar[s]);
-    }
-  }
+  if (tid == 0)
+    for (int s = 0; s < STAGES && s < ntiles; ++s) issue(s, s);
 
   // This thread's index-query chunks, pre-permuted by its chunk rotation.
   const int x = chunk_xor<NCH>(tid);
-  int4 qreg[S::QREG ? HI * NCH : 1];
+  int4 qreg[S::QREG ? HI * NCH * QW : 1];
   const int4 *qrow = reinterpret_cast<const int4 *>(q_idx + r * HI * DI);
   if constexpr (S::QREG) {
 #pragma unroll
     for (int h = 0; h < HI; ++h)
 #pragma unroll
-      for (int c = 0; c < NCH; ++c) qreg[h * NCH + c] = qrow[h * NCH + (c ^ x)];
+      for (int c = 0; c < NCH; ++c)
+#pragma unroll
+        for (int u = 0; u < QW; ++u) qreg[(h * NCH + c) * QW + u] = qrow[(h * NCH + (c ^ x)) * QW + u];
   } else {
-    for (int i = tid; i < HI * NCH; i += kScanThreads) sh_q[i] = qrow[i];
+    for (int i = tid; i < HI * NCH * QW; i += kScanThreads) sh_q[i] = qrow[i];
   }
   float wh[HI];
 #pragma unroll
@@ -124,13 +143,8 @@ __global__ void __launch_bounds__(kScanThreads, 2)
       break;
     }
     if (tid == 0 && it >= 1 && it - 1 + STAGES < ntiles) {
-      const int nt = it - 1 + STAGES, ps = (it - 1) % STAGES;
-      const int64_t keys = min64(TK, n1 - n0 - (int64_t)nt * TK);
-      const uint32_t bytes = (uint32_t)(keys * DI);
       asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-      mbar_arrive_expect_tx(&full_bar[ps], bytes);
-      bulk_g2s(smem_tiles + ps * S::TILE_BYTES, src + (int64_t)nt * TK * DI, bytes,
-               &full_bar[ps]);
+      issue(it - 1 + STAGES, (it - 1) % STAGES);
     }
     const unsigned char *tile = smem_tiles + s * S::TILE_BYTES;
     const int64_t tbase = n0 + (int64_t)it * TK;
@@ -140,7 +154,13 @@ __global__ void __launch_bounds__(kScanThreads, 2)
       const int kl = tid + j * kScanThreads;
       const bool valid = kl < tkeys;
       float score = 0.0f;
-      if (valid) {
+      if constexpr (S::FP4) {
+        if (valid) {
+          score = fp4_key_score<NCH, HI, S::QREG>(tile + kl * S::CB,
+                                                  tile + TK * S::CB + kl * S::EB, qreg, sh_q, wh, x);
+          srow[tbase + kl] = score;
+        }
+      } else if (valid) {
         const unsigned char *krow = tile + kl * DI;
         int dot[HI];
 #pragma unroll

@@ -206,6 +206,70 @@ __device__ __forceinline__ void e2m1x8_to_i8x8(uint32_t w, uint32_t &lo, uint32_
   hi = (prmt(kPos0, kPos1, sh) & ~mh) | (prmt(kNeg0, kNeg1, sh) & mh);
 }
 
+// Index score of one FP4 key (this library's reading, see the header of the
+// FP4 index key calls): per head h and key block b the exact integer
+// idot = sum over the block of q[h, i] * (2 * E2M1(code_i)), the head's dot
+// = fp32 sum over the blocks in ascending order of idot * 2^(exp_b - 128),
+// score = ((0 + w_0 * dot_0) + w_1 * dot_1) + ... + 0 (each op rounded).
+// kc: the key's NB x 16 code bytes, ke: its NB exponent bytes (shared
+// memory).  The thread visits block c ^ x at step c (bank-conflict-free
+// rotation); its query is either in registers, pre-permuted the same way
+// (qreg[(h * NB + c) * 2 + u] = query int4 u of block c ^ x), or in shared
+// memory in natural order (qs).
+template <int NB, int HI, bool QREG>
+__device__ __forceinline__ float fp4_key_score(const unsigned char *kc, const unsigned char *ke,
+                                               const int4 *qreg, const int4 *qs,
+                                               const float *wh, int x) {
+  uint32_t ew = 0;
+#pragma unroll
+  for (int b = 0; b < NB; ++b) ew |= (uint32_t)ke[b] << (8 * b);
+  float term[HI][NB];
+#pragma unroll
+  for (int cc = 0; cc < NB; ++cc) {
+    const int blk = cc ^ x;
+    const int4 kv = *reinterpret_cast<const int4 *>(kc + (blk << 4));
+    uint32_t kw[8];
+    e2m1x8_to_i8x8((uint32_t)kv.x, kw[0], kw[1]);
+    e2m1x8_to_i8x8((uint32_t)kv.y, kw[2], kw[3]);
+    e2m1x8_to_i8x8((uint32_t)kv.z, kw[4], kw[5]);
+    e2m1x8_to_i8x8((uint32_t)kv.w, kw[6], kw[7]);
+    const float scale = pow2_f32((int)((ew >> (8 * blk)) & 0xffu) - 128);
+#pragma unroll
+    for (int h = 0; h < HI; ++h) {
+      int4 q0, q1;
+      if constexpr (QREG) {
+        q0 = qreg[(h * NB + cc) * 2 + 0];
+        q1 = qreg[(h * NB + cc) * 2 + 1];
+      } else {
+        q0 = qs[(h * NB + blk) * 2 + 0];
+        q1 = qs[(h * NB + blk) * 2 + 1];
+      }
+      int idot = 0;
+      idot = __dp4a((int)kw[0], q0.x, idot);
+      idot = __dp4a((int)kw[1], q0.y, idot);
+      idot = __dp4a((int)kw[2], q0.z, idot);
+      idot = __dp4a((int)kw[3], q0.w, idot);
+      idot = __dp4a((int)kw[4], q1.x, idot);
+      idot = __dp4a((int)kw[5], q1.y, idot);
+      idot = __dp4a((int)kw[6], q1.z, idot);
+      idot = __dp4a((int)kw[7], q1.w, idot);
+      const float t = __fmul_rn(__int2float_rn(idot), scale);
+#pragma unroll
+      for (int b = 0; b < NB; ++b)
+        if (b == blk) term[h][b] = t;
+    }
+  }
+  float acc = 0.0f;
+#pragma unroll
+  for (int h = 0; h < HI; ++h) {
+    float dot = 0.0f;
+#pragma unroll
+    for (int b = 0; b < NB; ++b) dot = __fadd_rn(dot, term[h][b]);
+    acc = __fadd_rn(acc, __fmul_rn(wh[h], dot));
+  }
+  return __fadd_rn(acc, 0.0f);
+}
+
 // Four E2M1 codes pairs (one 32-bit word = 8 codes) -> 8 fp32 values times a
 // scale, through the sm_100a hardware converter (e2m1x2 -> f16x2, exact).
 __device__ __forceinline__ void e2m1x8_to_f32(uint32_t word, float s, float *out) {

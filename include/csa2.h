@@ -239,7 +239,7 @@ size_t csa2_index_topk_fp4k_workspace_size(int32_t B, int32_t H_I, int32_t d_I, 
  *   k_codes device, uint8 [B, N, d_I/2]; k_exps device, uint8 [B, N, d_I/32]
  *   idx_out device, int32 [B, topk]   (output)
  *   ws      device workspace of ws_bytes >= csa2_index_topk_fp4k_workspace_size
- * Supported: d_I in {32, 64}, H_I == 4, N % 16 == 0, N >= 1, topk <= 4096. */
+ * Supported: d_I in {32, 64}, H_I == 4, N % 16 == 0, N >= 1, topk <= 65536. */
 csa2_status csa2_index_topk_fp4k(const int8_t *q_idx, const float *w, const uint8_t *k_codes,
                                  const uint8_t *k_exps, int32_t B, int32_t H_I, int32_t d_I,
                                  int64_t N, int32_t topk, int32_t *idx_out, void *ws,
@@ -384,7 +384,7 @@ typedef struct csa2_layer_io {
      * csa2_pack_index_keys_fp4) instead of int8 -- k_idx then points at the
      * FP4 codes [B, N, d_I/2] and k_exps at the block exponents [B, N,
      * d_I/32].  NULL: int8 keys.  Layers over FP4 keys need the decode shape
-     * of csa2_index_topk_fp4k and H <= 16. */
+     * of csa2_index_topk_fp4k. */
     const uint8_t *k_exps;
     /* Optional, Full layers with int8 keys: this step's entry append
      * (csa2_append_entry) into the layer's own store before its index scan,
@@ -454,6 +454,22 @@ csa2_status csa2_trace_get(int32_t i, const char **name, float *ms);
 /* ---------------------------------------------------------------------- */
 /* Device status                                                           */
 /* ---------------------------------------------------------------------- */
+
+/* Decode kernels.  Decode rows (one query per sequence, every entry
+ * visible, no score output) are served either by two launches per layer --
+ * the index scan (scores to the workspace) and one thread-block cluster per
+ * query row for the top-k and the attention (CSA2_DECODE_SCAN_CLUSTER, the
+ * default) -- or by one cooperative launch that keeps each CTA's scores in
+ * shared memory and meets the other CTAs through global counters
+ * (CSA2_DECODE_FUSED).  Both compute the same results bit for bit (indices)
+ * and within the attention tolerance.  FP4 index keys and candidate pools
+ * are served by both.  Process-wide; the environment variable
+ * CSA2_DECODE_KERNEL=fused sets the initial choice.  Not synchronised with
+ * calls in flight on other host threads. */
+#define CSA2_DECODE_SCAN_CLUSTER 0
+#define CSA2_DECODE_FUSED 1
+csa2_status csa2_set_decode_kernel(int32_t kernel);
+int32_t csa2_get_decode_kernel(void);
 
 /* Self-test of the library's bounded waits (every wait on a pipeline
  * barrier, on another CTA's delivery or on another CTA's counter gives up

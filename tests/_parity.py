@@ -55,3 +55,13 @@ def assert_bits_equal(gpu: np.ndarray, ref: np.ndarray, what: str = ""):
     if not np.array_equal(gv, rv):
         nbad = int(np.sum(g.reshape(-1) != r.reshape(-1)))
         raise AssertionError(f"{what}: {nbad} elements differ")
+
+
+DECODE_KERNELS = [(csa2.DECODE_SCAN_CLUSTER, "scan_cluster"), (csa2.DECODE_FUSED, "fused")]
+
+
+def use_decode_kernel(kernel):
+    """Select the decode kernels (process-wide); returns the previous choice."""
+    prev = csa2.get_decode_kernel()
+    csa2.set_decode_kernel(kernel)
+    return prev

@@ -24,3 +24,14 @@ def pytest_collection_modifyitems(config, items):
     for item in items:
         if "gpu" in item.keywords:
             item.add_marker(skip)
+
+
+@pytest.fixture(params=[0, 1], ids=["scan_cluster", "fused"])
+def decode_kernel(request):
+    """Run a decode-path test under both decode kernels (the index scan +
+    per-row cluster kernels, and the fused single-launch kernel)."""
+    import compressed_sparse_attention_topk_b200 as csa2
+    prev = csa2.get_decode_kernel()
+    csa2.set_decode_kernel(request.param)
+    yield request.param
+    csa2.set_decode_kernel(prev)

@@ -58,7 +58,7 @@ def _fp4_case(seed, B, H_I, d_I, N):
 @pytest.mark.parametrize("B,d_I,N,topk", [(1, 64, 16, 5), (4, 64, 3008, 2048), (3, 32, 20000, 64),
                                           (2, 64, 262144, 2048), (5, 64, 4096, 4096),
                                           (40, 32, 4000, 256)])
-def test_index_topk_fp4_keys_bit_exact(B, d_I, N, topk):
+def test_index_topk_fp4_keys_bit_exact(B, d_I, N, topk, decode_kernel):
     q, w, codes, exps = _fp4_case(B * 10 + N, B, 4, d_I, N)
     got = host(csa2.index_topk_fp4k(dev(q), dev(w), dev(codes), dev(exps), topk))
     ref = oracle.index_topk_fp4k(q, w, codes, exps, topk)
@@ -66,7 +66,7 @@ def test_index_topk_fp4_keys_bit_exact(B, d_I, N, topk):
     assert csa2.get_device_status() == 0
 
 
-def test_index_topk_fp4_keys_ties():
+def test_index_topk_fp4_keys_ties(decode_kernel):
     # keys from a few levels only: many equal scores at the threshold
     rng = np.random.default_rng(4)
     B, H_I, d_I, N, topk = 3, 4, 64, 9008, 1000
@@ -96,7 +96,7 @@ def _layers_fp4(w0, layers):
 
 
 @pytest.mark.parametrize("B,N,W", [(4, 262144, 128), (2, 5008, 0), (3, 1008, 128)])
-def test_decode_layers_over_fp4_keys(B, N, W):
+def test_decode_layers_over_fp4_keys(B, N, W, decode_kernel):
     w0 = wl.with_sizes(wl.LONG, name=f"fp4k_{B}_{N}", B=B, N=N, W=W, seed=B + N)
     layers = wl.all_layer_inputs(w0)
     rng = np.random.default_rng(N)
@@ -117,7 +117,7 @@ def test_decode_layers_over_fp4_keys(B, N, W):
     assert csa2.get_device_status() == 0
 
 
-def test_layer_call_appends_the_step_entry_before_its_scan():
+def test_layer_call_appends_the_step_entry_before_its_scan(decode_kernel):
     """A Full layer given this step's entry appends it (FP4 entry + int8 key)
     into its store before scanning: bit-exact store, and the selection and
     attention of both layers see the new entry."""

@@ -10,8 +10,8 @@ import oracle
 import compressed_sparse_attention_topk_b200 as csa2
 from compressed_sparse_attention_topk_b200 import build as csa2_build
 from compressed_sparse_attention_topk_b200 import workloads as wl
-from tests._parity import (assert_bits_equal, assert_close, dev, gpu_store, host,
-                           oracle_store)
+from tests._parity import (DECODE_KERNELS, assert_bits_equal, assert_close, dev, gpu_store,
+                           host, oracle_store, use_decode_kernel)
 
 pytestmark = pytest.mark.gpu
 
@@ -89,13 +89,19 @@ def _check_index(q, w, k, topk, n_prior=-1, ratio=4, rows=None, check_scores=Tru
         if rows is not None:
             g_sc = g_sc[rows]
         assert_bits_equal(g_sc, o_sc, "scores")
-        # the same call without a score output: with one query per sequence
-        # this takes the fused decode kernel (scores stay on chip)
-        g2 = host(csa2.index_topk(dev(q), dev(w), dev(k), topk, n_prior, ratio))
-        g2 = g2.reshape(B * T, topk)
-        if rows is not None:
-            g2 = g2[rows]
-        assert_bits_equal(g2, o_idx, "indices without score output")
+        # the same call without a score output, under each decode kernel
+        # (with one query per sequence the fused kernel keeps the scores on
+        # chip)
+        for kernel, name in DECODE_KERNELS:
+            prev = use_decode_kernel(kernel)
+            try:
+                g2 = host(csa2.index_topk(dev(q), dev(w), dev(k), topk, n_prior, ratio))
+            finally:
+                use_decode_kernel(prev)
+            g2 = g2.reshape(B * T, topk)
+            if rows is not None:
+                g2 = g2[rows]
+            assert_bits_equal(g2, o_idx, f"indices without score output ({name})")
     assert_bits_equal(g_idx, o_idx, "indices")
     return g_idx
 
@@ -457,7 +463,7 @@ def _run_group_and_compare(w0, rows=None):
     (5, 20000, 4096, 70, 16, 128, 8, 64),
     (2, 100, 7, 128, 16, 128, 4, 32),
 ])
-def test_decode_layer_shapes(B, N, topk, W, H, D, H_I, d_I):
+def test_decode_layer_shapes(B, N, topk, W, H, D, H_I, d_I, decode_kernel):
     """Full + Reindex decode layers through the layer call (fused decode
     kernel): selection bit-exact, attention within tolerance."""
     w0 = wl.with_sizes(wl.LONG, name=f"decode_{B}_{N}_{topk}", B=B, N=N, topk=topk, W=W, H=H,
@@ -465,7 +471,7 @@ def test_decode_layer_shapes(B, N, topk, W, H, D, H_I, d_I):
     _run_group_and_compare(w0)
 
 
-def test_decode_layer_cuda_graph_replay():
+def test_decode_layer_cuda_graph_replay(decode_kernel):
     """The layer call captured into a CUDA graph (as the benchmark runs it)
     and replayed gives the eager results, bit for bit, on every replay."""
     w0 = wl.with_sizes(wl.LONG, name="graph_replay", B=4, N=20000, seed=77)
@@ -503,7 +509,7 @@ def test_group_workload_16_layers():
     assert csa2.group_cache_bytes(list(w0.modes), w0.N, 128, 8) == 2 * 1024 * 1024
 
 
-def test_long_decode_workload_full_size():
+def test_long_decode_workload_full_size(decode_kernel):
     """The 1M-token decode workload at full size (B=4, N=262144, Full +
     Reindex), in the launch configuration the benchmark times."""
     _run_group_and_compare(wl.LONG)

@@ -161,7 +161,7 @@ def _pool_layers(w0, layers, block, n_blocks):
                                                      (3, 20001, 8, 300, 512),
                                                      (2, 5000, 16, 40, 100),
                                                      (2, 3000, 8, 400, 64)])
-def test_pool_layers_in_the_layer_call(B, N, block, n_blocks, topk):
+def test_pool_layers_in_the_layer_call(B, N, block, n_blocks, topk, decode_kernel):
     from tests._parity import assert_close, oracle_store
     w0 = wl.with_sizes(wl.LONG, name=f"pool_layers_{N}", B=B, N=N, topk=topk, seed=N + B,
                        modes=((0, 0, 0), (csa2.REINDEX_POOL, 0, 1), (2, 0, 1)))
