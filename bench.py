@@ -80,6 +80,27 @@ def algorithmic_bytes(w0, key_format: str = "int8") -> dict:
     return {"keys": keys, "gather": gather, "window": window, "total": keys + gather + window}
 
 
+# Algorithmic bytes of one launch of each library kernel of the decode step
+# (per launch the kernel serves all B rows of one layer).
+KERNEL_BYTES = {
+    "index_scan": lambda w0, ab: w0.B * ab["keys"],
+    "topk_attend": lambda w0, ab: w0.B * (ab["gather"] + ab["window"]),
+    "decode_fused": lambda w0, ab: w0.B * ab["total"],
+}
+
+
+def step_traffic(kernels):
+    """DRAM bytes of a step from the committed ncu summaries, when every
+    kernel of the step has one (else None)."""
+    tot = 0
+    for k, v in kernels.items():
+        t = v.get("traffic")
+        if t is None:
+            return None
+        tot += t * v["launches_per_step"]
+    return tot
+
+
 def measured_peaks():
     p = os.path.join(ROOT, "MEASURED_PEAKS.json")
     if os.path.exists(p):
@@ -134,8 +155,9 @@ def pack_into_one_buffer(layers, keys, dev):
 
 
 KERNEL_SOURCES = {
-    "index_scan": ("index_scan.cuh", "common.cuh"),
-    "decode_fused": ("decode_fused.cuh", "attn_rows.cuh", "common.cuh"),
+    "index_scan": ("index_scan.cuh", "pack.cuh", "common.cuh"),
+    "topk_attend": ("row_cluster.cuh", "attn_rows.cuh", "pack.cuh", "common.cuh"),
+    "decode_fused": ("decode_fused.cuh", "attn_rows.cuh", "pack.cuh", "common.cuh"),
 }
 
 
@@ -568,15 +590,23 @@ def run_gpu(args, w0):
     step_bytes = w0.B * sum(layer_bytes(w0, args, l) for l in range(w0.L))
     ms_step = total_ms / args.steps
     step_gbs = step_bytes / (ms_step * 1e-3) / 1e9
-    # The dominant kernel: one launch per layer does the whole layer (scan,
-    # top-k, gather, attention), so its algorithmic bytes per launch are the
-    # layer's: B x (keys + gathered entries + window).
-    dom = "decode_fused" if "decode_fused" in per_kernel else "index_scan"
-    dom_n, dom_ms = per_kernel.get(dom, (0, 0.0))
-    dom_avg_ms = dom_ms / max(dom_n, 1)
-    dom_bytes = w0.B * (ab["total"] if dom == "decode_fused" else ab["keys"])
-    achieved = dom_bytes / (dom_avg_ms * 1e-3) / 1e9 if dom_n else None
-    kernel_ms_per_step = sum(v[1] for v in per_kernel.values()) / args.steps
+    # Per kernel: launches and device time per step.  The trace's event pairs
+    # add a fixed cost to each launch, so their sum exceeds the untraced step;
+    # each kernel's share of the traced time, applied to the untraced step,
+    # gives per-kernel times that add up to ms_per_step.
+    traced_ms_per_step = sum(v[1] for v in per_kernel.values()) / args.steps
+    kernels = {}
+    for k, (c, s_) in sorted(per_kernel.items()):
+        share = s_ / args.steps / traced_ms_per_step if traced_ms_per_step else 0.0
+        per_launch = share * ms_step / (c / args.steps)
+        b = KERNEL_BYTES.get(k, lambda w0_, ab_: None)(w0, ab)
+        kernels[k] = {"launches_per_step": c / args.steps, "share_of_step": share,
+                      "ms_per_launch": per_launch, "traced_ms_per_launch": s_ / c,
+                      "bytes_per_launch": b}
+        if b:
+            kernels[k].update({"achieved_gbs": b / (per_launch * 1e-3) / 1e9,
+                               "frac": b / (per_launch * 1e-3) / 1e9 / peak,
+                               "traffic": ncu_traffic(k)})
 
     line = None
     if rank == 0:
@@ -605,23 +635,17 @@ def run_gpu(args, w0):
                        "step_algorithmic_bytes": step_bytes,
                        "step_hbm_gbs": step_gbs, "step_hbm_frac": step_gbs / peak,
                        "wall_s_timed_region": wall_s},
-            "roofline": {"bound": "hbm", "kernel": dom, "timing": trace_kind,
-                         "achieved": achieved,
-                         "peak": peak, "peak_kind": f"{peak_kind} (copy bandwidth)",
-                         "unit": "GB/s", "frac": (achieved / peak) if achieved else None,
-                         "frac_of_8tbs_nominal": (achieved / 8000.0) if achieved else None,
-                         "traffic": ncu_traffic(dom),
-                         "bytes_per_launch": dom_bytes,
-                         "avg_launch_ms": dom_avg_ms,
-                         "step": {"achieved": step_gbs, "frac": step_gbs / peak,
-                                  "frac_of_8tbs_nominal": step_gbs / 8000.0,
-                                  "note": "algorithmic bytes of a whole step over ms_per_step "
-                                          "(launch gaps and workspace clears included)"}},
-            "kernels": {k: {"launches": c, "avg_us": s / c * 1e3,
-                            "ms_per_step": s / args.steps,
-                            "share_of_step": s / args.steps / ms_step}
-                        for k, (c, s) in sorted(per_kernel.items())},
-            "kernel_ms_per_step": kernel_ms_per_step,
+            "roofline": {"bound": "hbm", "scope": "decode step (both layers, every launch)",
+                         "achieved": step_gbs, "peak": peak,
+                         "peak_kind": f"{peak_kind} (copy bandwidth)", "unit": "GB/s",
+                         "frac": step_gbs / peak, "frac_of_8tbs_nominal": step_gbs / 8000.0,
+                         "bytes_per_step": step_bytes, "ms_per_step": ms_step,
+                         "traffic": step_traffic(kernels),
+                         "kernels": {k: {kk: v[kk] for kk in ("bytes_per_launch",
+                                                               "ms_per_launch", "achieved_gbs",
+                                                               "frac", "traffic") if kk in v}
+                                     for k, v in kernels.items() if v.get("bytes_per_launch")}},
+            "kernels": kernels, "kernel_timing": trace_kind + ", scaled to the untraced step",
             "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": h2d,
                     "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms / args.steps,
                     "segments_ms_per_step": {k: v / args.steps for k, v in e2e_seg.items()}},
