@@ -258,6 +258,29 @@ def oracle_sample(w0, seconds: float, min_runs: int = 1):
     return runs, dt
 
 
+def oracle_rows_sample(w0, lay, seconds: float) -> dict:
+    """Time the CPU oracle on query rows of a one-layer workload with several
+    query tokens per sequence (index + top-k over the row's visible entries,
+    then attention), eight rows per call, spread evenly over the chunk, until
+    `seconds` have passed."""
+    import oracle
+    B, N, D = lay["entries"].shape
+    c, s = oracle.pack_fp4(lay["entries"].reshape(B * N, D))
+    layer = dict(lay, codes=c.reshape(B, N, D // 2), scales=s.reshape(B, N, D // 16))
+    nrows = w0.B * w0.T
+    order = np.arange(nrows).reshape(-1, 8).T.reshape(-1) if nrows % 8 == 0 else np.arange(nrows)
+    done, t0 = 0, time.perf_counter()
+    while done == 0 or time.perf_counter() - t0 < seconds:
+        rows = order[done % nrows: done % nrows + 8]
+        oracle.layer_group([(0, 0, 0)], [layer], w0.topk, w0.n_prior, w0.ratio, rows=rows)
+        done += len(rows)
+    dt = time.perf_counter() - t0
+    return {"value": done / dt, "unit": "tokens/s/layer", "cores": 1, "kind": "oracle",
+            "sample": f"{done} query rows, cycling over the {nrows} of one layer call in an "
+                      f"order spread over the chunk, plain C oracle, single thread, {dt:.1f} s",
+            **host_cpu()}
+
+
 def host_cpu() -> dict:
     """The host's CPU model and logical core count (for the oracle timings);
     "unknown" where the system does not say."""
@@ -708,6 +731,9 @@ def run_prefill(args, w0):
     for name, m in recs:
         c, s_ = per.get(name, (0, 0.0))
         per[name] = (c + 1, s_ + m)
+    cpu = None
+    if not args.no_cpu_baseline:
+        cpu = oracle_rows_sample(w0, lay, args.cpu_seconds)
     print(json.dumps({
         "metric": ("CSA2 chunked-prefill tokens/s per layer (supplementary)" if w0.n_prior >= 0
                    else "CSA2 multi-token decode tokens/s per layer (supplementary)"),
@@ -715,6 +741,7 @@ def run_prefill(args, w0):
         "steps": args.steps, "config": {"workload": w0.name, "T": w0.T, "N": w0.N,
                                           "n_prior": w0.n_prior, "topk": w0.topk},
         "kernels": {k: {"launches": c, "total_ms": s_} for k, (c, s_) in per.items()},
+        "cpu_baseline": cpu,
     }), flush=True)
     return 0
 

@@ -33,7 +33,11 @@
 //      it.  Equal keys are equal scores; they are taken in index order
 //      (lower index first) up to the count still needed.  Prefix sums over
 //      ranks and threads give every thread its offset in the output row, so
-//      the indices come out ascending.
+//      the indices come out ascending.  When every equal key is taken (the
+//      usual case: the cluster holds exactly as many as are still needed),
+//      a CTA's selection does not depend on the other ranks: it attends at
+//      once, and the warps that do not attend exchange the counts and write
+//      the output indices meanwhile.
 //
 // Attention: each CTA attends over an even share of the window rows and over
 // the entries it selected itself (with given indices, an even share of the
@@ -48,8 +52,11 @@
 //   values  O[h, d] += sum_n (P[h, n] * s[n, g(d)]) * e2m1[n, d]
 //           with the fp32 weight P*s split into a bf16 pair hi + lo (two
 //           products), so the weight keeps ~16 bits.
-// Window rows use the same path with scale 1 (bf16 keys and values).  The
-// warps' states are merged in shared memory (their buffers alias the dead
+// Window rows use the same path with scale 1 (bf16 keys and values); they do
+// not depend on the selection, so one warp of its own attends over the CTA's
+// share of them (its first chunk's copies issued in the prologue, while the
+// scan that produces the scores may still run) alongside the entry warps,
+// and its state joins the merge.  The warps' states are merged in shared memory (their buffers alias the dead
 // top-k working set), and each CTA pushes its partial (max, sum, acc) of
 // head h into the shared memory of the CTA that owns h (h mod CL); once its
 // partials are in, each owner merges them locally by log-sum-exp.  Which CTA
@@ -72,7 +79,8 @@ constexpr int kStageScores = 16384;  // scores staged in shared memory per round
 constexpr int kCandCap = 2048;       // candidates kept in shared memory (more spill to global)
 constexpr int kSelCap = 4096;        // selected indices kept in shared memory
 constexpr int kHeads = 16;           // heads per pass (the MMA's M)
-constexpr int kAttnWarps = 10;       // warps that run attention chunks
+constexpr int kAttnWarps = 10;       // warps that run attention chunks of the selected entries
+constexpr int kWinWarp = kRowWarps - 1;  // the warp that attends over the CTA's window rows
 
 struct RowParams {
   // top-k
@@ -118,7 +126,9 @@ struct RowSmem {
   uint16_t qb[kHeads][D + 8];   // query of the head pass, bf16
   // pushed partials of the heads this CTA merges: (m, l, -, -, acc[D])
   alignas(16) float inbox[kHeads][D + 4];
-  float mf[kHeads][kAttnWarps + 1];  // per head: each attention warp's factor, then the max
+  // per head: the factor of each source (attention warps, then the window
+  // state), then the max
+  float mf[kHeads][kAttnWarps + 2];
   float fac[kHeads];            // final merge: factor of each inbox slot
   float mrg_m[kHeads], mrg_l[kHeads];  // final merge: max and sum of each merged head
   uint32_t scratch[40];
@@ -129,6 +139,8 @@ struct RowSmem {
   // exchange barriers, one per delivery (bytes counted by st.async):
   // digit-2 slices, digit-2 sums, digit-3 slices, digit-3 sums, counts, partials
   uint64_t xbar[6];
+  // the window warp's chunk area, then its partial state
+  ar::WarpArea<D> win;
 };
 
 __device__ __forceinline__ int64_t row_visible(int64_t N, int64_t n_prior, int32_t ratio,
@@ -200,8 +212,14 @@ __device__ void cluster_threshold(RowSmem<D> &sm, cg::cluster_group &cluster, ui
 }
 
 
+// Returns true when the CTA's selection is complete in `sel` but its
+// indices are not yet written to the output row: every tie at the threshold
+// key is taken and the selection fits `sel`, so the CTA's selection does not
+// depend on the other ranks' counts and attention may start at once; the
+// counts exchange and the index write are then left to the warps that do not
+// attend (write_row_indices).
 template <int D, int CL>
-__device__ void row_topk(RowSmem<D> &sm, const RowParams &p, cg::cluster_group &cluster,
+__device__ bool row_topk(RowSmem<D> &sm, const RowParams &p, cg::cluster_group &cluster,
                          int64_t r_local, int64_t r, int64_t K, bool bulk, int64_t s0, int64_t s1,
                          bool &abort, uint32_t &phase) {
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
@@ -329,9 +347,27 @@ __device__ void row_topk(RowSmem<D> &sm, const RowParams &p, cg::cluster_group &
     above_before = block_excl_scan<kRowThreads>(n_above, sm.scratch, tot_above);
     tie_before = block_excl_scan<kRowThreads>(n_tie, sm.scratch, tot_tie);
   }
-  // this CTA's counts to every rank; wait for every rank's
+  // this CTA's counts to every rank
   if (tid == 0) mbar_arrive_expect_tx(&sm.xbar[4], CL * 8);
   if (tid < CL) st_async_v2(&sm.cnt_all[c][0], tot_above, tot_tie, &sm.xbar[4], (uint32_t)tid);
+  // Every tie taken (no digit-3 split, or the cluster holds exactly as many
+  // keys equal to the threshold key as are still needed): the selection is
+  // the above-threshold and tied candidates, in index order.
+  const bool ties_all = !need3 || sm.thr[4] <= r3;
+  if (p.do_attn && ties_all && tot_above + tot_tie <= (uint32_t)kSelCap) {
+    uint32_t at = above_before + tie_before;
+    for (uint32_t i = i0; i < i1; ++i) {
+      const uint2 e = cand_at(i);
+      if (cand_class(e.x, t1, t2, t3, need3) != 0u) sm.sel[at++] = (int32_t)(s0 + e.y);
+    }
+    if (tid == 0) {
+      sm.sel_base = 0;
+      sm.sel_count = tot_above + tot_tie;
+    }
+    __syncthreads();
+    return true;
+  }
+  // wait for every rank's counts
   if (!mbar_wait_cluster_bounded(&sm.xbar[4], 0)) abort = true;
   if (warp == 0) {
     const uint32_t above = (lane < CL) ? sm.cnt_all[lane][0] : 0u;
@@ -370,6 +406,88 @@ __device__ void row_topk(RowSmem<D> &sm, const RowParams &p, cg::cluster_group &
     for (int64_t i = K + tid; i < p.topk; i += kRowThreads) orow[i] = -1;
   if (tid == 0) sm.sel_base = sm.out_base;
   __syncthreads();
+  return false;
+}
+
+// The output indices of a selection left pending by row_topk, written by the
+// warps [kAttnWarps, kWinWarp) while the others attend: wait for every
+// rank's counts, the rank's output offset from a warp scan over the ranks,
+// then the CTA's `sel` (all of it: every tie is taken) at that offset; the
+// last rank pads [K, topk) with -1.
+template <int D, int CL>
+__device__ void write_row_indices(RowSmem<D> &sm, const RowParams &p, int64_t r, int c,
+                                  int64_t K) {
+  constexpr int kSide = (kWinWarp - kAttnWarps) * 32;
+  const int st = threadIdx.x - kAttnWarps * 32, lane = threadIdx.x & 31;
+  mbar_wait_cluster_bounded(&sm.xbar[4], 0);  // a wait that gives up is in the status word
+  if (st < 32) {
+    const uint32_t sel = (lane < CL) ? sm.cnt_all[lane][0] + sm.cnt_all[lane][1] : 0u;
+    const uint32_t ob = warp_incl_scan(sel) - sel;
+    if (lane == c) sm.out_base = ob;
+  }
+  asm volatile("bar.sync 1, %0;" ::"n"(kSide) : "memory");
+  int32_t *orow = p.idx + r * (int64_t)p.topk;
+  const uint32_t ob = sm.out_base, n = sm.sel_count;
+  for (uint32_t i = st; i < n; i += kSide)
+    if (ob + i < (uint32_t)p.topk) orow[ob + i] = sm.sel[i];
+  if (c == CL - 1)
+    for (int64_t i = K + st; i < p.topk; i += kSide) orow[i] = -1;
+}
+
+// This CTA's window rows [w_lo, w_lo + nwin) of row r (rows t .. t + W - 1 of
+// its sequence's window slice).
+template <int CL>
+__device__ __forceinline__ void window_share(const RowParams &p, int64_t r, int c, int64_t &wrow0,
+                                             int &nwin) {
+  const int64_t b = r / p.T, t = r % p.T;
+  const int w_lo = (p.W * c) / CL;
+  nwin = (p.W * (c + 1)) / CL - w_lo;
+  wrow0 = b * ((int64_t)p.W - 1 + p.T) + t + w_lo;
+}
+
+// Issue (without waiting) the copies of window rows [row0, row0 + nrows)
+// (nrows <= 16) into the window area, missing rows zero-filled; one cp.async
+// group of the calling warp.
+template <int D>
+__device__ __forceinline__ void issue_window_rows(ar::WarpArea<D> &wa, const uint16_t *win_k,
+                                                  const uint16_t *win_v, int64_t row0, int nrows) {
+  constexpr int RP = D / 8;  // 16-byte pieces per row
+  const int lane = threadIdx.x & 31;
+  for (int i = lane; i < ar::kChunk * RP; i += 32) {
+    const int j = i / RP, u = i % RP;
+    const bool ok = j < nrows;
+    const int64_t row = ok ? row0 + j : row0;
+    ar::cp16(&wa.s.kt[j][8 * u], win_k + row * D + 8 * u, ok ? 16u : 0u);
+    ar::cp16(&wa.s.vt[j][8 * u], win_v + row * D + 8 * u, ok ? 16u : 0u);
+  }
+  ar::cp_commit();
+}
+
+// The window warp's part of a head pass: attention over this CTA's window
+// rows in chunks of 16 (the first chunk's copies already issued when
+// `first_issued`), then its state into the window area's merge slot.
+template <int D, int CL>
+__device__ void row_window_partial(RowSmem<D> &sm, const RowParams &p, int64_t r, int c,
+                                   bool first_issued) {
+  int64_t wrow0;
+  int nwin;
+  window_share<CL>(p, r, c, wrow0, nwin);
+  ar::WarpState<D> st;
+  ar::state_init(st);
+  for (int j0 = 0; j0 < nwin; j0 += ar::kChunk) {
+    const int n = min(ar::kChunk, nwin - j0);
+    uint32_t mask;
+    if (j0 == 0 && first_issued) {
+      ar::cp_wait<0>();
+      __syncwarp();
+      mask = (1u << n) - 1u;
+    } else {
+      mask = ar::load_window_rows<D>(sm.win, p.win_k, p.win_v, wrow0 + j0, n);
+    }
+    ar::attend_chunk16<D>(sm.win, sm.qb, st, mask, true, nullptr, p.q_scale);
+    __syncwarp();
+  }
+  ar::store_state<D>(sm.win, st);
 }
 
 // ---------------------------------------------------------------------------
@@ -387,34 +505,33 @@ __device__ void load_q(RowSmem<D> &sm, const RowParams &p, int64_t r, int h0, in
   }
 }
 
-// Attention of one head pass: this CTA's window rows and its entries (its
-// own selection `sel`, else the given index slots [lo, hi)), cut into
-// 16-key chunks that kAttnWarps warps take in turn, each with its own
-// running state; the CTA's merged partial of head h then goes to the owner
-// CTA h % CL, which merges the CL partials after one cluster barrier.
+// Attention of one head pass: this CTA's entries (its own selection `sel`,
+// else the given index slots [lo, hi)), cut into 16-key chunks that
+// kAttnWarps warps take in turn, each with its own running state, while the
+// last warp attends over the CTA's window rows (kWinWarp, its own area) and,
+// with idx_pending, the warps between write the selection's output indices.
+// The CTA's merged partial of head h then goes to the owner CTA h % CL,
+// which merges the CL partials.
 template <int D, int CL>
 __device__ void row_attend(RowSmem<D> &sm, const RowParams &p, cg::cluster_group &cluster,
                            int64_t r, int c, int h0, int nh, bool from_sel, int64_t lo,
-                           int64_t hi, int64_t sel_base) {
+                           int64_t hi, int64_t sel_base, bool win_issued, bool idx_pending,
+                           int64_t K) {
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int64_t b = r / p.T, t = r % p.T;
-  const int w_lo = (p.W * c) / CL, w_hi = (p.W * (c + 1)) / CL;
-  const int nwin = w_hi - w_lo;
+  const int64_t b = r / p.T;
+  const bool has_win = (p.W * (c + 1)) / CL > (p.W * c) / CL;
   const int64_t nsel = hi - lo;
-  const int64_t cw = (nwin + ar::kChunk - 1) / ar::kChunk;
-  const int64_t ce = p.N > 0 ? (nsel + ar::kChunk - 1) / ar::kChunk : 0;
+  const int64_t nch = p.N > 0 ? (nsel + ar::kChunk - 1) / ar::kChunk : 0;
   const int32_t *irow = p.idx + r * (int64_t)p.topk;
   const uint8_t *cseq = p.codes + b * p.N * (D / 2);
   const float *sseq = p.scales + b * p.N * (D / 16);
-  const int64_t wrow0 = b * ((int64_t)p.W - 1 + p.T) + t + w_lo;
   __syncthreads();  // top-k buffers dead, query in place
   if (warp < kAttnWarps) {
     ar::WarpArea<D> &wa = sm.u.aw[warp];
     ar::WarpState<D> st;
     ar::state_init(st);
-    const int64_t nch = cw + ce;
     auto entry_of = [&](int64_t ch) -> int32_t {  // this lane's key of entry chunk ch
-      const int64_t k = (ch - cw) * ar::kChunk + (lane & 15);
+      const int64_t k = ch * ar::kChunk + (lane & 15);
       if (k >= nsel) return -1;
       if (from_sel) {
         if (k < kSelCap) return sm.sel[k];
@@ -422,18 +539,9 @@ __device__ void row_attend(RowSmem<D> &sm, const RowParams &p, cg::cluster_group
       }
       return (lo + k < p.topk) ? irow[lo + k] : -1;
     };
-    // this warp's first entry chunk is gathered before its window chunks run
     int64_t ech = warp;
-    while (ech < cw) ech += kAttnWarps;
     uint32_t mask_cur = 0u;
     if (ech < nch) mask_cur = ar::gather_entries<D>(wa, 0, entry_of(ech), p.N, cseq, sseq);
-    for (int64_t ch = warp; ch < cw; ch += kAttnWarps) {
-      const int j0 = (int)ch * ar::kChunk;
-      const uint32_t mask = ar::load_window_rows<D>(wa, p.win_k, p.win_v, wrow0 + j0,
-                                                    min(ar::kChunk, nwin - j0));
-      ar::attend_chunk16<D>(wa, sm.qb, st, mask, true, nullptr, p.q_scale);
-      __syncwarp();
-    }
     // entry chunks, the next one gathered while the current one is used
     for (int it = 0; ech < nch; ++it, ech += kAttnWarps) {
       const int sb = it & 1;
@@ -452,16 +560,24 @@ __device__ void row_attend(RowSmem<D> &sm, const RowParams &p, cg::cluster_group
       mask_cur = mask_next;
     }
     ar::store_state<D>(wa, st);
+  } else if (warp == kWinWarp) {
+    if (has_win) row_window_partial<D, CL>(sm, p, r, c, win_issued);
+  } else if (idx_pending) {
+    write_row_indices<D, CL>(sm, p, r, c, K);
   }
   __syncthreads();
-  // per head: the max over the warps and each warp's factor
-  for (int i = tid; i < nh * kAttnWarps; i += kRowThreads) {
-    const int h = i / kAttnWarps, w = i % kAttnWarps;
+  // per head: the max over the sources (the attention warps, then the
+  // window warp) and each source's factor
+  const int ns = kAttnWarps + (has_win ? 1 : 0);
+  auto src_area = [&](int v) -> const ar::WarpArea<D> & {
+    return v < kAttnWarps ? sm.u.aw[v] : sm.win;
+  };
+  for (int i = tid; i < nh * ns; i += kRowThreads) {
+    const int h = i / ns, w = i % ns;
     float M = -INFINITY;
-#pragma unroll
-    for (int v = 0; v < kAttnWarps; ++v) M = fmaxf(M, sm.u.aw[v].merge.m[h]);
-    sm.mf[h][w] = M == -INFINITY ? 0.0f : exp2f(sm.u.aw[w].merge.m[h] - M);
-    if (w == 0) sm.mf[h][kAttnWarps] = M;
+    for (int v = 0; v < ns; ++v) M = fmaxf(M, src_area(v).merge.m[h]);
+    sm.mf[h][w] = M == -INFINITY ? 0.0f : exp2f(src_area(w).merge.m[h] - M);
+    if (w == 0) sm.mf[h][kAttnWarps + 1] = M;
   }
   __syncthreads();
   // this CTA's partial of each head (max, sum, acc) -> inbox slot
@@ -477,13 +593,11 @@ __device__ void row_attend(RowSmem<D> &sm, const RowParams &p, cg::cluster_group
     const int h = i / U, q = i % U;
     float4 v = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
     if (q == 0) {
-#pragma unroll
-      for (int w = 0; w < kAttnWarps; ++w) v.y = fmaf(sm.u.aw[w].merge.l[h], sm.mf[h][w], v.y);
-      v.x = sm.mf[h][kAttnWarps];
+      for (int w = 0; w < ns; ++w) v.y = fmaf(src_area(w).merge.l[h], sm.mf[h][w], v.y);
+      v.x = sm.mf[h][kAttnWarps + 1];
     } else {
-#pragma unroll
-      for (int w = 0; w < kAttnWarps; ++w) {
-        const float4 o = *reinterpret_cast<const float4 *>(&sm.u.aw[w].merge.o[h][4 * (q - 1)]);
+      for (int w = 0; w < ns; ++w) {
+        const float4 o = *reinterpret_cast<const float4 *>(&src_area(w).merge.o[h][4 * (q - 1)]);
         const float f = sm.mf[h][w];
         v.x = fmaf(o.x, f, v.x);
         v.y = fmaf(o.y, f, v.y);
@@ -570,6 +684,18 @@ __global__ void __launch_bounds__(kRowThreads, 1) row_cluster_kernel(const RowPa
   // With programmatic dependent launch this overlaps the scan's tail.
   for (int i = tid; i < kBins2; i += kRowThreads) sm.h2[i] = 0u;
   if (p.do_attn) load_q<D>(sm, p, r, 0, min(kHeads, p.H));
+  // The window rows do not depend on the selection: the window warp issues
+  // the copies of its first chunk now and waits for them when it attends.
+  bool win_issued = false;
+  if (p.do_attn && p.H > 0 && (tid >> 5) == kWinWarp) {
+    int64_t wrow0;
+    int nwin;
+    window_share<CL>(p, r, c, wrow0, nwin);
+    if (nwin > 0) {
+      issue_window_rows<D>(sm.win, p.win_k, p.win_v, wrow0, min(ar::kChunk, nwin));
+      win_issued = true;
+    }
+  }
   asm volatile("barrier.cluster.wait.aligned;" ::: "memory");
   pdl_wait_primary();  // the scores and histograms are complete from here on
   if (topk_here && tid == 0) {
@@ -583,11 +709,11 @@ __global__ void __launch_bounds__(kRowThreads, 1) row_cluster_kernel(const RowPa
                (uint32_t)(((n0 + 3) & ~3) * 4), &sm.bar);
   }
 
-  bool abort = false;
+  bool abort = false, idx_pending = false;
   uint32_t phases = 0;
   if (p.do_topk) {
     if (topk_here) {
-      row_topk<D, CL>(sm, p, cluster, r_local, r, K, bulk, s0, s1, abort, phases);
+      idx_pending = row_topk<D, CL>(sm, p, cluster, r_local, r, K, bulk, s0, s1, abort, phases);
     } else {
       if (c == 0) {
         int32_t *orow = p.idx + r * (int64_t)p.topk;
@@ -618,7 +744,8 @@ __global__ void __launch_bounds__(kRowThreads, 1) row_cluster_kernel(const RowPa
         __syncthreads();
         load_q<D>(sm, p, r, h0, nh);
       }
-      row_attend<D, CL>(sm, p, cluster, r, c, h0, nh, p.do_topk != 0, lo, hi, sel_base);
+      row_attend<D, CL>(sm, p, cluster, r, c, h0, nh, p.do_topk != 0, lo, hi, sel_base,
+                        win_issued && h0 == 0, idx_pending && h0 == 0, K);
     }
   }
   if (abort && tid == 0 && phases > 0)  // let a late bulk copy land before exit

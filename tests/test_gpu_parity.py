@@ -429,8 +429,10 @@ def _group_tensors(w0, layers):
     return tens
 
 
-def _run_group_and_compare(w0, rows=None):
+def _run_group_and_compare(w0, rows=None, mutate=None):
     layers = wl.all_layer_inputs(w0)
+    if mutate is not None:
+        mutate(layers)
     tens = _group_tensors(w0, layers)
     dims = csa2.make_dims(w0.B, w0.T, w0.H, w0.D, w0.N, w0.H_I, w0.d_I, w0.topk, w0.W,
                           w0.n_prior, w0.ratio)
@@ -469,6 +471,39 @@ def test_decode_layer_shapes(B, N, topk, W, H, D, H_I, d_I, decode_kernel):
     w0 = wl.with_sizes(wl.LONG, name=f"decode_{B}_{N}_{topk}", B=B, N=N, topk=topk, W=W, H=H,
                        D=D, H_I=H_I, d_I=d_I, seed=B * 1000 + N)
     _run_group_and_compare(w0)
+
+
+def test_decode_layer_heavy_ties(decode_kernel):
+    """Layers whose index scores take a few integer values (keys in {-1, 0, 1},
+    unit weights): the keys equal to the threshold outnumber the slots left,
+    so only the lowest-indexed of them are taken and each CTA's share depends
+    on the other ranks' counts before it attends."""
+    w0 = wl.with_sizes(wl.LONG, name="decode_ties", B=3, N=20000, seed=77)
+
+    def mutate(layers):
+        rng = np.random.default_rng(9)
+        layers[0]["k_idx"] = rng.integers(-1, 2, layers[0]["k_idx"].shape).astype(np.int8)
+        for lay in layers:
+            lay["q_idx"] = rng.integers(0, 2, lay["q_idx"].shape).astype(np.int8)
+            lay["w"][:] = 1.0
+
+    _run_group_and_compare(w0, mutate=mutate)
+
+
+def test_decode_layer_selection_crowded_into_one_slice(decode_kernel):
+    """A top-k of 6,000 whose entries all lie in the first 6,000 positions of
+    100,000: one CTA selects more than its on-chip list holds and attends over
+    the rest from the written output row."""
+    w0 = wl.with_sizes(wl.LONG, name="decode_crowded", B=1, N=100000, topk=6000, seed=78)
+
+    def mutate(layers):
+        k = layers[0]["k_idx"]
+        k[:, :6000] = np.abs(k[:, :6000]) // 2 + 60          # high keys first
+        k[:, 6000:] = k[:, 6000:] // 4                        # the rest small
+        for lay in layers:
+            lay["q_idx"] = np.abs(lay["q_idx"]) // 2 + 1      # positive queries
+
+    _run_group_and_compare(w0, mutate=mutate)
 
 
 def test_decode_layer_cuda_graph_replay(decode_kernel):
