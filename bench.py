@@ -85,6 +85,7 @@ def algorithmic_bytes(w0, key_format: str = "int8") -> dict:
 KERNEL_BYTES = {
     "index_scan": lambda w0, ab: w0.B * ab["keys"],
     "topk_attend": lambda w0, ab: w0.B * (ab["gather"] + ab["window"]),
+    "attend_handoff": lambda w0, ab: w0.B * (ab["gather"] + ab["window"]),
     "decode_fused": lambda w0, ab: w0.B * ab["total"],
 }
 
@@ -157,6 +158,7 @@ def pack_into_one_buffer(layers, keys, dev):
 KERNEL_SOURCES = {
     "index_scan": ("index_scan.cuh", "pack.cuh", "common.cuh"),
     "topk_attend": ("row_cluster.cuh", "attn_rows.cuh", "pack.cuh", "common.cuh"),
+    "attend_handoff": ("attn_handoff.cuh", "attn_rows.cuh", "common.cuh"),
     "decode_fused": ("decode_fused.cuh", "attn_rows.cuh", "pack.cuh", "common.cuh"),
 }
 

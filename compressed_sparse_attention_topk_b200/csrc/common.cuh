@@ -142,6 +142,39 @@ __device__ __forceinline__ void st_async_v2(void *dst, uint32_t a, uint32_t b, u
       : "memory");
 }
 
+// Arrive on the mbarrier at the offset of `bar` in CTA `rank` of the
+// cluster.  Relaxed: the arrival carries no data (the data these barriers
+// count travels by bulk copies, counted in bytes), so no earlier write of
+// the thread needs to be ordered before it (a release would wait for them).
+__device__ __forceinline__ void mbar_remote_arrive(uint64_t *bar, uint32_t rank) {
+  asm volatile("mbarrier.arrive.relaxed.cluster.shared::cluster.b64 _, [%0];" ::"r"(
+                   cluster_addr(bar, rank))
+               : "memory");
+}
+
+// Bulk copy (copy engine) of `bytes` from this CTA's shared memory at `src`
+// into CTA `rank`'s shared memory at the offset of `dst`, counted in bytes
+// on the mbarrier at the offset of `bar` in that CTA.  Addresses 16-byte
+// aligned, bytes a multiple of 16.  The copy reads `src` asynchronously:
+// the sender keeps `src` unchanged, and stays resident, until it knows the
+// bytes have landed.
+__device__ __forceinline__ void bulk_s2s_cluster(void *dst, const void *src, uint32_t bytes,
+                                                 uint64_t *bar, uint32_t rank) {
+  asm volatile(
+      "cp.async.bulk.shared::cluster.shared::cta.mbarrier::complete_tx::bytes [%0], [%1], %2, "
+      "[%3];" ::"r"(cluster_addr(dst, rank)),
+      "r"(smem_u32(src)), "r"(bytes), "r"(cluster_addr(bar, rank))
+      : "memory");
+}
+
+// Order this thread's earlier shared-memory writes before later reads of
+// them by bulk copies (the async proxy); every writing thread fences, then a
+// block barrier, then the copy is issued.
+__device__ __forceinline__ void fence_proxy_async_smem() {
+  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+
+
 // Wait for the given phase parity for at most ~2^32 cycles (about 2 s),
 // polling without suspension; on timeout record it in the status word and
 // return false.  The clock is read only once the phase is found incomplete:

@@ -9,6 +9,8 @@
 #include <cstdlib>
 #include <cstring>
 
+#include "attn_cluster.cuh"
+#include "attn_handoff.cuh"
 #include "attn_rows.cuh"
 #include "common.cuh"
 #include "decode_fused.cuh"
@@ -144,6 +146,26 @@ TopkWs topk_ws_layout(void *base, int64_t R, int64_t N) {
   return w;
 }
 
+// A decode layer's selection handed to the attention kernel (after the
+// top-k workspace): each selecting CTA's list [R][16][topk] and each
+// attention CTA's partial per head [R][16][H][D + 4].
+struct HandoffWs {
+  int32_t *lists;
+  float *part;
+  size_t bytes;
+};
+
+HandoffWs handoff_layout(void *base, int64_t R, int32_t topk, int32_t H, int32_t D) {
+  HandoffWs w{};
+  const size_t o_lists = 0;
+  const size_t o_part = align_up(size_t(R) * ah::kMaxG * topk * 4, 256);
+  w.bytes = o_part + align_up(size_t(R) * ah::kMaxG * H * (D + 4) * 4, 256);
+  char *p = static_cast<char *>(base);
+  w.lists = reinterpret_cast<int32_t *>(p + o_lists);
+  w.part = reinterpret_cast<float *>(p + o_part);
+  return w;
+}
+
 // Per-device one-time kernel attribute setup (dynamic shared memory above
 // 48 KiB, non-portable cluster size).  Must run before any stream capture;
 // the entry points call it on their first use on a device.
@@ -245,14 +267,15 @@ ScanLaunch pick_scan_group(int32_t d_I, int32_t H_I, int32_t T) {
 }
 
 // ---- the per-row cluster kernel -------------------------------------------
-template <int D, int CL>
+template <int D, int CL, bool HO = false>
 csa2_status launch_row_cl(const RowParams &p, int64_t nr, cudaStream_t st) {
   const size_t smem = sizeof(RowSmem<D>);
   static bool done[256] = {false};
   int dev = 0;
   cudaGetDevice(&dev);
   if (dev < 0 || dev >= 256 || !done[dev]) {
-    if (set_smem_attr(row_cluster_kernel<D, CL>, smem, CL > 8) != CSA2_OK) return CSA2_ERR_CUDA;
+    if (set_smem_attr(row_cluster_kernel<D, CL, HO>, smem, CL > 8) != CSA2_OK)
+      return CSA2_ERR_CUDA;
     if (dev >= 0 && dev < 256) done[dev] = true;
   }
   cudaLaunchConfig_t cfg = {};
@@ -270,8 +293,9 @@ csa2_status launch_row_cl(const RowParams &p, int64_t nr, cudaStream_t st) {
   attr[1].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = p.do_topk ? 2 : 1;
-  return cudaLaunchKernelEx(&cfg, row_cluster_kernel<D, CL>, p) == cudaSuccess ? CSA2_OK
-                                                                                : CSA2_ERR_CUDA;
+  return cudaLaunchKernelEx(&cfg, row_cluster_kernel<D, CL, HO>, p) == cudaSuccess
+             ? CSA2_OK
+             : CSA2_ERR_CUDA;
 }
 
 // Can clusters of 16 CTAs of the row kernel be scheduled on this device?
@@ -282,7 +306,7 @@ bool cluster16_ok() {
   cudaGetDevice(&dev);
   if (dev >= 0 && dev < 256 && cache[dev]) return cache[dev] == 1;
   const size_t smem = sizeof(RowSmem<D>);
-  bool ok = set_smem_attr(row_cluster_kernel<D, 16>, smem, true) == CSA2_OK;
+  bool ok = set_smem_attr(row_cluster_kernel<D, 16, false>, smem, true) == CSA2_OK;
   if (ok) {
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(16, 1, 1);
@@ -296,7 +320,8 @@ bool cluster16_ok() {
     cfg.attrs = attr;
     cfg.numAttrs = 1;
     int n = 0;
-    ok = cudaOccupancyMaxActiveClusters(&n, row_cluster_kernel<D, 16>, &cfg) == cudaSuccess &&
+    ok = cudaOccupancyMaxActiveClusters(&n, row_cluster_kernel<D, 16, false>, &cfg) ==
+             cudaSuccess &&
          n > 0;
   }
   cudaGetLastError();
@@ -316,6 +341,12 @@ int row_cluster_size(int64_t nr, int D) {
 csa2_status launch_row(const RowParams &p, int D, int64_t nr, cudaStream_t st) {
   TraceScope ts(p.do_topk ? (p.do_attn ? "topk_attend" : "topk_select") : "attend", st);
   const int cl = row_cluster_size(nr, D);
+  if (p.lists) {  // hand-off instances: 8 or fewer CTAs per row
+    if (p.do_attn || !p.do_topk || cl > 8) return CSA2_ERR_UNSUPPORTED;
+    if (D == 128)
+      return cl == 8 ? launch_row_cl<128, 8, true>(p, nr, st) : launch_row_cl<128, 4, true>(p, nr, st);
+    return cl == 8 ? launch_row_cl<64, 8, true>(p, nr, st) : launch_row_cl<64, 4, true>(p, nr, st);
+  }
   if (D == 128) {
     if (cl == 16) return launch_row_cl<128, 16>(p, nr, st);
     if (cl == 8) return launch_row_cl<128, 8>(p, nr, st);
@@ -324,6 +355,124 @@ csa2_status launch_row(const RowParams &p, int D, int64_t nr, cudaStream_t st) {
   if (cl == 16) return launch_row_cl<64, 16>(p, nr, st);
   if (cl == 8) return launch_row_cl<64, 8>(p, nr, st);
   return launch_row_cl<64, 4>(p, nr, st);
+}
+
+// ---- the per-row attention cluster kernel (attn_cluster.cuh) --------------
+template <int D, int CL>
+csa2_status launch_attn_cl(const ar::Params &a, int64_t nr, bool after_topk, cudaStream_t st) {
+  const size_t smem = sizeof(ac::Smem<D, CL>);
+  static bool done[256] = {false};
+  int dev = 0;
+  cudaGetDevice(&dev);
+  if (dev < 0 || dev >= 256 || !done[dev]) {
+    if (set_smem_attr(ac::attn_cluster_kernel<D, CL>, smem, CL > 8) != CSA2_OK)
+      return CSA2_ERR_CUDA;
+    if (dev >= 0 && dev < 256) done[dev] = true;
+  }
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3((unsigned)(nr * CL), 1, 1);
+  cfg.blockDim = dim3(ac::kThreads, 1, 1);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[2];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = CL;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  // After the selection, start early: the kernel loads the query and
+  // attends over the window, then waits for the selection's results itself.
+  attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[1].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = after_topk ? 2 : 1;
+  return cudaLaunchKernelEx(&cfg, ac::attn_cluster_kernel<D, CL>, a, after_topk ? 1 : 0) ==
+                 cudaSuccess
+             ? CSA2_OK
+             : CSA2_ERR_CUDA;
+}
+
+// Can clusters of 16 CTAs of the attention kernel be scheduled on this device?
+template <int D>
+bool attn_cluster16_ok() {
+  static int cache[256] = {0};  // 0 unknown, 1 yes, 2 no
+  int dev = 0;
+  cudaGetDevice(&dev);
+  if (dev >= 0 && dev < 256 && cache[dev]) return cache[dev] == 1;
+  const size_t smem = sizeof(ac::Smem<D, 16>);
+  bool ok = set_smem_attr(ac::attn_cluster_kernel<D, 16>, smem, true) == CSA2_OK;
+  if (ok) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(16, 1, 1);
+    cfg.blockDim = dim3(ac::kThreads, 1, 1);
+    cfg.dynamicSmemBytes = smem;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = 16;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    int n = 0;
+    ok = cudaOccupancyMaxActiveClusters(&n, ac::attn_cluster_kernel<D, 16>, &cfg) == cudaSuccess &&
+         n > 0;
+  }
+  cudaGetLastError();
+  if (dev >= 0 && dev < 256) cache[dev] = ok ? 1 : 2;
+  return ok;
+}
+
+// Attention of nr decode rows (a.row0 ...): CTAs per row as for the
+// selection (about two CTAs per SM in total); after_topk: launched right
+// after the selection of the same rows, with programmatic dependent launch.
+csa2_status launch_attn_cluster(const ar::Params &a, int D, int64_t nr, bool after_topk,
+                                cudaStream_t st) {
+  TraceScope ts("attend", st);
+  const int64_t target = 2 * int64_t(device_sms());
+  int cl = 4;
+  if (nr * 8 <= target) cl = 8;
+  if (nr * 16 <= target && (D == 128 ? attn_cluster16_ok<128>() : attn_cluster16_ok<64>()))
+    cl = 16;
+  if (D == 128) {
+    if (cl == 16) return launch_attn_cl<128, 16>(a, nr, after_topk, st);
+    if (cl == 8) return launch_attn_cl<128, 8>(a, nr, after_topk, st);
+    return launch_attn_cl<128, 4>(a, nr, after_topk, st);
+  }
+  if (cl == 16) return launch_attn_cl<64, 16>(a, nr, after_topk, st);
+  if (cl == 8) return launch_attn_cl<64, 8>(a, nr, after_topk, st);
+  return launch_attn_cl<64, 4>(a, nr, after_topk, st);
+}
+
+// ---- the attention kernel fed by the selection (attn_handoff.cuh) ---------
+template <int D>
+csa2_status launch_attn_handoff_d(const ah::Params &hp, int64_t nr, cudaStream_t st) {
+  const size_t smem = sizeof(ah::Smem<D>);
+  static bool done[256] = {false};
+  int dev = 0;
+  cudaGetDevice(&dev);
+  if (dev < 0 || dev >= 256 || !done[dev]) {
+    if (set_smem_attr(ah::attn_handoff_kernel<D>, smem, false) != CSA2_OK) return CSA2_ERR_CUDA;
+    if (dev >= 0 && dev < 256) done[dev] = true;
+  }
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3((unsigned)(nr * hp.G), 1, 1);
+  cfg.blockDim = dim3(ah::kThreads, 1, 1);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  // Start early (programmatic dependent launch): the kernel loads the query
+  // and attends over the window, then waits for each list's ready flag.
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, ah::attn_handoff_kernel<D>, hp) == cudaSuccess ? CSA2_OK
+                                                                                  : CSA2_ERR_CUDA;
+}
+
+csa2_status launch_attn_handoff(const ah::Params &hp, int D, int64_t nr, cudaStream_t st) {
+  TraceScope ts("attend_handoff", st);
+  if (hp.G < 1 || hp.G > ah::kMaxG || hp.G > kHandoffFlags) return CSA2_ERR_UNSUPPORTED;
+  return D == 128 ? launch_attn_handoff_d<128>(hp, nr, st) : launch_attn_handoff_d<64>(hp, nr, st);
 }
 
 csa2_status check_topk_args(const int8_t *q_idx, const float *w, const int8_t *k_idx, int32_t B,
@@ -988,6 +1137,18 @@ csa2_status run_index_topk(const int8_t *q_idx, const float *w, const int8_t *k_
   const int64_t bstride = (nbk + 3) & ~int64_t(3);
   if (pr && cudaMemsetAsync(pr->X.bhist, 0, size_t(B) * kHistStride * 4, st) != cudaSuccess)
     return CSA2_ERR_CUDA;
+  // Attention after the selection.  With many rows per launch (8 or fewer
+  // selecting CTAs per row) a separate kernel fed by each selecting CTA's
+  // list, its CTAs' partials merged by the row's last CTA (a few partials
+  // per row), when the workspace holds the lists (layer calls size it so);
+  // with few rows (16 CTAs per row) the per-row cluster kernel attends
+  // itself and merges its 16 partials on chip.
+  const bool handoff_ok =
+      att && topk <= kSelCap && att->H > 0 &&
+      ws_bytes >= L0.bytes + handoff_layout(nullptr, R0, topk, att->H, att->D).bytes;
+  const HandoffWs Hw = handoff_ok ? handoff_layout(static_cast<char *>(ws) + L0.bytes, R0, topk,
+                                                   att->H, att->D)
+                                  : HandoffWs{};
 
   for (int64_t row0 = 0; row0 < rows; row0 += R) {
     const int64_t nr = std::min<int64_t>(R, rows - row0);
@@ -1027,21 +1188,51 @@ csa2_status run_index_topk(const int8_t *q_idx, const float *w, const int8_t *k_
     p.idx = idx_out;
     p.do_topk = 1;
     int D = 64;
+    const bool handoff = handoff_ok && row_cluster_size(nr, att->D) <= 8;
     if (att) {
-      p.q = att->q;
       p.codes = att->codes;
       p.scales = att->scales;
-      p.win_k = att->win_k;
-      p.win_v = att->win_v;
-      p.H = att->H;
-      p.W = att->W;
-      p.q_scale = att->sm_scale * 1.4426950408889634f;
-      p.out = att->out;
-      p.lse = att->lse;
-      p.do_attn = 1;
       D = att->D;
+      if (handoff) {  // each CTA's selection goes to the attention kernel
+        p.lists = Hw.lists;
+        p.list_stride = topk;
+      } else {  // attention in the same kernel
+        p.q = att->q;
+        p.win_k = att->win_k;
+        p.win_v = att->win_v;
+        p.H = att->H;
+        p.W = att->W;
+        p.q_scale = att->sm_scale * 1.4426950408889634f;
+        p.out = att->out;
+        p.lse = att->lse;
+        p.do_attn = 1;
+      }
     }
     if (launch_row(p, D, nr, st) != CSA2_OK) return CSA2_ERR_CUDA;
+    if (handoff) {  // the attention of these rows, overlapping the selection
+      ah::Params hp{};
+      hp.a.q = att->q;
+      hp.a.codes = att->codes;
+      hp.a.scales = att->scales;
+      hp.a.win_k = att->win_k;
+      hp.a.win_v = att->win_v;
+      hp.a.N = N;
+      hp.a.T = T;
+      hp.a.H = att->H;
+      hp.a.W = att->W;
+      hp.a.topk = topk;
+      hp.a.q_scale = att->sm_scale * 1.4426950408889634f;
+      hp.a.out = att->out;
+      hp.a.lse = att->lse;
+      hp.a.row0 = row0;
+      hp.lists = Hw.lists;
+      hp.list_stride = topk;
+      hp.flags = L.hist1 + kBins1;
+      hp.flag_stride = kHistStride;
+      hp.part = Hw.part;
+      hp.G = row_cluster_size(nr, D);
+      if (launch_attn_handoff(hp, D, nr, st) != CSA2_OK) return CSA2_ERR_CUDA;
+    }
     if (pr) {  // block maxima of these rows' scores, before the next pass reuses them
       TraceScope ts("pool_block_max", st);
       block_max_kernel<<<dim3((unsigned)ceil_div(nbk, kPoolThreads), (unsigned)nr), kPoolThreads,
@@ -1309,29 +1500,25 @@ csa2_status run_attn(const uint16_t *q, const uint8_t *codes, const float *scale
     }
     return CSA2_OK;
   }
-  RowParams p{};
-  p.N = N;
-  p.T = T;
-  p.n_prior = -1;
-  p.ratio = 1;
-  p.topk = topk;
-  p.idx = const_cast<int32_t *>(idx);
-  p.q = q;
-  p.codes = codes;
-  p.scales = scales;
-  p.win_k = win_k;
-  p.win_v = win_v;
-  p.H = H;
-  p.W = W;
-  p.q_scale = sm_scale * 1.4426950408889634f;
-  p.out = out;
-  p.lse = lse;
-  p.do_topk = 0;
-  p.do_attn = 1;
+  ar::Params a{};
+  a.q = q;
+  a.codes = codes;
+  a.scales = scales;
+  a.idx = idx;
+  a.win_k = win_k;
+  a.win_v = win_v;
+  a.N = N;
+  a.T = T;
+  a.H = H;
+  a.W = W;
+  a.topk = topk;
+  a.q_scale = sm_scale * 1.4426950408889634f;
+  a.out = out;
+  a.lse = lse;
   for (int64_t row0 = 0; row0 < rows; row0 += kAttnRowsPerLaunch) {
     const int64_t nr = std::min<int64_t>(kAttnRowsPerLaunch, rows - row0);
-    p.row0 = row0;
-    if (launch_row(p, D, nr, st) != CSA2_OK) return CSA2_ERR_CUDA;
+    a.row0 = row0;
+    if (launch_attn_cluster(a, D, nr, false, st) != CSA2_OK) return CSA2_ERR_CUDA;
   }
   return CSA2_OK;
 }
@@ -1372,9 +1559,17 @@ PoolExt pool_ext_layout(void *base, int64_t B, int64_t N, int32_t block, int32_t
 }
 
 // The pool regions start after the largest scan / fused-kernel workspace.
+// Workspace of a layer's selection and its hand-off to the attention
+// kernel (the top-k regions, then the lists and partials).
+size_t handoff_ws_bytes(const csa2_dims *d) {
+  const int64_t R = topk_rows_per_pass(int64_t(d->B) * d->T, d->N);
+  return topk_ws_layout(nullptr, R, d->N).bytes +
+         handoff_layout(nullptr, R, d->topk, d->H, d->D).bytes;
+}
+
 size_t pool_ext_offset(const csa2_dims *d) {
   return align_up(std::max(fused_ws_bytes(int64_t(d->B) * d->T, d->N),
-                           topk_ws_bytes(d->B, d->T, d->N)),
+                           handoff_ws_bytes(d)),
                   256);
 }
 
@@ -1672,6 +1867,7 @@ size_t csa2_layer_group_workspace_size(const csa2_dims *d) {
   if (!d) return 0;
   if (d->B < 0 || d->T < 0 || d->H < 1 || (d->D != 64 && d->D != 128) || d->W < 0) return 0;
   size_t bytes = csa2_index_topk_workspace_size(d->B, d->T, d->H_I, d->d_I, d->N, d->topk);
+  if (bytes) bytes = std::max(bytes, handoff_ws_bytes(d));
   if (bytes && (d->pool_block || d->pool_blocks)) {
     if (!pool_dims_ok(d)) return 0;
     bytes = std::max(bytes, pool_ext_offset(d) + pool_ext_layout(nullptr, d->B, d->N,

@@ -26,9 +26,12 @@
 namespace csa2 {
 
 constexpr int kScanThreads = 256;
-// Per-row histogram rows in global memory: kBins1 counters (zeroed before
-// the scan), padded to keep rows 16-byte aligned.
-constexpr int kHistStride = kBins1 + 4;
+// Words per row of the digit-1 histogram region: the 2,048 bins, then (for
+// a selection handed to a following attention kernel) one ready flag per
+// selecting CTA and a done counter of the row's attention CTAs, all cleared
+// with the bins before each scan.
+constexpr int kHandoffFlags = 16;  // selecting CTAs per row, at most
+constexpr int kHistStride = kBins1 + 32;
 
 // Index key formats: int8, or FP4 (E2M1 codes with one power-of-two scale
 // per 32 elements: d_I/2 code bytes + d_I/32 exponent bytes per key, see

@@ -106,7 +106,30 @@ struct RowParams {
   float *out;               // [rows_global, H, D]
   float *lse;               // [rows_global, H] or null
   int do_topk, do_attn;
+  // hand-off to an attention kernel launched after this one (top-k only,
+  // the kernel's HO instances):
+  // CTA c of row r_local writes its selected indices (ascending) to
+  // lists[(r_local * CL + c) * list_stride ...] and then n + 1 into the
+  // ready flag hist1[r_local * kHistStride + kBins1 + c]; null: no hand-off
+  int32_t *lists;
+  int64_t list_stride;
 };
+
+// Publish this CTA's selection (sel[0..n), ascending) to the attention
+// kernel that follows: the indices, then (one thread, after a fence at GPU
+// scope) the ready flag n + 1.
+template <int CL, class S>
+__device__ void publish_selection(S &sm, const RowParams &p, int64_t r_local, int c,
+                                  uint32_t n) {
+  int32_t *dst = p.lists + (r_local * CL + c) * p.list_stride;
+  for (uint32_t i = threadIdx.x; i < n; i += kRowThreads) dst[i] = sm.sel[i];
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    uint32_t *flag = const_cast<uint32_t *>(p.hist1) + r_local * kHistStride + kBins1 + c;
+    __threadfence();
+    asm volatile("st.release.gpu.global.u32 [%0], %1;" ::"l"(flag), "r"(n + 1u) : "memory");
+  }
+}
 
 template <int D>
 struct RowSmem {
@@ -218,7 +241,7 @@ __device__ void cluster_threshold(RowSmem<D> &sm, cg::cluster_group &cluster, ui
 // depend on the other ranks' counts and attention may start at once; the
 // counts exchange and the index write are then left to the warps that do not
 // attend (write_row_indices).
-template <int D, int CL>
+template <int D, int CL, bool HO>
 __device__ bool row_topk(RowSmem<D> &sm, const RowParams &p, cg::cluster_group &cluster,
                          int64_t r_local, int64_t r, int64_t K, bool bulk, int64_t s0, int64_t s1,
                          bool &abort, uint32_t &phase) {
@@ -354,7 +377,8 @@ __device__ bool row_topk(RowSmem<D> &sm, const RowParams &p, cg::cluster_group &
   // keys equal to the threshold key as are still needed): the selection is
   // the above-threshold and tied candidates, in index order.
   const bool ties_all = !need3 || sm.thr[4] <= r3;
-  if (p.do_attn && ties_all && tot_above + tot_tie <= (uint32_t)kSelCap) {
+  const bool early = ties_all && tot_above + tot_tie <= (uint32_t)kSelCap;
+  if ((HO || p.do_attn) && early) {
     uint32_t at = above_before + tie_before;
     for (uint32_t i = i0; i < i1; ++i) {
       const uint2 e = cand_at(i);
@@ -365,7 +389,13 @@ __device__ bool row_topk(RowSmem<D> &sm, const RowParams &p, cg::cluster_group &
       sm.sel_count = tot_above + tot_tie;
     }
     __syncthreads();
-    return true;
+    if constexpr (!HO) {
+      return true;
+    } else {
+      // hand-off: the selection goes to the attention kernel now, the
+      // ordered output row once every rank's counts are in
+      publish_selection<CL>(sm, p, r_local, c, tot_above + tot_tie);
+    }
   }
   // wait for every rank's counts
   if (!mbar_wait_cluster_bounded(&sm.xbar[4], 0)) abort = true;
@@ -406,6 +436,9 @@ __device__ bool row_topk(RowSmem<D> &sm, const RowParams &p, cg::cluster_group &
     for (int64_t i = K + tid; i < p.topk; i += kRowThreads) orow[i] = -1;
   if (tid == 0) sm.sel_base = sm.out_base;
   __syncthreads();
+  if constexpr (HO) {  // hand-off of a selection that needed every rank's counts
+    if (!early) publish_selection<CL>(sm, p, r_local, c, min(sm.sel_count, (uint32_t)kSelCap));
+  }
   return false;
 }
 
@@ -653,11 +686,18 @@ __device__ void row_attend(RowSmem<D> &sm, const RowParams &p, cg::cluster_group
   }
 }
 
-template <int D, int CL>
+// HO: the top-k hands each CTA's selection to an attention kernel launched
+// after this one (p.lists, no attention here); its code is compiled only
+// into those instances.
+template <int D, int CL, bool HO>
 __global__ void __launch_bounds__(kRowThreads, 1) row_cluster_kernel(const RowParams p) {
   extern __shared__ __align__(128) unsigned char row_smem_raw[];
   RowSmem<D> &sm = *reinterpret_cast<RowSmem<D> *>(row_smem_raw);
   cg::cluster_group cluster = cg::this_cluster();
+  // with a hand-off, the attention kernel launched after this one with
+  // programmatic dependent launch may start now; it waits for each list's
+  // ready flag itself
+  if constexpr (HO) pdl_allow_dependents();
   const int tid = threadIdx.x;
   const int c = (int)cluster.block_rank();
   const int64_t r_local = blockIdx.x / CL, r = p.row0 + r_local;
@@ -713,7 +753,8 @@ __global__ void __launch_bounds__(kRowThreads, 1) row_cluster_kernel(const RowPa
   uint32_t phases = 0;
   if (p.do_topk) {
     if (topk_here) {
-      idx_pending = row_topk<D, CL>(sm, p, cluster, r_local, r, K, bulk, s0, s1, abort, phases);
+      idx_pending =
+          row_topk<D, CL, HO>(sm, p, cluster, r_local, r, K, bulk, s0, s1, abort, phases);
     } else {
       if (c == 0) {
         int32_t *orow = p.idx + r * (int64_t)p.topk;
@@ -723,6 +764,7 @@ __global__ void __launch_bounds__(kRowThreads, 1) row_cluster_kernel(const RowPa
         sm.sel_base = 0;
         sm.sel_count = 0;
       }
+      if constexpr (HO) publish_selection<CL>(sm, p, r_local, c, 0u);
     }
     // Attention reads this CTA's own selection from shared memory, so no
     // cluster barrier is needed between top-k and attention.
