@@ -135,10 +135,9 @@ def test_topk_heavy_ties_at_boundary(levels):
 
 def test_topk_crowded_into_few_slices():
     # The top-k sits in the last 3,000 entries (their head-0 dot product is
-    # |q_0|^2), i.e. in the last one or two slices of the row: those slices
-    # hold nearly every selected entry (the per-row cluster kernel's CTAs
-    # and the fused kernel's candidate lists are far from balanced), and the
-    # output offsets of the other slices are all zero.
+    # |q_0|^2), i.e. in the last one or two of the row's slices: the per-row
+    # cluster kernel's last CTAs select nearly every entry while the others
+    # select none, so the output offsets of the other slices are all zero.
     q, w, k = _index_case(2, 1, 4, 64, 60000, seed=11)
     for b in range(2):
         k[b, -3000:, :] = q[b, 0, 0, :]
@@ -146,9 +145,10 @@ def test_topk_crowded_into_few_slices():
 
 
 @pytest.mark.parametrize("N", [4096, 70000, 262144])
-def test_topk_candidate_lists_many_slices(N):
-    # one row split into many slices (up to one per SM): the selection meets
-    # the candidates of every slice in index order
+def test_topk_one_row_many_scan_slices(N):
+    # one row scanned by many CTAs (about two per SM), whose digit-1
+    # histograms the selection sums; at N = 262,144 each of the row
+    # kernel's 16 CTAs selects from 16,384 staged scores
     q, w, k = _index_case(1, 1, 4, 64, N, seed=N)
     _check_index(q, w, k, 2048)
 
