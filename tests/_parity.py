@@ -1,10 +1,12 @@
 """Helpers shared by the GPU parity tests: host->device marshalling of the
-seeded inputs, each side's own FP4 store, and the tolerance check."""
+seeded inputs, each side's own FP4 store, the tolerance check and the
+layer-group comparison against the oracle's layer walk."""
 import numpy as np
 import torch
 
 import oracle
 import compressed_sparse_attention_topk_b200 as csa2
+from compressed_sparse_attention_topk_b200 import workloads as wl
 
 # Attention agreement: |gpu - oracle| <= ATOL + RTOL * |oracle| (fp32 accumulation
 # against the fp64 oracle).
@@ -65,3 +67,51 @@ def use_decode_kernel(kernel):
     prev = csa2.get_decode_kernel()
     csa2.set_decode_kernel(kernel)
     return prev
+
+
+def group_tensors(w0, layers):
+    """Device tensors of a layer group's inputs (each Full layer's FP4 store
+    packed on the GPU) and its outputs."""
+    tens = []
+    for l, lay in enumerate(layers):
+        d = {k: dev(v) for k, v in lay.items() if k != "entries"}
+        d["q"] = d["q"] if w0.T > 1 else d["q"][:, 0].contiguous()
+        if "entries" in lay:
+            d["codes"], d["scales"] = gpu_store(lay["entries"])
+        d["idx"] = torch.empty((w0.B, w0.T, w0.topk), dtype=torch.int32, device="cuda")
+        shape = (w0.B, w0.T, w0.H) if w0.T > 1 else (w0.B, w0.H)
+        d["out"] = torch.empty(shape + (w0.D,), dtype=torch.float32, device="cuda")
+        d["lse"] = torch.empty(shape, dtype=torch.float32, device="cuda")
+        tens.append(d)
+    return tens
+
+
+def run_group_and_compare(w0, rows=None, mutate=None):
+    """The layer group of workload w0 through the layer call against the
+    oracle's layer walk: indices bit-exact, out and lse within tolerance;
+    `mutate` edits the seeded inputs first, `rows` restricts the comparison."""
+    layers = wl.all_layer_inputs(w0)
+    if mutate is not None:
+        mutate(layers)
+    tens = group_tensors(w0, layers)
+    dims = csa2.make_dims(w0.B, w0.T, w0.H, w0.D, w0.N, w0.H_I, w0.d_I, w0.topk, w0.W,
+                          w0.n_prior, w0.ratio)
+    csa2.layer_group_run(list(w0.modes), tens, dims)
+    for lay in layers:
+        if "entries" in lay:
+            lay["codes"], lay["scales"] = oracle_store(lay["entries"])
+    ref = oracle.layer_group(list(w0.modes), layers, w0.topk, w0.n_prior, w0.ratio, rows=rows)
+    for l, (mode, kv, ix) in enumerate(w0.modes):
+        g_idx = host(tens[ix]["idx"]).reshape(w0.B * w0.T, w0.topk)
+        o_idx = ref[l]["idx"].reshape(w0.B * w0.T, w0.topk)
+        if rows is not None:
+            g_idx, o_idx = g_idx[rows], o_idx[rows]
+        assert_bits_equal(g_idx, o_idx, f"layer {l} idx")
+        out = host(tens[l]["out"]).reshape(w0.B * w0.T, w0.H, w0.D)
+        lse = host(tens[l]["lse"]).reshape(w0.B * w0.T, w0.H)
+        if rows is not None:
+            out, lse = out[rows], lse[rows]
+        assert_close(out, ref[l]["out"], f"layer {l} out")
+        assert_close(lse, ref[l]["lse"], f"layer {l} lse")
+    assert csa2.get_device_status() == 0
+    return tens

@@ -11,7 +11,8 @@ import compressed_sparse_attention_topk_b200 as csa2
 from compressed_sparse_attention_topk_b200 import build as csa2_build
 from compressed_sparse_attention_topk_b200 import workloads as wl
 from tests._parity import (DECODE_KERNELS, assert_bits_equal, assert_close, dev, gpu_store,
-                           host, oracle_store, use_decode_kernel)
+                           group_tensors, host, oracle_store, run_group_and_compare,
+                           use_decode_kernel)
 
 pytestmark = pytest.mark.gpu
 
@@ -280,7 +281,7 @@ def test_multi_query_shared_scan_visibility():
 def test_multi_token_decode_workload_full_size():
     """5 query tokens per sequence at the 1M-context shape (B=4, N=262,144,
     Full + Reindex): shared scans, per-row top-k, attention; every row."""
-    _run_group_and_compare(wl.MTP5)
+    run_group_and_compare(wl.MTP5)
 
 
 @pytest.mark.parametrize("wl_name", ["tiny_decode_n1024", "decode_b32_n131072"])
@@ -414,49 +415,6 @@ def test_tiny_workload_end_to_end():
     assert_close(host(lse), ref_lse, "lse")
 
 
-def _group_tensors(w0, layers):
-    tens = []
-    for l, lay in enumerate(layers):
-        d = {k: dev(v) for k, v in lay.items() if k != "entries"}
-        d["q"] = d["q"] if w0.T > 1 else d["q"][:, 0].contiguous()
-        if "entries" in lay:
-            d["codes"], d["scales"] = gpu_store(lay["entries"])
-        d["idx"] = torch.empty((w0.B, w0.T, w0.topk), dtype=torch.int32, device="cuda")
-        shape = (w0.B, w0.T, w0.H) if w0.T > 1 else (w0.B, w0.H)
-        d["out"] = torch.empty(shape + (w0.D,), dtype=torch.float32, device="cuda")
-        d["lse"] = torch.empty(shape, dtype=torch.float32, device="cuda")
-        tens.append(d)
-    return tens
-
-
-def _run_group_and_compare(w0, rows=None, mutate=None):
-    layers = wl.all_layer_inputs(w0)
-    if mutate is not None:
-        mutate(layers)
-    tens = _group_tensors(w0, layers)
-    dims = csa2.make_dims(w0.B, w0.T, w0.H, w0.D, w0.N, w0.H_I, w0.d_I, w0.topk, w0.W,
-                          w0.n_prior, w0.ratio)
-    csa2.layer_group_run(list(w0.modes), tens, dims)
-    for lay in layers:
-        if "entries" in lay:
-            lay["codes"], lay["scales"] = oracle_store(lay["entries"])
-    ref = oracle.layer_group(list(w0.modes), layers, w0.topk, w0.n_prior, w0.ratio, rows=rows)
-    for l, (mode, kv, ix) in enumerate(w0.modes):
-        g_idx = host(tens[ix]["idx"]).reshape(w0.B * w0.T, w0.topk)
-        o_idx = ref[l]["idx"].reshape(w0.B * w0.T, w0.topk)
-        if rows is not None:
-            g_idx, o_idx = g_idx[rows], o_idx[rows]
-        assert_bits_equal(g_idx, o_idx, f"layer {l} idx")
-        out = host(tens[l]["out"]).reshape(w0.B * w0.T, w0.H, w0.D)
-        lse = host(tens[l]["lse"]).reshape(w0.B * w0.T, w0.H)
-        if rows is not None:
-            out, lse = out[rows], lse[rows]
-        assert_close(out, ref[l]["out"], f"layer {l} out")
-        assert_close(lse, ref[l]["lse"], f"layer {l} lse")
-    assert csa2.get_device_status() == 0
-    return tens
-
-
 @pytest.mark.parametrize("B,N,topk,W,H,D,H_I,d_I", [
     (2, 5000, 2048, 128, 16, 128, 4, 64),
     (3, 1000, 2048, 128, 16, 128, 4, 64),     # fewer entries than k: padding
@@ -470,7 +428,7 @@ def test_decode_layer_shapes(B, N, topk, W, H, D, H_I, d_I, decode_kernel):
     kernel): selection bit-exact, attention within tolerance."""
     w0 = wl.with_sizes(wl.LONG, name=f"decode_{B}_{N}_{topk}", B=B, N=N, topk=topk, W=W, H=H,
                        D=D, H_I=H_I, d_I=d_I, seed=B * 1000 + N)
-    _run_group_and_compare(w0)
+    run_group_and_compare(w0)
 
 
 def test_decode_layer_heavy_ties(decode_kernel):
@@ -487,7 +445,7 @@ def test_decode_layer_heavy_ties(decode_kernel):
             lay["q_idx"] = rng.integers(0, 2, lay["q_idx"].shape).astype(np.int8)
             lay["w"][:] = 1.0
 
-    _run_group_and_compare(w0, mutate=mutate)
+    run_group_and_compare(w0, mutate=mutate)
 
 
 def test_decode_layer_selection_crowded_into_one_slice(decode_kernel):
@@ -503,7 +461,7 @@ def test_decode_layer_selection_crowded_into_one_slice(decode_kernel):
         for lay in layers:
             lay["q_idx"] = np.abs(lay["q_idx"]) // 2 + 1      # positive queries
 
-    _run_group_and_compare(w0, mutate=mutate)
+    run_group_and_compare(w0, mutate=mutate)
 
 
 def test_decode_layer_cuda_graph_replay(decode_kernel):
@@ -511,7 +469,7 @@ def test_decode_layer_cuda_graph_replay(decode_kernel):
     and replayed gives the eager results, bit for bit, on every replay."""
     w0 = wl.with_sizes(wl.LONG, name="graph_replay", B=4, N=20000, seed=77)
     layers = wl.all_layer_inputs(w0)
-    tens = _group_tensors(w0, layers)
+    tens = group_tensors(w0, layers)
     dims = csa2.make_dims(w0.B, w0.T, w0.H, w0.D, w0.N, w0.H_I, w0.d_I, w0.topk, w0.W)
     group = csa2.LayerGroup(list(w0.modes), tens, dims)
     group.run()
@@ -540,19 +498,19 @@ def test_decode_layer_cuda_graph_replay(decode_kernel):
 def test_group_workload_16_layers():
     """4 groups of (Full, Reindex, Reuse, Reuse), B=8, N=4096, k=512."""
     w0 = wl.GROUP
-    tens = _run_group_and_compare(w0)
+    tens = run_group_and_compare(w0)
     assert csa2.group_cache_bytes(list(w0.modes), w0.N, 128, 8) == 2 * 1024 * 1024
 
 
 def test_long_decode_workload_full_size(decode_kernel):
     """The 1M-token decode workload at full size (B=4, N=262144, Full +
     Reindex), in the launch configuration the benchmark times."""
-    _run_group_and_compare(wl.LONG)
+    run_group_and_compare(wl.LONG)
 
 
 def test_decode_workload_full_size():
     """B=32, N=131072, d_I=32, k=2048, with salient outlier entries."""
-    _run_group_and_compare(wl.DECODE)
+    run_group_and_compare(wl.DECODE)
 
 
 def test_prefill_workload_sampled_rows():
@@ -564,4 +522,4 @@ def test_prefill_workload_sampled_rows():
     rng = np.random.default_rng(1234)
     rows = np.unique(np.concatenate([np.arange(64), np.arange(w0.T - 64, w0.T),
                                      rng.choice(w0.T, 128, replace=False)])).astype(np.int64)
-    _run_group_and_compare(w0, rows=rows)
+    run_group_and_compare(w0, rows=rows)
