@@ -32,11 +32,14 @@ inline cudaStream_t as_stream(void *s) { return reinterpret_cast<cudaStream_t>(s
 int device_sms() {
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess) return 148;
-  static int cache[256] = {0};
-  if (dev >= 0 && dev < 256 && cache[dev]) return cache[dev];
+  static std::atomic<int> cache[256];  // per device: 0 unknown
+  if (dev >= 0 && dev < 256) {
+    const int c = cache[dev].load(std::memory_order_relaxed);
+    if (c) return c;
+  }
   int v = 148;
   if (cudaDeviceGetAttribute(&v, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) v = 148;
-  if (dev >= 0 && dev < 256) cache[dev] = v;
+  if (dev >= 0 && dev < 256) cache[dev].store(v, std::memory_order_relaxed);
   return v;
 }
 
@@ -188,12 +191,12 @@ void launch_scan_kf(dim3 grid, cudaStream_t st, const int8_t *q_idx, const float
                     int64_t n_prior, int32_t ratio, int64_t row0, float *scores, int64_t stride,
                     uint32_t *hist1, int write_masked) {
   using S = ScanShape<DI, HI, KF>;
-  static bool done[256] = {false};
+  static std::atomic<bool> done[256];  // per device: attributes set
   int dev = 0;
   cudaGetDevice(&dev);
-  if (dev < 0 || dev >= 256 || !done[dev]) {
+  if (dev < 0 || dev >= 256 || !done[dev].load(std::memory_order_acquire)) {
     set_smem_attr(index_scan_kernel<DI, HI, KF>, S::SMEM, false);
-    if (dev >= 0 && dev < 256) done[dev] = true;
+    if (dev >= 0 && dev < 256) done[dev].store(true, std::memory_order_release);
   }
   index_scan_kernel<DI, HI, KF><<<grid, kScanThreads, S::SMEM, st>>>(
       q_idx, w, k_idx, k_exps, T, N, n_prior, ratio, row0, scores, stride, hist1, write_masked);
@@ -238,12 +241,12 @@ void launch_scan_group(dim3 grid, cudaStream_t st, const int8_t *q_idx, const fl
                        int64_t row0, float *scores, int64_t stride, uint32_t *hist1,
                        int write_masked) {
   using S = ScanGroupShape<DI, HI, TQ>;
-  static bool done[256] = {false};
+  static std::atomic<bool> done[256];  // per device: attributes set
   int dev = 0;
   cudaGetDevice(&dev);
-  if (dev < 0 || dev >= 256 || !done[dev]) {
+  if (dev < 0 || dev >= 256 || !done[dev].load(std::memory_order_acquire)) {
     set_smem_attr(index_scan_group_kernel<DI, HI, TQ>, S::SMEM, false);
-    if (dev >= 0 && dev < 256) done[dev] = true;
+    if (dev >= 0 && dev < 256) done[dev].store(true, std::memory_order_release);
   }
   index_scan_group_kernel<DI, HI, TQ><<<grid, S::THREADS, S::SMEM, st>>>(
       q_idx, w, k_idx, T, N, n_prior, ratio, row0, scores, stride, hist1, write_masked);
@@ -270,13 +273,13 @@ ScanLaunch pick_scan_group(int32_t d_I, int32_t H_I, int32_t T) {
 template <int D, int CL, bool HO = false>
 csa2_status launch_row_cl(const RowParams &p, int64_t nr, cudaStream_t st) {
   const size_t smem = sizeof(RowSmem<D>);
-  static bool done[256] = {false};
+  static std::atomic<bool> done[256];  // per device: attributes set
   int dev = 0;
   cudaGetDevice(&dev);
-  if (dev < 0 || dev >= 256 || !done[dev]) {
+  if (dev < 0 || dev >= 256 || !done[dev].load(std::memory_order_acquire)) {
     if (set_smem_attr(row_cluster_kernel<D, CL, HO>, smem, CL > 8) != CSA2_OK)
       return CSA2_ERR_CUDA;
-    if (dev >= 0 && dev < 256) done[dev] = true;
+    if (dev >= 0 && dev < 256) done[dev].store(true, std::memory_order_release);
   }
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3((unsigned)(nr * CL), 1, 1);
@@ -301,10 +304,11 @@ csa2_status launch_row_cl(const RowParams &p, int64_t nr, cudaStream_t st) {
 // Can clusters of 16 CTAs of the row kernel be scheduled on this device?
 template <int D>
 bool cluster16_ok() {
-  static int cache[256] = {0};  // 0 unknown, 1 yes, 2 no
+  static std::atomic<int> cache[256];  // per device: 0 unknown, 1 yes, 2 no
   int dev = 0;
   cudaGetDevice(&dev);
-  if (dev >= 0 && dev < 256 && cache[dev]) return cache[dev] == 1;
+  if (dev >= 0 && dev < 256 && cache[dev].load(std::memory_order_relaxed))
+    return cache[dev].load(std::memory_order_relaxed) == 1;
   const size_t smem = sizeof(RowSmem<D>);
   bool ok = set_smem_attr(row_cluster_kernel<D, 16, false>, smem, true) == CSA2_OK;
   if (ok) {
@@ -325,7 +329,7 @@ bool cluster16_ok() {
          n > 0;
   }
   cudaGetLastError();
-  if (dev >= 0 && dev < 256) cache[dev] = ok ? 1 : 2;
+  if (dev >= 0 && dev < 256) cache[dev].store(ok ? 1 : 2, std::memory_order_relaxed);
   return ok;
 }
 
@@ -361,13 +365,13 @@ csa2_status launch_row(const RowParams &p, int D, int64_t nr, cudaStream_t st) {
 template <int D, int CL>
 csa2_status launch_attn_cl(const ar::Params &a, int64_t nr, bool after_topk, cudaStream_t st) {
   const size_t smem = sizeof(ac::Smem<D, CL>);
-  static bool done[256] = {false};
+  static std::atomic<bool> done[256];  // per device: attributes set
   int dev = 0;
   cudaGetDevice(&dev);
-  if (dev < 0 || dev >= 256 || !done[dev]) {
+  if (dev < 0 || dev >= 256 || !done[dev].load(std::memory_order_acquire)) {
     if (set_smem_attr(ac::attn_cluster_kernel<D, CL>, smem, CL > 8) != CSA2_OK)
       return CSA2_ERR_CUDA;
-    if (dev >= 0 && dev < 256) done[dev] = true;
+    if (dev >= 0 && dev < 256) done[dev].store(true, std::memory_order_release);
   }
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3((unsigned)(nr * CL), 1, 1);
@@ -394,10 +398,11 @@ csa2_status launch_attn_cl(const ar::Params &a, int64_t nr, bool after_topk, cud
 // Can clusters of 16 CTAs of the attention kernel be scheduled on this device?
 template <int D>
 bool attn_cluster16_ok() {
-  static int cache[256] = {0};  // 0 unknown, 1 yes, 2 no
+  static std::atomic<int> cache[256];  // per device: 0 unknown, 1 yes, 2 no
   int dev = 0;
   cudaGetDevice(&dev);
-  if (dev >= 0 && dev < 256 && cache[dev]) return cache[dev] == 1;
+  if (dev >= 0 && dev < 256 && cache[dev].load(std::memory_order_relaxed))
+    return cache[dev].load(std::memory_order_relaxed) == 1;
   const size_t smem = sizeof(ac::Smem<D, 16>);
   bool ok = set_smem_attr(ac::attn_cluster_kernel<D, 16>, smem, true) == CSA2_OK;
   if (ok) {
@@ -417,7 +422,7 @@ bool attn_cluster16_ok() {
          n > 0;
   }
   cudaGetLastError();
-  if (dev >= 0 && dev < 256) cache[dev] = ok ? 1 : 2;
+  if (dev >= 0 && dev < 256) cache[dev].store(ok ? 1 : 2, std::memory_order_relaxed);
   return ok;
 }
 
@@ -446,12 +451,12 @@ csa2_status launch_attn_cluster(const ar::Params &a, int D, int64_t nr, bool aft
 template <int D>
 csa2_status launch_attn_handoff_d(const ah::Params &hp, int64_t nr, cudaStream_t st) {
   const size_t smem = sizeof(ah::Smem<D>);
-  static bool done[256] = {false};
+  static std::atomic<bool> done[256];  // per device: attributes set
   int dev = 0;
   cudaGetDevice(&dev);
-  if (dev < 0 || dev >= 256 || !done[dev]) {
+  if (dev < 0 || dev >= 256 || !done[dev].load(std::memory_order_acquire)) {
     if (set_smem_attr(ah::attn_handoff_kernel<D>, smem, false) != CSA2_OK) return CSA2_ERR_CUDA;
-    if (dev >= 0 && dev < 256) done[dev] = true;
+    if (dev >= 0 && dev < 256) done[dev].store(true, std::memory_order_release);
   }
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3((unsigned)(nr * hp.G), 1, 1);
@@ -570,18 +575,17 @@ using EncodeTiledFn = CUresult (*)(CUtensorMap *, CUtensorMapDataType, cuuint32_
                                    CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
 
 EncodeTiledFn encode_tiled() {
-  static EncodeTiledFn fn = nullptr;
-  static bool tried = false;
-  if (!tried) {
-    tried = true;
+  static const EncodeTiledFn fn = [] {  // looked up once (thread-safe initialisation)
+    EncodeTiledFn f = nullptr;
     void *ptr = nullptr;
     cudaDriverEntryPointQueryResult q = cudaDriverEntryPointSymbolNotFound;
     if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) ==
             cudaSuccess &&
         q == cudaDriverEntryPointSuccess)
-      fn = reinterpret_cast<EncodeTiledFn>(ptr);
+      f = reinterpret_cast<EncodeTiledFn>(ptr);
     cudaGetLastError();
-  }
+    return f;
+  }();
   return fn;
 }
 
@@ -639,13 +643,13 @@ csa2_status launch_pf_gemm(const CUtensorMap &amap, const CUtensorMap &bmap,
                            const pf::GemmParams &p, int64_t nsplit, int64_t nblk,
                            cudaStream_t st) {
   const size_t smem = pf::gemm_smem_bytes<DI>();
-  static bool done[256] = {false};
+  static std::atomic<bool> done[256];  // per device: attributes set
   int dev = 0;
   cudaGetDevice(&dev);
-  if (dev < 0 || dev >= 256 || !done[dev]) {
+  if (dev < 0 || dev >= 256 || !done[dev].load(std::memory_order_acquire)) {
     if (set_smem_attr(pf::pf_gemm_kernel<DI, SAMPLE>, smem, false) != CSA2_OK)
       return CSA2_ERR_CUDA;
-    if (dev >= 0 && dev < 256) done[dev] = true;
+    if (dev >= 0 && dev < 256) done[dev].store(true, std::memory_order_release);
   }
   TraceScope ts(SAMPLE ? "pf_sample_mma" : "pf_filter_mma", st);
   pf::pf_gemm_kernel<DI, SAMPLE>
@@ -661,14 +665,14 @@ csa2_status pf_run_rows(const int8_t *q_idx, const float *w, const int8_t *k_idx
   const int cap = pf_cap(topk);
   const size_t sel_smem = pf::sel_head_bytes<DI, HI>() + size_t(cap) * 8;
   {
-    static bool done[256] = {false};
+    static std::atomic<bool> done[256];  // per device: attributes set
     int dev = 0;
     cudaGetDevice(&dev);
-    if (dev < 0 || dev >= 256 || !done[dev]) {
+    if (dev < 0 || dev >= 256 || !done[dev].load(std::memory_order_acquire)) {
       if (set_smem_attr(pf::pf_select_kernel<DI, HI>, pf::sel_head_bytes<DI, HI>() + 16384 * 8,
                         false) != CSA2_OK)
         return CSA2_ERR_CUDA;
-      if (dev >= 0 && dev < 256) done[dev] = true;
+      if (dev >= 0 && dev < 256) done[dev].store(true, std::memory_order_release);
     }
   }
   CUtensorMap kmap;
@@ -951,12 +955,12 @@ csa2_status run_fused_t(const fd::Params &base, int64_t rows, cudaStream_t st, v
                         size_t ws_bytes) {
   auto kern = fd::decode_fused_kernel<DI, HI, D, KF>;
   const size_t tile = fd::Shape<DI, HI, KF>::TILE_BYTES;
-  static size_t static_smem[256] = {0};
-  static int bps[256] = {0};
+  static std::atomic<size_t> static_smem[256];  // per device, set before bps
+  static std::atomic<int> bps[256];             // per device: 0 unknown
   int dev = 0;
   cudaGetDevice(&dev);
   if (dev < 0 || dev >= 256) return CSA2_ERR_CUDA;
-  if (!bps[dev]) {
+  if (!bps[dev].load(std::memory_order_acquire)) {
     cudaFuncAttributes fa{};
     if (cudaFuncGetAttributes(&fa, kern) != cudaSuccess) return CSA2_ERR_CUDA;
     const size_t mx = size_t(232448) - fa.sharedSizeBytes - 1024;
@@ -965,8 +969,8 @@ csa2_status run_fused_t(const fd::Params &base, int64_t rows, cudaStream_t st, v
     if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&nb, kern, fd::kThreads, mx) !=
         cudaSuccess)
       return CSA2_ERR_CUDA;
-    static_smem[dev] = fa.sharedSizeBytes;
-    bps[dev] = nb > 0 ? nb : -1;
+    static_smem[dev].store(fa.sharedSizeBytes, std::memory_order_relaxed);
+    bps[dev].store(nb > 0 ? nb : -1, std::memory_order_release);
   }
   if (bps[dev] < 1) return CSA2_ERR_UNSUPPORTED;
   const FusedPlan pl = plan_fused(rows, base.N, DI, HI, D, base.topk, static_smem[dev],
@@ -1453,12 +1457,12 @@ constexpr int64_t kAttnRowsPerLaunch = 16384;
 template <int D>
 csa2_status launch_attn_rows(const ar::Params &p, int64_t nr, cudaStream_t st) {
   const size_t smem = sizeof(ar::Smem<D>);
-  static bool done[256] = {false};
+  static std::atomic<bool> done[256];  // per device: attributes set
   int dev = 0;
   cudaGetDevice(&dev);
-  if (dev < 0 || dev >= 256 || !done[dev]) {
+  if (dev < 0 || dev >= 256 || !done[dev].load(std::memory_order_acquire)) {
     if (set_smem_attr(ar::attn_rows_kernel<D>, smem, false) != CSA2_OK) return CSA2_ERR_CUDA;
-    if (dev >= 0 && dev < 256) done[dev] = true;
+    if (dev >= 0 && dev < 256) done[dev].store(true, std::memory_order_release);
   }
   TraceScope ts("attend_rows", st);
   const unsigned passes = (unsigned)ceil_div(p.H, ar::kHeads);
