@@ -413,11 +413,14 @@ def run_gpu(args, w0):
     # the new token's window row (K and V of every sequence); the step writes
     # that row into the window's last slot on the device, and the older
     # window rows stay resident (a decode loop keeps its window on the GPU).
-    for d in tens:
-        d["new_k"] = d["win_k"][:, -1].clone()
-        d["new_v"] = d["win_v"][:, -1].clone()
-    in_keys = ("q", "q_idx", "w", "new_k", "new_v") + (("app_src", "app_key") if args.append
-                                                        else ())
+    # The layers' windows (K and V) are views of one tensor [2L, B, rows, D],
+    # so the new rows of every layer (one block [2L, B, D] among the per-token
+    # inputs) go into their slots with one copy.
+    win_all = torch.stack([t for d in tens for t in (d["win_k"], d["win_v"])])
+    for l, d in enumerate(tens):
+        d["win_k"], d["win_v"] = win_all[2 * l], win_all[2 * l + 1]
+    tens[0]["new_rows"] = win_all[:, :, -1].clone()
+    in_keys = ("q", "q_idx", "w", "new_rows") + (("app_src", "app_key") if args.append else ())
     out_keys = ("out", "lse", "idx")
     dev_in, _ = pack_into_one_buffer(tens, in_keys, dev)
     dev_out, _ = pack_into_one_buffer(tens, out_keys, dev)
@@ -558,6 +561,16 @@ def run_gpu(args, w0):
     host_out = torch.empty_like(dev_out, device="cpu").pin_memory()
     h2d = host_in.numel()
     d2h = host_out.numel()
+    # A step's input staging (the pinned host->device copy, then each layer's
+    # new window row into its slot) and its result copy, each replayed as one
+    # CUDA graph, as a serving loop would launch them.
+    in_graph, out_graph = torch.cuda.CUDAGraph(), torch.cuda.CUDAGraph()
+    with torch.cuda.graph(in_graph):
+        dev_in.copy_(host_in, non_blocking=True)
+        win_all[:, :, -1].copy_(tens[0]["new_rows"])
+    with torch.cuda.graph(out_graph):
+        host_out.copy_(dev_out, non_blocking=True)
+    torch.cuda.synchronize()
 
     def e2e_steps(K):
         """K end-to-end steps; per step the device ms of (inputs in + window
@@ -568,10 +581,7 @@ def run_gpu(args, w0):
             flush()
             a, b = ev(), ev()
             a.record(stream)
-            dev_in.copy_(host_in, non_blocking=True)
-            for d in tens:
-                d["win_k"][:, -1].copy_(d["new_k"])
-                d["win_v"][:, -1].copy_(d["new_v"])
+            in_graph.replay()
             b.record(stream)
             segs = [("h2d", a, b)]
             for l in range(w0.L):
@@ -584,7 +594,7 @@ def run_gpu(args, w0):
                 segs.append(("layers", a, b))
             a, b = ev(), ev()
             a.record(stream)
-            host_out.copy_(dev_out, non_blocking=True)
+            out_graph.replay()
             b.record(stream)
             segs.append(("d2h", a, b))
             res.append(segs)
