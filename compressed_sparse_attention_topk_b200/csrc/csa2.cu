@@ -199,7 +199,25 @@ void launch_scan_kf(dim3 grid, cudaStream_t st, const int8_t *q_idx, const float
     if (dev >= 0 && dev < 256) done[dev].store(true, std::memory_order_release);
   }
   index_scan_kernel<DI, HI, KF><<<grid, kScanThreads, S::SMEM, st>>>(
-      q_idx, w, k_idx, k_exps, T, N, n_prior, ratio, row0, scores, stride, hist1, write_masked);
+      q_idx, w, k_idx, k_exps, T, N, n_prior, ratio, row0, scores, stride, hist1, write_masked,
+      ScanBlockMax{});
+}
+
+// The int8-key scan that also takes a Full row's block maxima (ScanBlockMax).
+template <int DI, int HI>
+void launch_scan_bm(dim3 grid, cudaStream_t st, const int8_t *q_idx, const float *w,
+                    const int8_t *k_idx, int64_t N, int64_t row0, float *scores, int64_t stride,
+                    uint32_t *hist1, const ScanBlockMax &bm) {
+  using S = ScanShape<DI, HI, kScanKeysInt8>;
+  static std::atomic<bool> done[256];  // per device: attributes set
+  int dev = 0;
+  cudaGetDevice(&dev);
+  if (dev < 0 || dev >= 256 || !done[dev].load(std::memory_order_acquire)) {
+    set_smem_attr(index_scan_kernel<DI, HI, kScanKeysInt8, true>, S::SMEM, false);
+    if (dev >= 0 && dev < 256) done[dev].store(true, std::memory_order_release);
+  }
+  index_scan_kernel<DI, HI, kScanKeysInt8, true><<<grid, kScanThreads, S::SMEM, st>>>(
+      q_idx, w, k_idx, nullptr, 1, N, -1, 1, row0, scores, stride, hist1, 0, bm);
 }
 
 template <int DI, int HI>
@@ -217,6 +235,17 @@ using ScanLaunch = void (*)(dim3, cudaStream_t, const int8_t *, const float *, c
 using ScanLaunchFp4 = void (*)(dim3, cudaStream_t, const int8_t *, const float *, const int8_t *,
                                const uint8_t *, int32_t, int64_t, int64_t, int32_t, int64_t,
                                float *, int64_t, uint32_t *, int);
+
+using ScanLaunchBM = void (*)(dim3, cudaStream_t, const int8_t *, const float *, const int8_t *,
+                              int64_t, int64_t, float *, int64_t, uint32_t *,
+                              const ScanBlockMax &);
+
+// Decode shapes whose scan also takes the block maxima of a Full layer's pool.
+ScanLaunchBM pick_scan_bm(int32_t d_I, int32_t H_I) {
+  if (d_I == 32 && H_I == 4) return &launch_scan_bm<32, 4>;
+  if (d_I == 64 && H_I == 4) return &launch_scan_bm<64, 4>;
+  return nullptr;
+}
 
 ScanLaunchFp4 pick_scan_fp4(int32_t d_I, int32_t H_I) {
   if (d_I == 32 && H_I == 4) return &launch_scan_kf<32, 4, kScanKeysFp4>;
@@ -1139,6 +1168,12 @@ csa2_status run_index_topk(const int8_t *q_idx, const float *w, const int8_t *k_
   const int sms = device_sms();
   const int64_t nbk = pr ? ceil_div(N, pr->block) : 0;
   const int64_t bstride = (nbk + 3) & ~int64_t(3);
+  // the scan takes the block maxima itself for blocks of 2^i <= 16 positions
+  const ScanLaunchBM scan_bm =
+      (pr && !fp4 && T == 1 && score_out == nullptr && pr->block <= 16 &&
+       (pr->block & (pr->block - 1)) == 0)
+          ? pick_scan_bm(d_I, H_I)
+          : nullptr;
   if (pr && cudaMemsetAsync(pr->X.bhist, 0, size_t(B) * kHistStride * 4, st) != cudaSuccess)
     return CSA2_ERR_CUDA;
   // Attention after the selection.  With many rows per launch (8 or fewer
@@ -1169,7 +1204,11 @@ csa2_status run_index_topk(const int8_t *q_idx, const float *w, const int8_t *k_
     const int G = (int)std::min(g_want, g_max);
     {
       TraceScope ts("index_scan", st);
-      if (scan4)
+      if (scan_bm)  // a Full row's pool: the block maxima come with the scores
+        scan_bm(dim3(G, (unsigned)units), st, q_idx, w, k_idx, N, row0, scores, stride, L.hist1,
+                ScanBlockMax{pr->X.bscores + row0 * bstride, bstride,
+                             pr->X.bhist + row0 * kHistStride, pr->block});
+      else if (scan4)
         scan4(dim3(G, (unsigned)units), st, q_idx, w, k_idx, k_exps, T, N, n_prior, ratio, row0,
               scores, stride, L.hist1, score_out != nullptr);
       else
@@ -1237,7 +1276,7 @@ csa2_status run_index_topk(const int8_t *q_idx, const float *w, const int8_t *k_
       hp.G = row_cluster_size(nr, D);
       if (launch_attn_handoff(hp, D, nr, st) != CSA2_OK) return CSA2_ERR_CUDA;
     }
-    if (pr) {  // block maxima of these rows' scores, before the next pass reuses them
+    if (pr && !scan_bm) {  // block maxima of these rows' scores, before the next pass reuses them
       TraceScope ts("pool_block_max", st);
       block_max_kernel<<<dim3((unsigned)ceil_div(nbk, kPoolThreads), (unsigned)nr), kPoolThreads,
                          0, st>>>(scores, stride, N, pr->block, pr->X.bscores + row0 * bstride,

@@ -61,21 +61,38 @@ __device__ __forceinline__ int chunk_xor(int t) {
   return (NCH == 1) ? 0 : (t / (8 / NCH)) % NCH;
 }
 
+// Block maxima taken by the scan itself (a Full layer's candidate pool, see
+// pool.cuh): per row, the largest score of every `block` consecutive
+// positions (block a power of two <= 16, so a block's keys sit on
+// consecutive lanes of one warp and never cross a slice or a tile) into
+// bscores [rows, bstride], and their digit-1 histogram into bhist [rows,
+// kHistStride] (zeroed).
+struct ScanBlockMax {
+  float *bscores;
+  int64_t bstride;
+  uint32_t *bhist;
+  int32_t block;
+};
+
 // grid = (G slices, rows).  hist1: [rows][kHistStride], zeroed.  With FP4
 // keys, k_idx holds the codes [B, N, d_I/2] and k_exps the exponents [B, N,
-// d_I/32] (N % 16 == 0, so every copy starts on a 16-byte boundary).
-template <int DI, int HI, int KF = kScanKeysInt8>
+// d_I/32] (N % 16 == 0, so every copy starts on a 16-byte boundary).  BM:
+// also the block maxima of `bm` (int8 keys).
+template <int DI, int HI, int KF = kScanKeysInt8, bool BM = false>
 __global__ void __launch_bounds__(kScanThreads, 2)
     index_scan_kernel(const int8_t *__restrict__ q_idx, const float *__restrict__ w,
                       const int8_t *__restrict__ k_idx, const uint8_t *__restrict__ k_exps,
                       int32_t T, int64_t N, int64_t n_prior, int32_t ratio, int64_t row0,
                       float *__restrict__ scores, int64_t score_stride,
-                      uint32_t *__restrict__ hist1, int write_masked) {
+                      uint32_t *__restrict__ hist1, int write_masked, const ScanBlockMax bm) {
   using S = ScanShape<DI, HI, KF>;
   constexpr int NCH = S::NCH, STAGES = S::STAGES, TK = S::TILE_KEYS, QW = S::QW;
+  static_assert(!BM || KF == kScanKeysInt8, "block maxima with int8 keys");
+  const int bshift = BM ? __ffs(bm.block) - 1 : 0;
   extern __shared__ __align__(128) unsigned char smem_tiles[];
   __shared__ uint64_t full_bar[STAGES];
   __shared__ uint32_t sh_hist[kBins1];
+  __shared__ uint32_t sh_bhist[BM ? kBins1 : 1];
   __shared__ __align__(16) int4 sh_q[S::QREG ? 1 : HI * NCH * QW];
 
   const int tid = threadIdx.x;
@@ -107,6 +124,8 @@ __global__ void __launch_bounds__(kScanThreads, 2)
   // for this grid's results before reading them.
   pdl_allow_dependents();
   for (int i = tid; i < kBins1; i += kScanThreads) sh_hist[i] = 0u;
+  if constexpr (BM)
+    for (int i = tid; i < kBins1; i += kScanThreads) sh_bhist[i] = 0u;
   if (tid == 0) {
     for (int s = 0; s < STAGES; ++s) mbar_init(&full_bar[s], 1);
     fence_barrier_init();
@@ -193,6 +212,16 @@ __global__ void __launch_bounds__(kScanThreads, 2)
       // plain shared-memory reduction (a warp-aggregating match costs more
       // on its narrow issue pipe than the bin conflicts it saves)
       if (valid) atomicAdd(&sh_hist[key_d1(score_key(score))], 1u);
+      if constexpr (BM) {  // the block's largest score, by its first lane
+        float m = valid ? score : -__int_as_float(0x7f800000);
+#pragma unroll
+        for (int o = 1; o < 16; o <<= 1)
+          if (o < bm.block) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+        if (valid && (kl & (bm.block - 1)) == 0) {
+          bm.bscores[r_local * bm.bstride + ((tbase + kl) >> bshift)] = m;
+          atomicAdd(&sh_bhist[key_d1(score_key(m))], 1u);
+        }
+      }
     }
   }
   if (abort_it >= 0) {
@@ -219,6 +248,13 @@ __global__ void __launch_bounds__(kScanThreads, 2)
   for (int i = tid; i < kBins1; i += kScanThreads) {
     const uint32_t v = sh_hist[i];
     if (v) atomicAdd(grow + i, v);
+  }
+  if constexpr (BM) {
+    uint32_t *brow = bm.bhist + r_local * kHistStride;
+    for (int i = tid; i < kBins1; i += kScanThreads) {
+      const uint32_t v = sh_bhist[i];
+      if (v) atomicAdd(brow + i, v);
+    }
   }
 }
 

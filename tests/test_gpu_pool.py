@@ -157,14 +157,20 @@ def _pool_layers(w0, layers, block, n_blocks):
     return tens
 
 
-@pytest.mark.parametrize("B,N,block,n_blocks,topk", [(4, 262144, 8, 2048, 2048),
-                                                     (3, 20001, 8, 300, 512),
-                                                     (2, 5000, 16, 40, 100),
-                                                     (2, 3000, 8, 400, 64)])
-def test_pool_layers_in_the_layer_call(B, N, block, n_blocks, topk, decode_kernel):
+@pytest.mark.parametrize("B,N,block,n_blocks,topk,d_I", [(4, 262144, 8, 2048, 2048, 64),
+                                                         (3, 20001, 8, 300, 512, 64),
+                                                         (2, 5000, 16, 40, 100, 64),
+                                                         (2, 3000, 8, 400, 64, 64),
+                                                         (3, 9999, 4, 500, 256, 64),
+                                                         (2, 4097, 2, 1000, 128, 32),
+                                                         (2, 3001, 1, 1500, 64, 32),
+                                                         (2, 5003, 32, 50, 128, 64)])
+def test_pool_layers_in_the_layer_call(B, N, block, n_blocks, topk, d_I, decode_kernel):
+    """Blocks of 2^i <= 16 positions take their maxima in the Full layer's
+    scan itself; other block sizes in a pass over the scores after it."""
     from tests._parity import assert_close, oracle_store
-    w0 = wl.with_sizes(wl.LONG, name=f"pool_layers_{N}", B=B, N=N, topk=topk, seed=N + B,
-                       modes=((0, 0, 0), (csa2.REINDEX_POOL, 0, 1), (2, 0, 1)))
+    w0 = wl.with_sizes(wl.LONG, name=f"pool_layers_{N}", B=B, N=N, topk=topk, d_I=d_I,
+                       seed=N + B, modes=((0, 0, 0), (csa2.REINDEX_POOL, 0, 1), (2, 0, 1)))
     layers = wl.all_layer_inputs(w0)
     tens = _pool_layers(w0, layers, block, n_blocks)
     dims = csa2.make_dims(B, 1, w0.H, w0.D, N, w0.H_I, w0.d_I, topk, w0.W, pool_block=block,
