@@ -35,6 +35,7 @@ EXPORTED = (
     "csa2_index_pool", "csa2_pool_topk_workspace_size", "csa2_pool_topk", "csa2_append_entry",
     "csa2_pack_index_keys_fp4", "csa2_index_topk_fp4k_workspace_size", "csa2_index_topk_fp4k",
     "csa2_wait_timeout_selftest", "csa2_set_decode_kernel", "csa2_get_decode_kernel",
+    "csa2_stage_copies",
 )
 DECODE_SCAN_CLUSTER, DECODE_FUSED = 0, 1
 
@@ -56,6 +57,15 @@ class Dims(ctypes.Structure):
                 ("n_prior", ctypes.c_int64), ("ratio", ctypes.c_int32),
                 ("sm_scale", ctypes.c_float), ("pool_block", ctypes.c_int32),
                 ("pool_blocks", ctypes.c_int32)]
+
+
+class Copy2D(ctypes.Structure):
+    _fields_ = [("src", ctypes.c_void_p), ("dst", ctypes.c_void_p), ("rows", ctypes.c_int64),
+                ("row_bytes", ctypes.c_int64), ("src_stride", ctypes.c_int64),
+                ("dst_stride", ctypes.c_int64)]
+
+
+MAX_STAGE_COPIES = 16
 
 
 class LayerIO(ctypes.Structure):
@@ -105,6 +115,7 @@ def lib() -> ctypes.CDLL:
         "csa2_index_pool": ([P, P, P, i32, i32, i32, i64, i32, i32, P, P, sz, P], i32),
         "csa2_pool_topk_workspace_size": ([i32, i32, i32], sz),
         "csa2_pool_topk": ([P, P, P, i32, i32, i32, i64, P, i32, i32, P, P, sz, P], i32),
+        "csa2_stage_copies": ([P, i32, P], i32),
         "csa2_get_device_status": ([P, P], i32),
         "csa2_wait_timeout_selftest": ([i64, P], i32),
         "csa2_set_decode_kernel": ([i32], i32),
@@ -167,6 +178,49 @@ def workspace(nbytes: int, device=None):
         buf = torch.empty(max(nbytes, 256), dtype=torch.uint8, device=dev)
         _ws_cache[key] = buf
     return buf
+
+
+# --- staging copies -----------------------------------------------------------
+
+def _rows_of(t, name):
+    """(rows, row bytes, row stride in bytes) of a tensor whose last dim is
+    contiguous and whose leading dims collapse to rows of one stride."""
+    es = t.element_size()
+    if t.dim() == 0:
+        return 1, es, es
+    if t.shape[-1] > 1 and t.stride(-1) != 1:
+        raise ValueError(f"{name}: the last dim must be contiguous")
+    if t.dim() == 1:
+        return 1, t.shape[0] * es, t.shape[0] * es
+    for i in range(t.dim() - 2):
+        if t.shape[i] > 1 and t.stride(i) != t.stride(i + 1) * t.shape[i + 1]:
+            raise ValueError(f"{name}: the leading dims must collapse to rows of one stride")
+    rows = 1
+    for n in t.shape[:-1]:
+        rows *= n
+    return rows, t.shape[-1] * es, t.stride(-2) * es
+
+
+def stage_copies(pairs):
+    """One launch copying each (src, dst) tensor pair (same shape and dtype;
+    each a CUDA tensor of the current device or a pinned CPU tensor; last
+    dim contiguous, leading dims collapsing to rows of one stride; 16-byte
+    aligned rows), at most MAX_STAGE_COPIES pairs, on the current stream."""
+    torch = _torch()
+    pairs = list(pairs)
+    if len(pairs) > MAX_STAGE_COPIES:
+        raise ValueError(f"at most {MAX_STAGE_COPIES} copies per launch")
+    arr = (Copy2D * max(len(pairs), 1))()
+    for i, (src, dst) in enumerate(pairs):
+        for name, t in (("src", src), ("dst", dst)):
+            if not isinstance(t, torch.Tensor) or not (t.is_cuda or t.is_pinned()):
+                raise TypeError(f"pairs[{i}].{name} must be a CUDA or pinned CPU tensor")
+        if src.shape != dst.shape or src.dtype != dst.dtype:
+            raise ValueError(f"pairs[{i}]: src and dst differ in shape or dtype")
+        rows, rb, ss = _rows_of(src, f"pairs[{i}].src")
+        _, _, ds = _rows_of(dst, f"pairs[{i}].dst")
+        arr[i] = Copy2D(src.data_ptr(), dst.data_ptr(), rows, rb, ss, ds)
+    _check(lib().csa2_stage_copies(arr, len(pairs), _stream()), "csa2_stage_copies")
 
 
 # --- FP4 ----------------------------------------------------------------------

@@ -13,6 +13,7 @@
 #include "attn_handoff.cuh"
 #include "attn_rows.cuh"
 #include "common.cuh"
+#include "stage.cuh"
 #include "decode_fused.cuh"
 #include "index_scan.cuh"
 #include "pack.cuh"
@@ -1715,6 +1716,72 @@ csa2_status csa2_pack_fp4(const float *src, int64_t rows, int32_t D, uint8_t *co
   const int64_t blocks = std::min<int64_t>(ceil_div(groups, 256), int64_t(device_sms()) * 16);
   TraceScope ts("pack_fp4", as_stream(stream));
   pack_fp4_kernel<<<(unsigned)blocks, 256, 0, as_stream(stream)>>>(src, groups, codes, scales);
+  return after_launch();
+}
+
+namespace {
+// Where the bytes [p, p + len) live: 0 = this device's memory, 1 = page-
+// locked host memory the device addresses at the same pointer, -1 = neither
+// (pageable host memory, another device's memory), checked at both ends.
+csa2_status memory_kind(const void *p, int64_t len, int &kind) {
+  kind = -1;
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return CSA2_ERR_CUDA;
+  int k[2];
+  const char *ends[2] = {static_cast<const char *>(p), static_cast<const char *>(p) + (len - 1)};
+  for (int e = 0; e < 2; ++e) {
+    cudaPointerAttributes a{};
+    if (cudaPointerGetAttributes(&a, ends[e]) != cudaSuccess) {
+      cudaGetLastError();
+      return CSA2_ERR_CUDA;
+    }
+    if ((a.type == cudaMemoryTypeDevice || a.type == cudaMemoryTypeManaged) && a.device == dev)
+      k[e] = 0;
+    else if (a.type == cudaMemoryTypeHost && a.devicePointer == ends[e])
+      k[e] = 1;
+    else
+      k[e] = -1;
+  }
+  if (k[0] == k[1]) kind = k[0];
+  return CSA2_OK;
+}
+}  // namespace
+
+csa2_status csa2_stage_copies(const csa2_copy2d *copies, int32_t n, void *stream) {
+  if (n < 0 || n > kStageMax || (n > 0 && !copies)) return CSA2_ERR_INVALID_ARG;
+  // every copy's sizes and alignment first, then where its memory lives
+  for (int i = 0; i < n; ++i) {
+    const csa2_copy2d &c = copies[i];
+    if (c.rows < 0 || c.row_bytes < 0) return CSA2_ERR_INVALID_ARG;
+    if (c.rows == 0 || c.row_bytes == 0) continue;
+    if (!c.src || !c.dst || !aligned(c.src, 16) || !aligned(c.dst, 16) || c.row_bytes % 16 != 0 ||
+        c.src_stride < 0 || c.src_stride % 16 != 0 || c.dst_stride % 16 != 0 ||
+        (c.rows > 1 && c.dst_stride < c.row_bytes))
+      return CSA2_ERR_INVALID_ARG;
+  }
+  StageList L{};
+  int64_t most = 0;
+  int m = 0;
+  for (int i = 0; i < n; ++i) {
+    const csa2_copy2d &c = copies[i];
+    if (c.rows == 0 || c.row_bytes == 0) continue;
+    int ks, kd;
+    csa2_status rc = memory_kind(c.src, (c.rows - 1) * c.src_stride + c.row_bytes, ks);
+    if (rc != CSA2_OK) return rc;
+    rc = memory_kind(c.dst, (c.rows - 1) * c.dst_stride + c.row_bytes, kd);
+    if (rc != CSA2_OK) return rc;
+    if (ks < 0 || kd < 0) return CSA2_ERR_INVALID_ARG;
+    L.c[m] = StageCopy{static_cast<const int4 *>(c.src), static_cast<int4 *>(c.dst), c.rows,
+                       c.row_bytes / 16, c.src_stride / 16, c.dst_stride / 16, ks, kd};
+    most = std::max(most, c.rows * (c.row_bytes / 16));
+    ++m;
+  }
+  if (m == 0) return CSA2_OK;
+  L.n = m;
+  const int64_t x = std::min<int64_t>(ceil_div(most, int64_t(kStageThreads) * kStageUnroll),
+                                      int64_t(device_sms()) * 4);
+  TraceScope ts("stage_copies", as_stream(stream));
+  stage_copies_kernel<<<dim3((unsigned)x, (unsigned)m), kStageThreads, 0, as_stream(stream)>>>(L);
   return after_launch();
 }
 

@@ -434,6 +434,47 @@ csa2_status csa2_layer_group_run(const csa2_layer_mode *modes, const csa2_layer_
                                  const csa2_dims *dims, void *ws, size_t ws_bytes, void *stream);
 
 /* ---------------------------------------------------------------------- */
+/* Staging copies                                                          */
+/* ---------------------------------------------------------------------- */
+
+/* One copy of csa2_stage_copies: `rows` rows of `row_bytes` bytes, row i
+ * from src + i * src_stride to dst + i * dst_stride (byte strides).  src
+ * and dst are each either memory of the current device or page-locked host
+ * memory that the device addresses at the same pointer (cudaHostAlloc /
+ * cudaMallocHost under unified addressing).  Pointers, row_bytes and both
+ * strides are multiples of 16 bytes; dst_stride >= row_bytes when rows > 1;
+ * src_stride >= 0. */
+typedef struct csa2_copy2d {
+    const void *src;
+    void *dst;
+    int64_t rows;
+    int64_t row_bytes;
+    int64_t src_stride;
+    int64_t dst_stride;
+} csa2_copy2d;
+
+#define CSA2_MAX_STAGE_COPIES 16
+
+/* Up to CSA2_MAX_STAGE_COPIES copies in one kernel launch on `stream`: a
+ * decode step's inputs from pinned host buffers into their device buffers
+ * (a window's new row straight into its slot), or its results back to the
+ * host.  Every thread moves 16-byte pieces through the mapped host buffer
+ * itself (host memory read uncached, written through), so all pieces are in
+ * flight at once and a step pays about one round trip over the host link
+ * instead of a copy-engine transfer per buffer.  The pages describe no such
+ * call: it is the library's input/output path.  The copies run concurrently:
+ * no destination may overlap another copy's source or destination.  The
+ * host must leave a host source unchanged, and not read a host destination,
+ * until the stream has passed the launch.
+ *   copies  host array [n]; rows == 0 or row_bytes == 0 skips a copy.
+ * Errors: CSA2_ERR_INVALID_ARG for n outside [0, CSA2_MAX_STAGE_COPIES], a
+ * null pointer, misalignment, a negative size or stride, or memory the
+ * device cannot address at that pointer (pageable host memory, another
+ * device's memory; both ends of each range are checked); CSA2_ERR_CUDA when
+ * a pointer query or the launch fails. */
+csa2_status csa2_stage_copies(const csa2_copy2d *copies, int32_t n, void *stream);
+
+/* ---------------------------------------------------------------------- */
 /* Kernel timing trace                                                     */
 /* ---------------------------------------------------------------------- */
 

@@ -171,3 +171,47 @@ def test_noalloc_refuses_by_the_documented_workspace_size(lib):
     rc = lib.csa2_index_topk_noalloc(fake, fake, fake, 4, 1, 4, 64, 1_000_000, -1, 4, 2048,
                                      fake, None, None)
     assert rc == csa2.CSA2_ERR_UNSUPPORTED
+
+
+def test_stage_copies_validate_before_any_query(lib):
+    """csa2_stage_copies refuses bad counts, sizes, strides and alignment
+    before it asks where a pointer lives or launches anything."""
+    C = csa2.Copy2D
+    ok = C(256, 512, 2, 32, 32, 64)
+
+    def run(*copies, n=None):
+        arr = (C * max(len(copies), 1))(*copies)
+        return lib.csa2_stage_copies(arr, len(copies) if n is None else n, None)
+
+    assert lib.csa2_stage_copies(None, 0, None) == csa2.CSA2_OK
+    assert run(C(None, None, 0, 16, 16, 16)) == csa2.CSA2_OK          # no rows: skipped
+    assert run(C(None, None, 4, 0, 16, 16)) == csa2.CSA2_OK           # empty rows: skipped
+    assert lib.csa2_stage_copies(None, 1, None) == csa2.CSA2_ERR_INVALID_ARG
+    assert run(ok, n=-1) == csa2.CSA2_ERR_INVALID_ARG
+    assert run(*([ok] * 17)) == csa2.CSA2_ERR_INVALID_ARG             # > CSA2_MAX_STAGE_COPIES
+    assert run(C(None, 512, 1, 16, 16, 16)) == csa2.CSA2_ERR_INVALID_ARG
+    assert run(C(256, None, 1, 16, 16, 16)) == csa2.CSA2_ERR_INVALID_ARG
+    assert run(C(264, 512, 1, 16, 16, 16)) == csa2.CSA2_ERR_INVALID_ARG  # src misaligned
+    assert run(C(256, 520, 1, 16, 16, 16)) == csa2.CSA2_ERR_INVALID_ARG  # dst misaligned
+    assert run(C(256, 512, 1, 24, 32, 32)) == csa2.CSA2_ERR_INVALID_ARG  # row bytes % 16
+    assert run(C(256, 512, 2, 32, 40, 64)) == csa2.CSA2_ERR_INVALID_ARG  # src stride % 16
+    assert run(C(256, 512, 2, 32, 32, 16)) == csa2.CSA2_ERR_INVALID_ARG  # rows overlap in dst
+    assert run(C(256, 512, 2, 32, -32, 64)) == csa2.CSA2_ERR_INVALID_ARG
+    assert run(C(256, 512, -1, 32, 32, 64)) == csa2.CSA2_ERR_INVALID_ARG
+    assert run(ok, C(256, 512, 1, 8, 16, 16)) == csa2.CSA2_ERR_INVALID_ARG  # second copy bad
+
+
+def test_stage_copies_binding_collapses_rows():
+    """The binding's row view: leading dims that collapse to one stride, a
+    strided slot per row, and views it must refuse."""
+    import torch
+    w = torch.zeros(6, 4, 128, 64, dtype=torch.bfloat16)
+    assert csa2._rows_of(w[:, :, -1], "x") == (24, 128, 128 * 64 * 2)
+    assert csa2._rows_of(w[2], "x") == (512, 128, 128)
+    assert csa2._rows_of(torch.zeros(100, dtype=torch.uint8), "x") == (1, 100, 100)
+    with pytest.raises(ValueError):
+        csa2._rows_of(w[:, 1:3, -1], "x")       # dims 0 and 1 do not collapse
+    with pytest.raises(ValueError):
+        csa2._rows_of(w[..., ::2], "x")         # last dim not contiguous
+    with pytest.raises(TypeError):
+        csa2.stage_copies([(torch.zeros(16), torch.zeros(16))])  # pageable CPU tensors
