@@ -282,10 +282,34 @@ void launch_scan_group(dim3 grid, cudaStream_t st, const int8_t *q_idx, const fl
       q_idx, w, k_idx, T, N, n_prior, ratio, row0, scores, stride, hist1, write_masked);
 }
 
+template <int DI, int TQ>
+void launch_scan_mma(dim3 grid, cudaStream_t st, const int8_t *q_idx, const float *w,
+                     const int8_t *k_idx, int32_t T, int64_t N, int64_t n_prior, int32_t ratio,
+                     int64_t row0, float *scores, int64_t stride, uint32_t *hist1,
+                     int write_masked) {
+  using S = ScanMmaShape<DI, TQ>;
+  static std::atomic<bool> done[256];  // per device: attributes set
+  int dev = 0;
+  cudaGetDevice(&dev);
+  if (dev < 0 || dev >= 256 || !done[dev].load(std::memory_order_acquire)) {
+    set_smem_attr(index_scan_mma_kernel<DI, TQ>, S::smem(TQ), false);
+    if (dev >= 0 && dev < 256) done[dev].store(true, std::memory_order_release);
+  }
+  index_scan_mma_kernel<DI, TQ><<<grid, S::THREADS, S::smem(T), st>>>(
+      q_idx, w, k_idx, T, N, n_prior, ratio, row0, scores, stride, hist1, write_masked);
+}
+
 // Several query rows per sequence (2 <= T <= 8, d_I <= 64): one scan of the
-// keys serves all of them.
+// keys serves all of them; with 4 index heads and d_I in {32, 64} the dots
+// run on the tensor cores (index_scan_mma_kernel).
 ScanLaunch pick_scan_group(int32_t d_I, int32_t H_I, int32_t T) {
   if (T < 2 || T > 8 || d_I > 64) return nullptr;
+  if (H_I == 4 && (d_I == 32 || d_I == 64)) {
+    if (d_I == 32) return T <= 2 ? &launch_scan_mma<32, 2> : T <= 4 ? &launch_scan_mma<32, 4>
+                                                                    : &launch_scan_mma<32, 8>;
+    return T <= 2 ? &launch_scan_mma<64, 2> : T <= 4 ? &launch_scan_mma<64, 4>
+                                                     : &launch_scan_mma<64, 8>;
+  }
 #define CSA2_SG_CASE(DI, HI)                                                    \
   if (d_I == DI && H_I == HI) {                                                 \
     if (T <= 2) return &launch_scan_group<DI, HI, 2>;                           \

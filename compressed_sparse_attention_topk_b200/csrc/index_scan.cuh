@@ -449,3 +449,213 @@ __global__ void __launch_bounds__(64 * TQ, TQ <= 4 ? 2 : 1)
 }
 
 }  // namespace csa2
+
+namespace csa2 {
+
+// ---------------------------------------------------------------------------
+// Multi-token scan on tensor cores (4 index heads, d_I in {32, 64}).
+//
+// With T query tokens per sequence the index dots of one key against all
+// 4T query heads are a small exact integer contraction, so each warp takes
+// 16 keys of the tile at a time as the rows of an int8 mma.sync m16n8k32
+// (A = 16 keys x 32 bytes, ldmatrix from the staged tile; B = 8 query heads,
+// i.e. 2 tokens, held in registers; int32 accumulators, exact) instead of
+// the dp4a chains of index_scan_group_kernel.  In the accumulator a lane
+// holds heads 2(tig&1), +1 of token 2u + tig/2 for keys gid and gid + 8; one
+// exchange with lane ^ 1 gives each lane all 4 heads of one key (the even
+// lane key gid, the odd lane key gid + 8), whose score it forms in the same
+// fixed fp32 order as the other scans.  Keys stream through the same bulk-
+// copy ring; slices, visibility, histograms and scores as
+// index_scan_group_kernel.
+// grid = (G slices, sequences of the pass); 256 threads; dynamic shared
+// memory STAGES * 16 KiB + T * kBins1 * 4 (the per-token histograms).
+// ---------------------------------------------------------------------------
+template <int DI, int TQ>
+struct ScanMmaShape {
+  static_assert(DI == 32 || DI == 64, "d_I in {32, 64}");
+  static constexpr int HI = 4;
+  static constexpr int KS = DI / 32;             // k-steps of 32 bytes
+  static constexpr int NT = (TQ * HI + 7) / 8;   // n-tiles of 8 query heads (2 tokens)
+  static constexpr int THREADS = 256;
+  static constexpr int TILE_BYTES = 16384;
+  static constexpr int TILE_KEYS = TILE_BYTES / DI;
+  static constexpr int SUB = TILE_KEYS / 16;     // 16-key row blocks per tile
+  static constexpr int STAGES = 4;
+  static size_t smem(int T) { return size_t(STAGES) * TILE_BYTES + size_t(T) * kBins1 * 4; }
+};
+
+__device__ __forceinline__ void mma_s8_16832(int (&d)[4], const uint32_t (&a)[4], uint32_t b0,
+                                             uint32_t b1) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k32.row.col.s32.s8.s8.s32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, "
+      "{%8,%9}, {%0,%1,%2,%3};"
+      : "+r"(d[0]), "+r"(d[1]), "+r"(d[2]), "+r"(d[3])
+      : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+}
+
+template <int DI, int TQ>
+__global__ void __launch_bounds__(256, 2)
+    index_scan_mma_kernel(const int8_t *__restrict__ q_idx, const float *__restrict__ w,
+                          const int8_t *__restrict__ k_idx, int32_t T, int64_t N,
+                          int64_t n_prior, int32_t ratio, int64_t row0,
+                          float *__restrict__ scores, int64_t score_stride,
+                          uint32_t *__restrict__ hist1, int write_masked) {
+  using S = ScanMmaShape<DI, TQ>;
+  constexpr int STAGES = S::STAGES, TK = S::TILE_KEYS, NT = S::NT, KS = S::KS;
+  extern __shared__ __align__(128) unsigned char smem_tiles[];
+  uint32_t *sh_hist = reinterpret_cast<uint32_t *>(smem_tiles + STAGES * S::TILE_BYTES);
+  __shared__ uint64_t full_bar[STAGES];
+
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int gid = lane >> 2, tig = lane & 3;
+  const bool odd = tig & 1;
+  const int64_t gl = blockIdx.y;    // sequence within the pass
+  const int64_t rl0 = gl * T;       // its first row within the pass
+  const int64_t b = (row0 + rl0) / T;
+  const int G = gridDim.x, g = blockIdx.x;
+
+  int64_t V = N;  // the group's largest visible count (visibility grows with t)
+  if (n_prior >= 0) {
+    V = n_prior + (int64_t)T / ratio;
+    if (V > N) V = N;
+  }
+  const int64_t n0 = ((V * g) / G) & ~int64_t(15);
+  const int64_t n1 = (g == G - 1) ? V : (((V * (g + 1)) / G) & ~int64_t(15));
+  const int ntiles = (int)((n1 - n0 + TK - 1) / TK);
+  const int8_t *src = k_idx + (b * N + n0) * DI;
+
+  pdl_allow_dependents();
+  for (int i = tid; i < T * kBins1; i += S::THREADS) sh_hist[i] = 0u;
+  if (tid == 0) {
+    for (int s = 0; s < STAGES; ++s) mbar_init(&full_bar[s], 1);
+    fence_barrier_init();
+  }
+  // B fragments: query head j = 8u + gid (token j / 4, head j % 4), bytes
+  // [32k + 4 tig, +4) and [32k + 16 + 4 tig, +4); zero past the last token
+  uint32_t bq[NT][KS][2];
+#pragma unroll
+  for (int u = 0; u < NT; ++u) {
+    const int j = 8 * u + gid, tq = j >> 2;
+    const int8_t *qr = q_idx + ((b * T + (tq < T ? tq : 0)) * 4 + (j & 3)) * (int64_t)DI;
+#pragma unroll
+    for (int k = 0; k < KS; ++k) {
+      bq[u][k][0] = tq < T ? *reinterpret_cast<const uint32_t *>(qr + 32 * k + 4 * tig) : 0u;
+      bq[u][k][1] = tq < T ? *reinterpret_cast<const uint32_t *>(qr + 32 * k + 16 + 4 * tig) : 0u;
+    }
+  }
+  // this lane's token in n-tile u, its weights and its visible count
+  float wt[NT][4];
+  int64_t vq[NT];
+#pragma unroll
+  for (int u = 0; u < NT; ++u) {
+    const int tq = 2 * u + (tig >> 1);
+#pragma unroll
+    for (int h = 0; h < 4; ++h) wt[u][h] = tq < T ? w[(b * T + tq) * 4 + h] : 0.0f;
+    int64_t v = tq < T ? N : 0;
+    if (n_prior >= 0 && tq < T) {
+      v = n_prior + (int64_t)(tq + 1) / ratio;
+      if (v > N) v = N;
+    }
+    vq[u] = v;
+  }
+  __syncthreads();
+  if (tid == 0) {
+    for (int s = 0; s < STAGES && s < ntiles; ++s) {
+      const int64_t keys = min64(TK, n1 - n0 - (int64_t)s * TK);
+      const uint32_t bytes = (uint32_t)(keys * DI);
+      mbar_arrive_expect_tx(&full_bar[s], bytes);
+      bulk_g2s(smem_tiles + s * S::TILE_BYTES, src + (int64_t)s * TK * DI, bytes, &full_bar[s]);
+    }
+  }
+
+  int abort_it = -1;
+  for (int it = 0; it < ntiles; ++it) {
+    const int s = it % STAGES;
+    const bool ok = mbar_wait_bounded(&full_bar[s], (uint32_t)(it / STAGES) & 1u);
+    if (__syncthreads_or(!ok)) {
+      abort_it = it;
+      break;
+    }
+    if (tid == 0 && it >= 1 && it - 1 + STAGES < ntiles) {
+      const int nt = it - 1 + STAGES, ps = (it - 1) % STAGES;
+      const int64_t keys = min64(TK, n1 - n0 - (int64_t)nt * TK);
+      const uint32_t bytes = (uint32_t)(keys * DI);
+      asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+      mbar_arrive_expect_tx(&full_bar[ps], bytes);
+      bulk_g2s(smem_tiles + ps * S::TILE_BYTES, src + (int64_t)nt * TK * DI, bytes,
+               &full_bar[ps]);
+    }
+    const unsigned char *tile = smem_tiles + s * S::TILE_BYTES;
+    const int64_t tbase = n0 + (int64_t)it * TK;
+    const int tkeys = (int)min64(TK, n1 - tbase);
+    for (int sub = warp; sub < S::SUB; sub += S::THREADS / 32) {
+      const int kb = sub * 16;  // first key of these 16 in the tile
+      if (kb >= tkeys) break;   // warp-uniform
+      // A fragments (keys kb..kb+15 x 32 bytes per k-step): matrix m = lane / 8
+      // of ldmatrix.x4 holds rows (m & 1) * 8 + 0..7, bytes (m >> 1) * 16 + 0..15
+      uint32_t a[KS][4];
+      const unsigned char *arow = tile + (kb + (lane & 7) + ((lane >> 3) & 1) * 8) * DI + (lane >> 4) * 16;
+#pragma unroll
+      for (int k = 0; k < KS; ++k)
+        asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0, %1, %2, %3}, [%4];"
+                     : "=r"(a[k][0]), "=r"(a[k][1]), "=r"(a[k][2]), "=r"(a[k][3])
+                     : "r"(smem_u32(arow + 32 * k)));
+      const int kk = kb + gid + (odd ? 8 : 0);  // this lane's key in the tile
+      const int64_t n = tbase + kk;
+#pragma unroll
+      for (int u = 0; u < NT; ++u) {
+        int c[4] = {0, 0, 0, 0};
+#pragma unroll
+        for (int k = 0; k < KS; ++k) mma_s8_16832(c, a[k], bq[u][k][0], bq[u][k][1]);
+        // even lane: key gid, its heads 0,1 + the partner's heads 2,3 of key
+        // gid; odd lane: key gid + 8, the partner's heads 0,1 + its 2,3
+        const int x0 = __shfl_xor_sync(0xffffffffu, odd ? c[0] : c[2], 1);
+        const int x1 = __shfl_xor_sync(0xffffffffu, odd ? c[1] : c[3], 1);
+        const int d0 = odd ? x0 : c[0], d1 = odd ? x1 : c[1];
+        const int d2 = odd ? c[2] : x0, d3 = odd ? c[3] : x1;
+        const int tq = 2 * u + (tig >> 1);
+        if (tq < T && kk < tkeys && n < vq[u]) {
+          float acc = 0.0f;
+          acc = __fadd_rn(acc, __fmul_rn(wt[u][0], __int2float_rn(d0)));
+          acc = __fadd_rn(acc, __fmul_rn(wt[u][1], __int2float_rn(d1)));
+          acc = __fadd_rn(acc, __fmul_rn(wt[u][2], __int2float_rn(d2)));
+          acc = __fadd_rn(acc, __fmul_rn(wt[u][3], __int2float_rn(d3)));
+          const float score = __fadd_rn(acc, 0.0f);
+          scores[(rl0 + tq) * score_stride + n] = score;
+          atomicAdd(&sh_hist[tq * kBins1 + key_d1(score_key(score))], 1u);
+        }
+      }
+    }
+  }
+  if (abort_it >= 0) {
+    if (tid == 0) {
+      const int upto = min(ntiles, max(abort_it - 1, 0) + STAGES);
+      for (int k = 0; k < STAGES && k < upto; ++k) {
+        const int last = k + ((upto - 1 - k) / STAGES) * STAGES;
+        mbar_wait_bounded(&full_bar[k], (uint32_t)(last / STAGES) & 1u);
+      }
+    }
+    __syncthreads();
+    return;
+  }
+  // entries a row may not see: -inf when scores are requested
+  if (write_masked && n_prior >= 0) {
+    for (int tt = 0; tt < T; ++tt) {
+      int64_t Vt = n_prior + (int64_t)(tt + 1) / ratio;
+      if (Vt > N) Vt = N;
+      const int64_t m0 = Vt + ((N - Vt) * g) / G, m1 = Vt + ((N - Vt) * (g + 1)) / G;
+      float *srow = scores + (rl0 + tt) * score_stride;
+      for (int64_t m = m0 + tid; m < m1; m += S::THREADS) srow[m] = -__int_as_float(0x7f800000);
+    }
+  }
+  __syncthreads();
+  for (int tt = 0; tt < T; ++tt) {
+    uint32_t *grow = hist1 + (rl0 + tt) * kHistStride;
+    for (int i = tid; i < kBins1; i += S::THREADS) {
+      const uint32_t v = sh_hist[tt * kBins1 + i];
+      if (v) atomicAdd(grow + i, v);
+    }
+  }
+}
+
+}  // namespace csa2

@@ -271,6 +271,28 @@ def test_multi_query_shared_scan(T, d_I, H_I):
     _check_index(q, w, k, 300, check_scores=False)
 
 
+@pytest.mark.parametrize("T,d_I,N,topk", [(4, 32, 1, 1), (6, 64, 15, 20), (7, 32, 17, 16),
+                                           (4, 64, 300, 64), (8, 32, 4097, 512),
+                                           (3, 64, 131, 131), (2, 32, 257, 300)])
+def test_multi_query_tensor_core_scan_edges(T, d_I, N, topk):
+    """The tensor-core multi-token scan (4 index heads): fewer keys than one
+    16-key block, a ragged last block and tile, k >= N, every token count
+    of the three n-tile widths; scores and indices bit-exact."""
+    q, w, k = _index_case(2, T, 4, d_I, N, seed=T * 1000 + N)
+    _check_index(q, w, k, topk)
+
+
+def test_multi_query_tensor_core_scan_extreme_values():
+    """Index queries and keys at the int8 extremes (dots up to 64 x 127 x 128
+    in one int32 accumulator) and negative weights."""
+    q, w, k = _index_case(2, 5, 4, 64, 5000, seed=5)
+    q[0] = -128
+    k[0, ::2] = -128
+    k[0, 1::2] = 127
+    w[1] = -np.abs(w[1])
+    _check_index(q, w, k, 700)
+
+
 def test_multi_query_shared_scan_visibility():
     B, T, n_prior, ratio = 2, 7, 5000, 2         # each row sees a different prefix
     N = n_prior + T // ratio
