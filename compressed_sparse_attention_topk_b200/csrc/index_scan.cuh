@@ -543,12 +543,16 @@ __global__ void __launch_bounds__(256, 2)
       bq[u][k][1] = tq < T ? *reinterpret_cast<const uint32_t *>(qr + 32 * k + 16 + 4 * tig) : 0u;
     }
   }
-  // this lane's token in n-tile u, its weights and its visible count
+  // this lane's token in n-tile u: its weights, visible count (0 past the
+  // last token), score row and histogram
   float wt[NT][4];
   int64_t vq[NT];
+  float *srow[NT];
+  uint32_t *hrow[NT];
 #pragma unroll
   for (int u = 0; u < NT; ++u) {
     const int tq = 2 * u + (tig >> 1);
+    const int tc = tq < T ? tq : 0;
 #pragma unroll
     for (int h = 0; h < 4; ++h) wt[u][h] = tq < T ? w[(b * T + tq) * 4 + h] : 0.0f;
     int64_t v = tq < T ? N : 0;
@@ -557,6 +561,8 @@ __global__ void __launch_bounds__(256, 2)
       if (v > N) v = N;
     }
     vq[u] = v;
+    srow[u] = scores + (rl0 + tc) * score_stride;
+    hrow[u] = sh_hist + tc * kBins1;
   }
   __syncthreads();
   if (tid == 0) {
@@ -588,9 +594,19 @@ __global__ void __launch_bounds__(256, 2)
     const unsigned char *tile = smem_tiles + s * S::TILE_BYTES;
     const int64_t tbase = n0 + (int64_t)it * TK;
     const int tkeys = (int)min64(TK, n1 - tbase);
-    for (int sub = warp; sub < S::SUB; sub += S::THREADS / 32) {
-      const int kb = sub * 16;  // first key of these 16 in the tile
-      if (kb >= tkeys) break;   // warp-uniform
+    // per n-tile: this lane's keys of the tile that its token sees
+    int lim[NT];
+    float *sp[NT];
+#pragma unroll
+    for (int u = 0; u < NT; ++u) {
+      const int64_t rem = vq[u] - tbase;
+      lim[u] = (int)min64(tkeys, rem > 0 ? rem : 0);
+      sp[u] = srow[u] + tbase;
+    }
+#pragma unroll
+    for (int i = 0; i < S::SUB / (S::THREADS / 32); ++i) {
+      const int kb = (warp + i * (S::THREADS / 32)) * 16;  // first key of these 16 in the tile
+      if (kb >= tkeys) break;                              // warp-uniform
       // A fragments (keys kb..kb+15 x 32 bytes per k-step): matrix m = lane / 8
       // of ldmatrix.x4 holds rows (m & 1) * 8 + 0..7, bytes (m >> 1) * 16 + 0..15
       uint32_t a[KS][4];
@@ -601,7 +617,6 @@ __global__ void __launch_bounds__(256, 2)
                      : "=r"(a[k][0]), "=r"(a[k][1]), "=r"(a[k][2]), "=r"(a[k][3])
                      : "r"(smem_u32(arow + 32 * k)));
       const int kk = kb + gid + (odd ? 8 : 0);  // this lane's key in the tile
-      const int64_t n = tbase + kk;
 #pragma unroll
       for (int u = 0; u < NT; ++u) {
         int c[4] = {0, 0, 0, 0};
@@ -613,16 +628,15 @@ __global__ void __launch_bounds__(256, 2)
         const int x1 = __shfl_xor_sync(0xffffffffu, odd ? c[1] : c[3], 1);
         const int d0 = odd ? x0 : c[0], d1 = odd ? x1 : c[1];
         const int d2 = odd ? c[2] : x0, d3 = odd ? c[3] : x1;
-        const int tq = 2 * u + (tig >> 1);
-        if (tq < T && kk < tkeys && n < vq[u]) {
+        if (kk < lim[u]) {
           float acc = 0.0f;
           acc = __fadd_rn(acc, __fmul_rn(wt[u][0], __int2float_rn(d0)));
           acc = __fadd_rn(acc, __fmul_rn(wt[u][1], __int2float_rn(d1)));
           acc = __fadd_rn(acc, __fmul_rn(wt[u][2], __int2float_rn(d2)));
           acc = __fadd_rn(acc, __fmul_rn(wt[u][3], __int2float_rn(d3)));
           const float score = __fadd_rn(acc, 0.0f);
-          scores[(rl0 + tq) * score_stride + n] = score;
-          atomicAdd(&sh_hist[tq * kBins1 + key_d1(score_key(score))], 1u);
+          sp[u][kk] = score;
+          atomicAdd(&hrow[u][key_d1(score_key(score))], 1u);
         }
       }
     }
