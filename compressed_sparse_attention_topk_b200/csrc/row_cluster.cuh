@@ -496,33 +496,6 @@ __device__ __forceinline__ void issue_window_rows(ar::WarpArea<D> &wa, const uin
   ar::cp_commit();
 }
 
-// The window warp's part of a head pass: attention over this CTA's window
-// rows in chunks of 16 (the first chunk's copies already issued when
-// `first_issued`), then its state into the window area's merge slot.
-template <int D, int CL>
-__device__ void row_window_partial(RowSmem<D> &sm, const RowParams &p, int64_t r, int c,
-                                   bool first_issued) {
-  int64_t wrow0;
-  int nwin;
-  window_share<CL>(p, r, c, wrow0, nwin);
-  ar::WarpState<D> st;
-  ar::state_init(st);
-  for (int j0 = 0; j0 < nwin; j0 += ar::kChunk) {
-    const int n = min(ar::kChunk, nwin - j0);
-    uint32_t mask;
-    if (j0 == 0 && first_issued) {
-      ar::cp_wait<0>();
-      __syncwarp();
-      mask = (1u << n) - 1u;
-    } else {
-      mask = ar::load_window_rows<D>(sm.win, p.win_k, p.win_v, wrow0 + j0, n);
-    }
-    ar::attend_chunk16<D>(sm.win, sm.qb, st, mask, true, nullptr, p.q_scale);
-    __syncwarp();
-  }
-  ar::store_state<D>(sm.win, st);
-}
-
 // ---------------------------------------------------------------------------
 // Attention on tensor cores (mma.sync m16n8k16, bf16 x bf16 -> fp32).
 // ---------------------------------------------------------------------------
@@ -559,10 +532,17 @@ __device__ void row_attend(RowSmem<D> &sm, const RowParams &p, cg::cluster_group
   const uint8_t *cseq = p.codes + b * p.N * (D / 2);
   const float *sseq = p.scales + b * p.N * (D / 16);
   __syncthreads();  // top-k buffers dead, query in place
-  if (warp < kAttnWarps) {
-    ar::WarpArea<D> &wa = sm.u.aw[warp];
+  const bool win_warp = warp == kWinWarp;
+  if (warp < kAttnWarps || (win_warp && has_win)) {
+    // The entry warps and the window warp run one loop with one copy of the
+    // chunk body (window or entry chunk chosen at run time), so an SM
+    // fetches that code once.
+    ar::WarpArea<D> &wa = win_warp ? sm.win : sm.u.aw[warp];
     ar::WarpState<D> st;
     ar::state_init(st);
+    int64_t wrow0 = 0;
+    int nwin = 0;
+    if (win_warp) window_share<CL>(p, r, c, wrow0, nwin);
     auto entry_of = [&](int64_t ch) -> int32_t {  // this lane's key of entry chunk ch
       const int64_t k = ch * ar::kChunk + (lane & 15);
       if (k >= nsel) return -1;
@@ -572,30 +552,51 @@ __device__ void row_attend(RowSmem<D> &sm, const RowParams &p, cg::cluster_group
       }
       return (lo + k < p.topk) ? irow[lo + k] : -1;
     };
-    int64_t ech = warp;
+    int64_t ech = win_warp ? nch : warp;  // the window warp takes no entry chunk
     uint32_t mask_cur = 0u;
     if (ech < nch) mask_cur = ar::gather_entries<D>(wa, 0, entry_of(ech), p.N, cseq, sseq);
-    // entry chunks, the next one gathered while the current one is used
-    for (int it = 0; ech < nch; ++it, ech += kAttnWarps) {
-      const int sb = it & 1;
-      uint32_t mask_next = 0u;
-      const bool more = ech + kAttnWarps < nch;
-      if (more) mask_next = ar::gather_entries<D>(wa, sb ^ 1, entry_of(ech + kAttnWarps), p.N, cseq, sseq);
-      if (more)
-        ar::cp_wait<1>();
-      else
-        ar::cp_wait<0>();
+    int wj = 0;  // the window warp's next row
+    int ei = 0;  // entry chunks done
+#pragma unroll 1
+    for (;;) {
+      const bool is_win = wj < nwin;
+      uint32_t mask;
+      int sb = 0;
+      if (is_win) {
+        const int n = min(ar::kChunk, nwin - wj);
+        if (wj == 0 && win_issued) {  // the first chunk's copies were issued early
+          ar::cp_wait<0>();
+          __syncwarp();
+          mask = (1u << n) - 1u;
+        } else {
+          mask = ar::load_window_rows<D>(wa, p.win_k, p.win_v, wrow0 + wj, n);
+        }
+        wj += ar::kChunk;
+      } else {
+        if (ech >= nch) break;
+        // entry chunk ech in buffer sb, the next one gathered meanwhile
+        sb = ei & 1;
+        uint32_t mask_next = 0u;
+        const bool more = ech + kAttnWarps < nch;
+        if (more)
+          mask_next = ar::gather_entries<D>(wa, sb ^ 1, entry_of(ech + kAttnWarps), p.N, cseq, sseq);
+        if (more)
+          ar::cp_wait<1>();
+        else
+          ar::cp_wait<0>();
+        __syncwarp();
+        ar::convert_entries<D>(wa, sb);
+        __syncwarp();
+        mask = mask_cur;
+        mask_cur = mask_next;
+        ech += kAttnWarps;
+        ++ei;
+      }
+      ar::attend_chunk16<D>(wa, sm.qb, st, mask, is_win, wa.s.scales[sb], p.q_scale);
       __syncwarp();
-      ar::convert_entries<D>(wa, sb);
-      __syncwarp();
-      ar::attend_chunk16<D>(wa, sm.qb, st, mask_cur, false, wa.s.scales[sb], p.q_scale);
-      __syncwarp();
-      mask_cur = mask_next;
     }
     ar::store_state<D>(wa, st);
-  } else if (warp == kWinWarp) {
-    if (has_win) row_window_partial<D, CL>(sm, p, r, c, win_issued);
-  } else if (idx_pending) {
+  } else if (!win_warp && idx_pending) {
     write_row_indices<D, CL>(sm, p, r, c, K);
   }
   __syncthreads();
