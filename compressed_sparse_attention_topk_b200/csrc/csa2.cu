@@ -355,45 +355,60 @@ csa2_status launch_row_cl(const RowParams &p, int64_t nr, cudaStream_t st) {
              : CSA2_ERR_CUDA;
 }
 
-// Can clusters of 16 CTAs of the row kernel be scheduled on this device?
-template <int D>
-bool cluster16_ok() {
-  static std::atomic<int> cache[256];  // per device: 0 unknown, 1 yes, 2 no
-  int dev = 0;
-  cudaGetDevice(&dev);
-  if (dev >= 0 && dev < 256 && cache[dev].load(std::memory_order_relaxed))
-    return cache[dev].load(std::memory_order_relaxed) == 1;
-  const size_t smem = sizeof(RowSmem<D>);
-  bool ok = set_smem_attr(row_cluster_kernel<D, 16, false>, smem, true) == CSA2_OK;
-  if (ok) {
-    cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3(16, 1, 1);
-    cfg.blockDim = dim3(kRowThreads, 1, 1);
-    cfg.dynamicSmemBytes = smem;
-    cudaLaunchAttribute attr[1];
-    attr[0].id = cudaLaunchAttributeClusterDimension;
-    attr[0].val.clusterDim.x = 16;
-    attr[0].val.clusterDim.y = 1;
-    attr[0].val.clusterDim.z = 1;
-    cfg.attrs = attr;
-    cfg.numAttrs = 1;
-    int n = 0;
-    ok = cudaOccupancyMaxActiveClusters(&n, row_cluster_kernel<D, 16, false>, &cfg) ==
-             cudaSuccess &&
-         n > 0;
+// Clusters of cl CTAs of `kernel` (threads per CTA, dynamic shared memory
+// smem) that this device can hold at once; 0 when none can be launched.
+template <class K>
+int max_active_clusters(K kernel, int cl, int threads, size_t smem) {
+  if (set_smem_attr(kernel, smem, cl > 8) != CSA2_OK) {
+    cudaGetLastError();
+    return 0;
   }
-  cudaGetLastError();
-  if (dev >= 0 && dev < 256) cache[dev].store(ok ? 1 : 2, std::memory_order_relaxed);
-  return ok;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3((unsigned)cl, 1, 1);
+  cfg.blockDim = dim3((unsigned)threads, 1, 1);
+  cfg.dynamicSmemBytes = smem;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = (unsigned)cl;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  int n = 0;
+  if (cudaOccupancyMaxActiveClusters(&n, kernel, &cfg) != cudaSuccess) {
+    cudaGetLastError();
+    return 0;
+  }
+  return n;
 }
 
-// Rows of one launch -> CTAs per row: as many as keep about two CTAs per SM.
+// The row kernel's resident clusters of CL CTAs (cached per device).
+template <int D, int CL>
+int row_clusters_resident() {
+  static std::atomic<int> cache[256];  // per device: 0 unknown, else count + 1
+  int dev = 0;
+  cudaGetDevice(&dev);
+  if (dev >= 0 && dev < 256) {
+    const int c = cache[dev].load(std::memory_order_relaxed);
+    if (c) return c - 1;
+  }
+  const int n = max_active_clusters(row_cluster_kernel<D, CL, false>, CL, kRowThreads,
+                                    sizeof(RowSmem<D>));
+  if (dev >= 0 && dev < 256) cache[dev].store(n + 1, std::memory_order_relaxed);
+  return n;
+}
+
+// Rows of one launch -> CTAs per row: the largest cluster (16, 8 or 4 CTAs)
+// whose clusters for all nr rows the device holds at once, so that no row's
+// cluster waits for another's to finish (4 when neither fits).  A second
+// wave costs a whole selection: 32 decode rows take 80 us per step in
+// clusters of 8 (256 CTAs for 148 SMs) and 68 us in clusters of 4.
 int row_cluster_size(int64_t nr, int D) {
-  const int64_t target = 2 * int64_t(device_sms());
-  int cl = 4;
-  if (nr * 8 <= target) cl = 8;
-  if (nr * 16 <= target && (D == 128 ? cluster16_ok<128>() : cluster16_ok<64>())) cl = 16;
-  return cl;
+  if (nr <= (D == 128 ? row_clusters_resident<128, 16>() : row_clusters_resident<64, 16>()))
+    return 16;
+  if (nr <= (D == 128 ? row_clusters_resident<128, 8>() : row_clusters_resident<64, 8>()))
+    return 8;
+  return 4;
 }
 
 csa2_status launch_row(const RowParams &p, int D, int64_t nr, cudaStream_t st) {
@@ -449,48 +464,35 @@ csa2_status launch_attn_cl(const ar::Params &a, int64_t nr, bool after_topk, cud
              : CSA2_ERR_CUDA;
 }
 
-// Can clusters of 16 CTAs of the attention kernel be scheduled on this device?
-template <int D>
-bool attn_cluster16_ok() {
-  static std::atomic<int> cache[256];  // per device: 0 unknown, 1 yes, 2 no
+// The attention cluster kernel's resident clusters of CL CTAs (cached per
+// device).
+template <int D, int CL>
+int attn_clusters_resident() {
+  static std::atomic<int> cache[256];  // per device: 0 unknown, else count + 1
   int dev = 0;
   cudaGetDevice(&dev);
-  if (dev >= 0 && dev < 256 && cache[dev].load(std::memory_order_relaxed))
-    return cache[dev].load(std::memory_order_relaxed) == 1;
-  const size_t smem = sizeof(ac::Smem<D, 16>);
-  bool ok = set_smem_attr(ac::attn_cluster_kernel<D, 16>, smem, true) == CSA2_OK;
-  if (ok) {
-    cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3(16, 1, 1);
-    cfg.blockDim = dim3(ac::kThreads, 1, 1);
-    cfg.dynamicSmemBytes = smem;
-    cudaLaunchAttribute attr[1];
-    attr[0].id = cudaLaunchAttributeClusterDimension;
-    attr[0].val.clusterDim.x = 16;
-    attr[0].val.clusterDim.y = 1;
-    attr[0].val.clusterDim.z = 1;
-    cfg.attrs = attr;
-    cfg.numAttrs = 1;
-    int n = 0;
-    ok = cudaOccupancyMaxActiveClusters(&n, ac::attn_cluster_kernel<D, 16>, &cfg) == cudaSuccess &&
-         n > 0;
+  if (dev >= 0 && dev < 256) {
+    const int c = cache[dev].load(std::memory_order_relaxed);
+    if (c) return c - 1;
   }
-  cudaGetLastError();
-  if (dev >= 0 && dev < 256) cache[dev].store(ok ? 1 : 2, std::memory_order_relaxed);
-  return ok;
+  const int n = max_active_clusters(ac::attn_cluster_kernel<D, CL>, CL, ac::kThreads,
+                                    sizeof(ac::Smem<D, CL>));
+  if (dev >= 0 && dev < 256) cache[dev].store(n + 1, std::memory_order_relaxed);
+  return n;
 }
 
 // Attention of nr decode rows (a.row0 ...): CTAs per row as for the
-// selection (about two CTAs per SM in total); after_topk: launched right
+// selection; after_topk: launched right
 // after the selection of the same rows, with programmatic dependent launch.
 csa2_status launch_attn_cluster(const ar::Params &a, int D, int64_t nr, bool after_topk,
                                 cudaStream_t st) {
   TraceScope ts("attend", st);
-  const int64_t target = 2 * int64_t(device_sms());
+  // the largest cluster whose clusters for all the rows are resident at once
   int cl = 4;
-  if (nr * 8 <= target) cl = 8;
-  if (nr * 16 <= target && (D == 128 ? attn_cluster16_ok<128>() : attn_cluster16_ok<64>()))
+  if (nr <= (D == 128 ? attn_clusters_resident<128, 16>() : attn_clusters_resident<64, 16>()))
     cl = 16;
+  else if (nr <= (D == 128 ? attn_clusters_resident<128, 8>() : attn_clusters_resident<64, 8>()))
+    cl = 8;
   if (D == 128) {
     if (cl == 16) return launch_attn_cl<128, 16>(a, nr, after_topk, st);
     if (cl == 8) return launch_attn_cl<128, 8>(a, nr, after_topk, st);
